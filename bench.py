@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the intra-expert sparse MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mixtral_decode] [--sparsity 0.7]
+
+A step is one pass of the whole layer (router, permute, fused gate+up with
+SwiGLU/threshold/compaction, union scan, sparse down projection, combine)
+over each decode batch of the workload; for the Mixtral-8x7B-shaped layer
+(bf16, d_model 4096, 8 experts top-2, d_ff 14336) that is the batches
+T = 1, 8, 32, 64 (105 tokens per step). The metric is MoE-layer tokens/s,
+measured on the device with CUDA events between a barrier and a
+synchronize on both sides, max over ranks. The touched experts' weights
+(>= 470 MB per forward) are larger than L2, so no flush is needed.
+
+The same steps are run on the library's own dense path (no threshold, every
+W_down row read) for the speedup, end to end through the Python API with
+host buffers (e2e), and, on rank 0 at N=1, through the CPU oracle on the
+host cores (cpu_baseline). ``--impl reference`` times only the oracle.
+Multi-GPU runs are weak-scaling replicas: every rank runs the full workload
+on its own GPU and copy of the weights; the path has no exchange step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from moe_inputs import WORKLOADS, make_tokens, make_weights  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and effective HBM GB/s vs own dense path, 0-90% sparsity"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="mixtral_decode")
+    ap.add_argument("--sparsity", type=float, default=0.7)
+    ap.add_argument("--tokens", type=str, default="", help="comma list overriding the batches")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_tau(workload: str, q: float):
+    with open(os.path.join(ROOT, "tests", "golden", "tau_calibration.json")) as f:
+        e = json.load(f)[workload]["taus"][f"{q:.2f}"]
+    return e["tau"], e.get("tau_shared", 0.0), e["measured_sparsity"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float, local: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=f"cuda:{local}")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_step_time(wl, tokens, tau, tau_s, w_host):
+    from oracle import moe_oracle as om
+    sh = wl.shape
+    t0 = time.perf_counter()
+    for T in tokens:
+        x = make_tokens(sh.d_model, T, wl.token_seed, sh.dtype)
+        om.layer_forward(x, w_host.W_router, w_host.W_gate, w_host.W_up, w_host.W_down, tau,
+                         sh.top_k, sh.renormalize, router_bias=w_host.router_bias,
+                         Ws_gate=w_host.Ws_gate, Ws_up=w_host.Ws_up, Ws_down=w_host.Ws_down,
+                         tau_shared=tau_s)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    tau, tau_s, _ = load_tau(args.workload, args.sparsity)
+    w = make_weights(wl.shape, wl.weight_seed)
+    sample = [8] if 8 in wl.tokens else [min(wl.tokens)]
+    for _ in range(args.warmup):
+        oracle_step_time(wl, sample, tau, tau_s, w)
+    t = sum(oracle_step_time(wl, sample, tau, tau_s, w) for _ in range(args.steps))
+    toks = sum(sample) * args.steps
+    cores = len(os.sched_getaffinity(0))
+    value = toks / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "batches": sample, "target_sparsity": args.sparsity,
+                   "tau": tau},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"decode batch T={sample} of {args.workload} per step "
+                                   f"(fp64 numpy oracle on {cores} host threads)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, world, rank, local):
+    from intra_expert_activation_b200 import MoESparseLayer
+
+    dev = torch.device("cuda", local)
+    wl = WORKLOADS[args.workload]
+    sh = wl.shape
+    tokens = [int(t) for t in args.tokens.split(",")] if args.tokens else list(wl.tokens)
+    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity)
+    w_host = make_weights(sh, wl.weight_seed)
+    mv = lambda t: None if t is None else t.to(dev).contiguous()
+    W = {k: mv(getattr(w_host, k)) for k in ("W_router", "W_gate", "W_up", "W_down",
+                                             "router_bias", "Ws_gate", "Ws_up", "Ws_down")}
+    xs_host = [make_tokens(sh.d_model, T, wl.token_seed, sh.dtype) for T in tokens]
+    xs = [x.to(dev) for x in xs_host]
+    outs = [torch.empty((T, sh.d_model), dtype=x.dtype, device=dev) for T, x in zip(tokens, xs)]
+    tmax = max(tokens)
+    esize = 2 if sh.dtype == "bf16" else 4
+
+    def make(path):
+        L = MoESparseLayer(sh.d_model, sh.d_ff, sh.n_experts, sh.top_k, tmax,
+                           renormalize=sh.renormalize, n_shared=sh.n_shared,
+                           d_ff_shared=sh.d_ff_shared, dtype=sh.dtype, path=path, device=local)
+        if sh.n_shared:
+            L.set_shared(W["Ws_gate"], W["Ws_up"], W["Ws_down"], tau_s)
+        return L
+
+    def step(L, out_list=outs, x_list=xs):
+        for x, o in zip(x_list, out_list):
+            L.forward(x, W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau, sh.top_k,
+                      router_bias=W["router_bias"], out=o)
+
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(L, ring):
+        for _ in range(args.warmup):
+            step(L)
+        L.set_timing(ring)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        n0 = L.launch_count()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(L)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ms = e0.elapsed_time(e1)
+        launches = L.launch_count() - n0
+        per = L.timing_all(ring) if ring else []
+        L.set_timing(0)
+        return ms, launches, per
+
+    sparse = make("auto")
+    clocks = Clocks(local)
+    ms_sparse, launches, per_fwd = timed(sparse, args.steps * len(tokens))
+    clk = clocks.stop()
+    ms_sparse = max_over_ranks(world, ms_sparse, local)
+    tok_step = sum(tokens)
+    value = tok_step * args.steps * world / (ms_sparse / 1e3)
+
+    # per-batch statistics of the sparse path (one extra forward each, untimed)
+    stats = []
+    for x, o in zip(xs, outs):
+        sparse.forward(x, W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau, sh.top_k,
+                       router_bias=W["router_bias"], out=o)
+        stats.append(sparse.stats())
+    assert sparse.status() == 0, "device status word set"
+
+    dense_line = None
+    per_dense = []
+    if not args.no_dense:
+        dense = make("dense")
+        ms_dense, _, per_dense = timed(dense, args.steps * len(tokens))
+        ms_dense = max_over_ranks(world, ms_dense, local)
+        dense_line = {"value": tok_step * args.steps * world / (ms_dense / 1e3),
+                      "ms_per_step": ms_dense / args.steps}
+        dense.close()
+
+    # per-kernel times, grouped by batch (forwards cycle through `tokens`)
+    nb = len(tokens)
+    def avg_stage(per, i, stage):
+        v = [f[stage] for j, f in enumerate(per) if j % nb == i]
+        return sum(v) / len(v) if v else 0.0
+
+    per_T = []
+    gate_bytes_tot = gate_ms_tot = down_bytes_tot = down_ms_tot = 0.0
+    for i, T in enumerate(tokens):
+        st = stats[i]
+        P = T * sh.top_k
+        touched = st["n_experts_touched"]
+        g_bytes = touched * 2 * sh.d_ff * sh.d_model * esize + P * sh.d_model * esize \
+            + P * sh.d_ff * esize
+        if sh.n_shared:
+            g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
+        d_bytes = st["down_rows_read"] * sh.d_model * esize
+        g_ms = avg_stage(per_fwd, i, "gate_up")
+        d_ms = avg_stage(per_fwd, i, "down_gemv") + avg_stage(per_fwd, i, "down_tc")
+        fwd_ms = sum(avg_stage(per_fwd, i, s) for s in per_fwd[0]) if per_fwd else 0.0
+        fwd_dense = sum(avg_stage(per_dense, i, s) for s in per_dense[0]) if per_dense else None
+        d_dense = (avg_stage(per_dense, i, "down_gemv") + avg_stage(per_dense, i, "down_tc")) \
+            if per_dense else None
+        gate_bytes_tot += g_bytes * args.steps
+        gate_ms_tot += g_ms * args.steps
+        down_bytes_tot += d_bytes * args.steps
+        down_ms_tot += d_ms * args.steps
+        sp = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
+        per_T.append({
+            "T": T, "sparsity": round(sp, 4), "experts_touched": touched,
+            "down_rows_read": st["down_rows_read"],
+            "down_rows_dense": touched * sh.d_ff,
+            "groups": {"gemv": st["n_groups_gemv"], "tc_gather": st["n_groups_tc_gather"],
+                       "tc_allrows": st["n_groups_tc_allrows"]},
+            "stage_us": {k: round(1e3 * avg_stage(per_fwd, i, k), 2) for k in
+                         (per_fwd[0] if per_fwd else {})},
+            "layer_us": round(1e3 * fwd_ms, 2),
+            "dense_layer_us": None if fwd_dense is None else round(1e3 * fwd_dense, 2),
+            "speedup_vs_dense": None if not fwd_dense else round(fwd_dense / fwd_ms, 3),
+            "gate_up_GBps": round(g_bytes / (g_ms * 1e-3) / 1e9, 1) if g_ms else None,
+            "down_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1) if d_ms else None,
+            "dense_down_us": None if d_dense is None else round(1e3 * d_dense, 2),
+        })
+
+    peak, peak_kind = peaks()
+    g_ach = gate_bytes_tot / (gate_ms_tot * 1e-3) / 1e9 if gate_ms_tot else 0.0
+    d_ach = down_bytes_tot / (down_ms_tot * 1e-3) / 1e9 if down_ms_tot else 0.0
+    steps_launches = launches
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        xs_pin = [x.pin_memory() for x in xs_host]
+        outs_pin = [torch.empty((T, sh.d_model), dtype=x.dtype).pin_memory()
+                    for T, x in zip(tokens, xs_host)]
+        xs_dev = [torch.empty_like(x, device=dev) for x in xs_host]
+
+        def e2e_step():
+            for xp, xd, o, op in zip(xs_pin, xs_dev, outs, outs_pin):
+                xd.copy_(xp, non_blocking=True)
+                sparse.forward(xd, W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau,
+                               sh.top_k, router_bias=W["router_bias"], out=o)
+                op.copy_(o, non_blocking=True)
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ms_e2e = max_over_ranks(world, a.elapsed_time(b), local)
+        nbytes = sum(x.numel() * x.element_size() for x in xs_host)
+        e2e = {"value": tok_step * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t = oracle_step_time(wl, tokens, tau, tau_s, w_host)
+        cores = len(os.sched_getaffinity(0))
+        cpu = {"value": tok_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"one step: decode batches T={tokens} of {args.workload} through the "
+                         f"fp64 numpy oracle on {cores} host threads ({t:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_sparse / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batches": tokens, "tokens_per_step": tok_step,
+                       "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
+                       "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
+                       "calibrated_sparsity": round(calib_sparsity, 4),
+                       "l2": "no flush: touched expert weights (>= 470 MB per forward) exceed L2",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"kernel": "gate_up_tc", "bound": "hbm", "achieved": round(g_ach, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(g_ach / peak, 4),
+                         "traffic": None, "peak_kind": peak_kind},
+            "roofline_down": {"kernel": "down (GEMV / TC, rows actually read)", "bound": "hbm",
+                              "achieved": round(d_ach, 1), "peak": peak, "unit": "GB/s",
+                              "frac": round(d_ach / peak, 4), "peak_kind": peak_kind},
+            "dense": dense_line,
+            "speedup_vs_dense": None if not dense_line else
+            round(dense_line["ms_per_step"] / (ms_sparse / args.steps), 4),
+            "per_T": per_T,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": steps_launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    sparse.close()
+    return 0
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init(args) if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,200 @@
+/*
+ * moe_sparse.h -- C ABI of a B200 (sm_100a) Mixture-of-Experts feed-forward
+ * layer that skips inactive neurons inside each routed expert.
+ *
+ * The operation, per batch of T tokens x[T][d_model]:
+ *
+ *   1. Router. logits = x W_router^T (+ router_bias), softmax over all E
+ *      experts, the top_k experts by probability (ties go to the lower
+ *      expert index), weights p_sel / sum(p_sel) when desc.renormalize,
+ *      else p_sel. The pages keep the dense model's router as it is
+ *      [gist.science EN "Uncovering Intra-expert Activation Sparsity for
+ *      Efficient Mixture-of-Expert Model Execution", Technical Summary >
+ *      Methodology > System Implementation in vLLM].
+ *   2. Dense gate and up projections of every routed (token, expert) pair
+ *      [same list, "Gate Projection": the gate projection runs densely to
+ *      produce the activation scores] and the SwiGLU value
+ *      h = SiLU(x W_gate[e]^T) * (x W_up[e]^T)
+ *      [mlsanity.com page, "Builds on": GLU Variants Improve Transformer].
+ *   3. Threshold mask in one pass, no sort: neuron j is active iff
+ *      |h_j| > tau; at or below tau it is inactive
+ *      [same list, "Activation Masking"]. The test is taken on the fp32 h
+ *      before any rounding.
+ *   4. Down projection that reads only the W_down rows of active neurons
+ *      [same list, "Fused Up-Down Projection": gather the active neurons'
+ *      weights, pack them densely, multiply densely]; y = sum_{j active}
+ *      h_j W_down[e][j, :].
+ *   5. Combine out[t] = sum_i w[t,i] y[t,i] + sum_s y_shared[s,t]; shared
+ *      experts are always active with weight 1 and their own threshold
+ *      [gist.science EN, Technical Summary > Methodology > "Empirical
+ *      Analysis": routed vs always-active shared experts].
+ *   The sparse/dense codepath choice by batch size [same list, "Dynamic
+ *   Switching"] is made per expert token group on the device from the
+ *   group's token count and the size of its active-row union.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are DEVICE pointers on desc.device, contiguous, row-major,
+ *     16-byte aligned, in desc.dtype (x, weights, out), except router_bias
+ *     (float32). The caller owns them; the library never frees them.
+ *       x         [T][d_model]
+ *       W_router  [n_experts][d_model]            logits = x W_router^T
+ *       W_gate    [n_experts][d_ff][d_model]      row j: neuron j's input weights
+ *       W_up      [n_experts][d_ff][d_model]
+ *       W_down    [n_experts][d_ff][d_model]      row j: neuron j's output vector
+ *       out       [T][d_model]
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - The context owns a device workspace sized at init for max_tokens and
+ *     top_k_max; moe_sparse_forward never allocates and never synchronises
+ *     the host.
+ *   - Argument errors return synchronously before any launch. Launch
+ *     errors return MOE_ERR_CUDA. Errors found by kernels (a bounded wait
+ *     that ran out) are recorded in a device status word read by
+ *     moe_sparse_get_status.
+ *   - One context serves one stream at a time.
+ *   - Shapes: d_model % 256 == 0 and d_ff % 128 == 0 for MOE_BF16;
+ *     d_model % 128 == 0 and d_ff % 32 == 0 for MOE_F32; 1 <= n_experts <= 256;
+ *     1 <= top_k <= min(n_experts, 16); 1 <= max_tokens <= 65536.
+ */
+#ifndef MOE_SPARSE_H
+#define MOE_SPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,        /* bad argument, null pointer, size out of range */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid but not implemented (shape, dtype, device) */
+  MOE_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
+  MOE_ERR_NOMEM = 4,          /* device allocation failed in init */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait ran out (status word) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+typedef enum {
+  MOE_PATH_AUTO = 0,          /* threshold on; per group: GEMV, gathered TC or all-rows TC */
+  MOE_PATH_DENSE = 1,         /* no threshold: every neuron active (the dense baseline) */
+  MOE_PATH_SPARSE_GEMV = 2,   /* threshold on; every group on the CUDA-core row stream */
+  MOE_PATH_SPARSE_TC = 3,     /* threshold on; gathered-row tensor-core path (groups <= 64 tokens) */
+  MOE_PATH_SPARSE_TC_ALLROWS = 4 /* threshold on; tensor cores over all rows with masked h */
+} moe_path;
+
+typedef struct {
+  int32_t d_model;
+  int32_t d_ff;
+  int32_t n_experts;
+  int32_t top_k_max;
+  int32_t max_tokens;
+  int32_t renormalize;        /* 1: w = p_sel / sum(p_sel); 0: w = p_sel */
+  int32_t n_shared;           /* always-on shared experts, 0..8 */
+  int32_t d_ff_shared;        /* their d_ff (same divisibility as d_ff); ignored if n_shared == 0 */
+  int32_t dtype;              /* moe_dtype */
+  int32_t path;               /* moe_path */
+  int32_t debug;              /* 1: keep per-pair active bitmaps for moe_sparse_get_debug */
+  int32_t device;             /* CUDA device ordinal */
+  int32_t gemv_max_tokens;    /* AUTO: groups with <= this many tokens use the GEMV path (0: 4) */
+  float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: 0.9) */
+} moe_sparse_desc;
+
+typedef struct {
+  int64_t n_routed_h;         /* routed (token, expert) pairs x d_ff: h values tested */
+  int64_t n_routed_active;    /* of those, |h| > tau */
+  int64_t n_shared_h;
+  int64_t n_shared_active;
+  int64_t down_rows_read;     /* W_down rows streamed by the down projection, all groups */
+  int64_t n_groups;           /* expert token groups (routed + shared) */
+  int64_t n_groups_gemv;
+  int64_t n_groups_tc_gather;
+  int64_t n_groups_tc_allrows;
+  int64_t n_experts_touched;  /* routed experts with at least one token */
+} moe_stats;
+
+typedef struct moe_sparse_ctx moe_sparse_ctx;
+
+/* Host-only check of a descriptor (no CUDA call). MOE_OK if init would accept it. */
+MOE_API moe_status moe_sparse_validate_desc(const moe_sparse_desc* desc);
+
+/* Device workspace bytes init allocates for desc (host-only, no CUDA call). */
+MOE_API moe_status moe_sparse_workspace_bytes(const moe_sparse_desc* desc, size_t* bytes);
+
+/* Create a context on desc->device: validates desc, allocates the workspace.
+ * On failure *ctx is NULL and nothing is left allocated. */
+MOE_API moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** ctx);
+
+/* Always-on shared experts (desc.n_shared > 0): W*_s are device pointers
+ * [n_shared][d_ff_shared][d_model] in desc.dtype, kept by pointer (the caller
+ * keeps them alive); tau_shared is their own threshold. Must be called
+ * before the first forward of a context with shared experts. */
+MOE_API moe_status moe_sparse_set_shared(moe_sparse_ctx* ctx, const void* Wg_s, const void* Wu_s,
+                                 const void* Wd_s, float tau_shared);
+
+/* One layer forward, steps 1-5 above, enqueued on stream. 0 <= T <= max_tokens
+ * (T == 0 launches nothing); 1 <= top_k <= top_k_max; router_bias may be NULL.
+ * tau is ignored by MOE_PATH_DENSE. out is fully overwritten. */
+MOE_API moe_status moe_sparse_forward(moe_sparse_ctx* ctx, const void* x, int32_t T,
+                              const void* W_router, const float* router_bias,
+                              const void* W_gate, const void* W_up, const void* W_down,
+                              float tau, int32_t top_k, void* out, void* stream);
+
+/* Routing and active sets of the last forward, in pair order p = t*top_k + i,
+ * copied into caller DEVICE buffers on stream (any pointer may be NULL):
+ *   topk_idx [T][top_k] int32, topk_w [T][top_k] float32,
+ *   active_bits [T*top_k][ceil(d_ff/32)] uint32 (bit j%32 of word j/32 = neuron j active;
+ *              needs desc.debug = 1),
+ *   active_bits_shared [n_shared][T][ceil(d_ff_shared/32)] (needs desc.debug = 1). */
+MOE_API moe_status moe_sparse_get_debug(moe_sparse_ctx* ctx, int32_t* topk_idx, float* topk_w,
+                                uint32_t* active_bits, uint32_t* active_bits_shared,
+                                void* stream);
+
+/* Counters of the last forward (synchronises stream, then copies to the host struct). */
+MOE_API moe_status moe_sparse_get_stats(moe_sparse_ctx* ctx, moe_stats* stats, void* stream);
+
+/* Reads and clears the device status word (synchronises the device).
+ * *device_err receives MOE_OK or MOE_ERR_DEVICE_TIMEOUT. */
+MOE_API moe_status moe_sparse_get_status(moe_sparse_ctx* ctx, int32_t* device_err);
+
+/* Per-stage timing of later forwards with CUDA events recorded on the
+ * forward's stream between its kernels. ring > 0 keeps event sets for the
+ * last `ring` forwards (at most 4096); 0 turns timing off. */
+MOE_API moe_status moe_sparse_set_timing(moe_sparse_ctx* ctx, int32_t ring);
+
+/* Milliseconds of each stage of the last timed forward (synchronises its
+ * events). Stages: 0 route, 1 permute, 2 gate_up, 3 union_scan, 4 down_gemv,
+ * 5 down_tc, 6 combine; a stage that launched nothing reports 0. */
+MOE_API moe_status moe_sparse_get_timing(moe_sparse_ctx* ctx, float* ms, int32_t n);
+
+/* Stage milliseconds of every timed forward since the last call, oldest
+ * first: ms[f * n_stages + s] for f < *n_forwards (at most max_forwards and
+ * at most the ring size; older ones are dropped). Synchronises the events and
+ * restarts the collection. */
+MOE_API moe_status moe_sparse_get_timing_all(moe_sparse_ctx* ctx, float* ms, int32_t n_stages,
+                                             int32_t max_forwards, int32_t* n_forwards);
+
+/* Kernels this context has launched since init (host-side count). */
+MOE_API moe_status moe_sparse_launch_count(const moe_sparse_ctx* ctx, int64_t* n);
+
+/* Name of stage i (static string), or NULL. */
+MOE_API const char* moe_sparse_stage_name(int32_t i);
+
+/* Last error message of ctx (or of the last failed init if ctx is NULL). */
+MOE_API const char* moe_sparse_last_error(const moe_sparse_ctx* ctx);
+
+/* Frees the workspace and the context. NULL is accepted. */
+MOE_API moe_status moe_sparse_destroy(moe_sparse_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_SPARSE_H */

@@ -1,0 +1,196 @@
+// Small kernels between the big ones:
+//  union_scan   per expert token group: compact the active-row union bitmap
+//               into an ordered row list, and choose the down-projection path
+//               from the group's token count and union size (the pages'
+//               sparse/dense switch by batch size [gist.science EN "Uncovering
+//               Intra-expert Activation Sparsity for Efficient
+//               Mixture-of-Expert Model Execution", Technical Summary >
+//               Methodology > System Implementation in vLLM > "Dynamic
+//               Switching"], taken per group on the device).
+//  combine      out[t] = sum_i w[t,i] * Y[slot(t,i)] + sum_s Y[shared slot(s,t)],
+//               in a fixed order.
+//  debug_gather routing and active bitmaps of the last forward in pair order.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kScanThreads = 256;
+
+__global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Workspace ws) {
+  const int g = blockIdx.x;
+  if (g >= __ldcg(ws.meta + kMetaGroups)) return;
+  const Group gr = ws.groups[g];
+  const bool shared = gr.expert >= dm.E;
+  const int F_e = shared ? dm.Fs : dm.F;
+  const int words = F_e / 32;
+  const uint32_t* bits = ws.union_bits + static_cast<size_t>(g) * dm.fw;
+  int* rows = ws.union_rows + static_cast<size_t>(g) * dm.F_max;
+
+  __shared__ int warp_tot[kScanThreads / 32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // word-ordered exclusive scan of popcounts, kScanThreads words per round
+  for (int w0 = 0; w0 < words; w0 += kScanThreads) {
+    const int w = w0 + threadIdx.x;
+    const uint32_t b = w < words ? __ldcg(bits + w) : 0u;
+    const int c = __popc(b);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int base = carry;
+    for (int i = 0; i < warp; ++i) base += warp_tot[i];
+    int pos = base + incl - c;
+    uint32_t bb = b;
+    while (bb) {
+      const int bit = __ffs(bb) - 1;
+      rows[pos++] = w * 32 + bit;
+      bb &= bb - 1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int tot = 0;
+      for (int i = 0; i < kScanThreads / 32; ++i) tot += warp_tot[i];
+      carry += tot;
+    }
+    __syncthreads();
+  }
+
+  if (threadIdx.x == 0) {
+    const int cnt = carry;
+    const int m = gr.m;
+    int path;
+    if (dm.no_tc || dm.mode == kModeGemv) {
+      path = kPathGemv;
+    } else if (dm.mode == kModeDense) {
+      path = m <= dm.gemv_max ? kPathGemv : kPathTcAll;
+    } else if (dm.mode == kModeTc) {
+      path = m <= kGatherMaxTokens ? kPathTcGather : kPathTcAll;
+    } else if (dm.mode == kModeTcAll) {
+      path = kPathTcAll;
+    } else {
+      if (m <= dm.gemv_max)
+        path = kPathGemv;
+      else if (m <= kGatherMaxTokens && cnt <= dm.gather_density * F_e)
+        path = kPathTcGather;
+      else
+        path = kPathTcAll;
+    }
+    ws.union_cnt[g] = cnt;
+    ws.group_path[g] = path;
+    const int li = atomicAdd(ws.meta + (path == kPathGemv ? kMetaGemvCount : kMetaTcCount), 1);
+    (path == kPathGemv ? ws.gemv_list : ws.tc_list)[li] = g;
+    atomicAdd(ws.counters + kCntDownRows,
+              static_cast<unsigned long long>(path == kPathTcAll ? F_e : cnt));
+    atomicAdd(ws.counters + (path == kPathGemv ? kCntGemv
+                             : path == kPathTcGather ? kCntTcGather : kCntTcAll), 1ull);
+  }
+}
+
+template <typename TX>
+__device__ __forceinline__ void store4(TX* p, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* p, float4 v) {
+  *reinterpret_cast<float4*>(p) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v) {
+  union { __nv_bfloat162 b[2]; uint2 u; } pk;
+  pk.b[0] = __floats2bfloat162_rn(v.x, v.y);
+  pk.b[1] = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) = pk.u;
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX* out) {
+  const int t = blockIdx.x;
+  const int d = dm.d, k = dm.k;
+  __shared__ int slot[16];
+  __shared__ float w[16];
+  if (threadIdx.x < k) {
+    slot[threadIdx.x] = ws.slot_of[t * k + threadIdx.x];
+    w[threadIdx.x] = ws.topk_w[t * k + threadIdx.x];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < k; ++i) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + static_cast<size_t>(slot[i]) * d + c));
+      acc.x = fmaf(w[i], v.x, acc.x);
+      acc.y = fmaf(w[i], v.y, acc.y);
+      acc.z = fmaf(w[i], v.z, acc.z);
+      acc.w = fmaf(w[i], v.w, acc.w);
+    }
+    for (int s = 0; s < dm.S; ++s) {
+      const size_t srow = static_cast<size_t>(dm.slots_routed + s * dm.T_pad + t);
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + srow * d + c));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    store4<TX>(out + static_cast<size_t>(t) * d + c, acc);
+  }
+}
+
+__global__ void debug_gather_kernel(Dims dm, Workspace ws, int32_t* topk_idx, float* topk_w,
+                                    uint32_t* bits, uint32_t* bits_shared) {
+  const int P = dm.T * dm.k;
+  const int fwr = (dm.F + 31) / 32, fws = (dm.Fs + 31) / 32;
+  const int stride = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += stride) {
+    if (topk_idx) topk_idx[i] = ws.topk_idx[i];
+    if (topk_w) topk_w[i] = ws.topk_w[i];
+  }
+  if (bits && ws.act_bits) {
+    for (long long i = blockIdx.x * blockDim.x + threadIdx.x; i < (long long)P * fwr; i += stride) {
+      const int p = static_cast<int>(i / fwr), w = static_cast<int>(i % fwr);
+      bits[i] = ws.act_bits[static_cast<size_t>(ws.slot_of[p]) * dm.fw + w];
+    }
+  }
+  if (bits_shared && ws.act_bits && dm.S > 0) {
+    const long long n = (long long)dm.S * dm.T * fws;
+    for (long long i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+      const int w = static_cast<int>(i % fws);
+      const long long st = i / fws;
+      const int t = static_cast<int>(st % dm.T), s = static_cast<int>(st / dm.T);
+      const size_t slot = static_cast<size_t>(dm.slots_routed + s * dm.T_pad + t);
+      bits_shared[i] = ws.act_bits[slot * dm.fw + w];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st) {
+  union_scan_kernel<<<dm.groups_max, kScanThreads, 0, st>>>(dm, ws);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
+                           cudaStream_t st) {
+  const int threads = dm.d / 4 >= 256 ? 256 : ((dm.d / 4 + 31) / 32) * 32;
+  if (bf16)
+    combine_kernel<__nv_bfloat16>
+        <<<dm.T, threads, 0, st>>>(dm, ws, static_cast<__nv_bfloat16*>(out));
+  else
+    combine_kernel<float><<<dm.T, threads, 0, st>>>(dm, ws, static_cast<float*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_gather(const Dims& dm, const Workspace& ws, int32_t* topk_idx,
+                                float* topk_w, uint32_t* bits, uint32_t* bits_shared,
+                                cudaStream_t st) {
+  debug_gather_kernel<<<256, 256, 0, st>>>(dm, ws, topk_idx, topk_w, bits, bits_shared);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,269 @@
+// Down projection on the 5th-generation tensor cores, reading only the
+// W_down rows of an expert token group's active-neuron union.
+//
+// The pages' kernel gathers the weights of the active neurons, packs them
+// densely in shared memory and multiplies densely [gist.science EN
+// "Uncovering Intra-expert Activation Sparsity for Efficient Mixture-of-Expert
+// Model Execution", Technical Summary > Methodology > System Implementation in
+// vLLM > "Fused Up-Down Projection"]. Here the packing is done by TMA: each
+// active row is one 1-row box (128-byte swizzled) placed at its packed
+// position, so the tensor core sees a dense K-block of union rows.
+//
+// Work unit: (group, 128-column slice of d_model); K = the group's union rows.
+//   D[128 columns][N tokens] = W_down[e][U, slice]^T . H^T[U, group slots]
+// Both operands are MN-major in shared memory: a W_down row is 128
+// contiguous output columns (M), an H^T row is 64 contiguous slots (N).
+//   gathered mode: K-block = 64 union rows, each fetched as 1-row boxes
+//     (A: 2 boxes of 64 columns, B: 1 box of 64 slots); rows past the union
+//     are fetched out of range, which TMA fills with zeros.
+//   all-rows mode: K-block = 64 consecutive rows with 64-row boxes; h of
+//     inactive neurons is an exact zero, so the sum is the same.
+// Warp roles as in the gate/up kernel: warp 0 TMA, warp 1 MMA + TMEM owner,
+// warps 2-5 drain TMEM into Y[slot][col] (fp32), coalesced across lanes.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr uint32_t kAAtom = 64 * 128;  // one 64-row x 128-byte swizzled atom column
+constexpr uint32_t kABytes = 2 * kAAtom;
+
+struct DownUnit {
+  Group gr;
+  int g;
+  int slice;
+  int gather;     // 1: gathered rows, 0: all rows
+  int nk;         // K-blocks
+  int cnt;        // union rows (gathered)
+  int row_base;   // first row of this expert in the 2-D [experts*F][d] view
+  int shared;
+};
+
+__device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_slices) {
+  DownUnit du;
+  du.g = __ldcg(p.ws.tc_list + u / n_slices);
+  du.slice = u % n_slices;
+  du.gr = p.ws.groups[du.g];
+  du.shared = du.gr.expert >= p.dm.E;
+  const int F_e = du.shared ? p.dm.Fs : p.dm.F;
+  const int e_local = du.shared ? du.gr.expert - p.dm.E : du.gr.expert;
+  du.row_base = e_local * F_e;
+  du.gather = __ldcg(p.ws.group_path + du.g) == kPathTcGather;
+  du.cnt = __ldcg(p.ws.union_cnt + du.g);
+  du.nk = du.gather ? (du.cnt + kKBlock - 1) / kKBlock : F_e / kKBlock;
+  return du;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    down_tc_kernel(const __grid_constant__ DownTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stages = p.stages;
+  const uint32_t stage_bytes = kABytes + p.b_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
+  uint64_t* empty = full + stages;
+  uint64_t* tfull = empty + stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int n_slices = p.dm.d / kDownSlice;
+  const int n_units = __ldcg(p.ws.meta + kMetaTcCount) * n_slices;
+  const uint32_t buf_cols = p.n_max;
+  const int ht_oob = p.dm.F_max;  // H^T row past the end: zero fill
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_wd_row);
+      tma_prefetch_desc(&p.tm_wd_blk);
+      tma_prefetch_desc(&p.tm_ht_row);
+      tma_prefetch_desc(&p.tm_ht_blk);
+    }
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const DownUnit du = decode(p, u, n_slices);
+      const int N = (du.gr.m + 15) & ~15;
+      const int x0 = du.slice * kDownSlice;
+      const int* rows = p.ws.union_rows + static_cast<size_t>(du.g) * p.dm.F_max;
+      const CUtensorMap* wrow = du.shared ? &p.tm_wds_row : &p.tm_wd_row;
+      const CUtensorMap* wblk = du.shared ? &p.tm_wds_blk : &p.tm_wd_blk;
+      const int w_oob = du.shared ? p.dm.S * p.dm.Fs : p.dm.E * p.dm.F;
+      for (int kc = 0; kc < du.nk; ++kc, ++it) {
+        const uint32_t s = it % stages;
+        const uint32_t ph = (it / stages) & 1u;
+        if (!warp_wait(empty + s, ph ^ 1u, abort_flag, p.ws.status)) { ok = false; break; }
+        uint8_t* sa = smem + s * stage_bytes;
+        uint8_t* sb = sa + kABytes;
+        if (du.gather) {
+          if (lane == 0) mbar_arrive_expect_tx(full + s, kABytes + 64 * 128);
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = lane + 32 * h;
+            const int pos = kc * kKBlock + r;
+            const bool valid = pos < du.cnt;
+            const int j = valid ? __ldcg(rows + pos) : 0;
+            const int wy = valid ? du.row_base + j : w_oob;
+            const int hy = valid ? j : ht_oob;
+            tma_load_2d(sa + r * 128, wrow, full + s, x0, wy);
+            tma_load_2d(sa + kAAtom + r * 128, wrow, full + s, x0 + 64, wy);
+            tma_load_2d(sb + r * 128, &p.tm_ht_row, full + s, du.gr.slot0, hy);
+          }
+        } else {
+          const int nb = (N + 63) / 64;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(full + s, kABytes + nb * 64 * 128);
+            const int wy = du.row_base + kc * kKBlock;
+            tma_load_2d(sa, wblk, full + s, x0, wy);
+            tma_load_2d(sa + kAAtom, wblk, full + s, x0 + 64, wy);
+          }
+          __syncwarp();
+          if (lane < nb)
+            tma_load_2d(sb + lane * kAAtom, &p.tm_ht_blk, full + s, du.gr.slot0 + 64 * lane,
+                        kc * kKBlock);
+        }
+        __syncwarp();
+      }
+    }
+    const uint32_t n_tail = it < (uint32_t)stages ? it : (uint32_t)stages;
+    if (lane == 0) {
+      volatile int never = 0;
+      for (uint32_t i = it - n_tail; i < it; ++i)
+        mbar_wait(full + (i % stages), (i / stages) & 1u, &never, p.ws.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    uint32_t it = 0, uidx = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const DownUnit du = decode(p, u, n_slices);
+      if (du.nk == 0) continue;  // empty union: the epilogue writes zeros
+      const int N = (du.gr.m + 15) & ~15;
+      const uint32_t idesc = idesc_bf16_f32(kDownSlice, N, 1, 1);
+      const uint32_t b = uidx % 2;
+      const uint32_t tph = (uidx / 2) & 1u;
+      if (!warp_wait(tempty + b, tph ^ 1u, abort_flag, p.ws.status)) break;
+      tc_fence_after();
+      const uint32_t d_t = tmem_base + b * buf_cols;
+      for (int kc = 0; kc < du.nk; ++kc, ++it) {
+        const uint32_t s = it % stages;
+        const uint32_t ph = (it / stages) & 1u;
+        if (!warp_wait(full + s, ph, abort_flag, p.ws.status)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint64_t ad = smem_desc_sw128(sa, kAAtom, 1024);
+          const uint64_t bd = smem_desc_sw128(sa + kABytes, kAAtom, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kKBlock / 16; ++kk) {
+            // 16 K-rows of 128 B per step = 2048 B (descriptor units of 16 B)
+            mma_bf16(d_t, ad + 128 * kk, bd + 128 * kk, idesc, (kc | kk) != 0);
+          }
+          mma_commit(empty + s);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(tfull + b);
+      __syncwarp();
+      ++uidx;
+    }
+    if (lane == 0) {
+      mma_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, &never, p.ws.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    const int d = p.dm.d;
+    uint32_t uidx = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const DownUnit du = decode(p, u, n_slices);
+      const int m = du.gr.m;
+      const int col = du.slice * kDownSlice + 32 * q + lane;
+      float* yc = p.ws.y + static_cast<size_t>(du.gr.slot0) * d + col;
+      if (du.nk == 0) {
+        for (int c = 0; c < m; ++c) yc[static_cast<size_t>(c) * d] = 0.f;
+        continue;
+      }
+      const int N = (m + 15) & ~15;
+      const uint32_t b = uidx % 2;
+      const uint32_t tph = (uidx / 2) & 1u;
+      if (!warp_wait(tfull + b, tph, abort_flag, p.ws.status)) break;
+      tc_fence_after();
+      const uint32_t ta = tmem_base + lane_off + b * buf_cols;
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + c0, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + b);
+      ++uidx;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace
+
+size_t down_tc_smem_bytes(int b_bytes, int stages) {
+  return 1024 + static_cast<size_t>(stages) * (kABytes + b_bytes) +
+         (2 * stages + 5) * sizeof(uint64_t) + 16;
+}
+
+cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(down_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  down_tc_kernel<<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

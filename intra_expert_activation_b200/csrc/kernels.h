@@ -1,0 +1,129 @@
+// Internal interface between the C-ABI host code and the kernels: layer
+// dimensions, workspace pointers, kernel parameter blocks, launch wrappers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr uint32_t kSpinLimit = 4u << 20;  // ~1 s of polling with backoff
+constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT
+
+constexpr int kGroupMax = 256;      // tokens per expert token group (gate/up tile N)
+constexpr int kGatherMaxTokens = 64;  // groups on the gathered TC path hold <= 64 tokens
+constexpr int kSlotAlign = 8;       // expert slot ranges start at multiples of 8 slots
+constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
+constexpr int kDownSlice = 128;     // d_model columns per down TC tile (M)
+constexpr int kKBlock = 64;         // K elements per pipeline stage (128 B of bf16)
+
+// meta[] words written by the router's scan
+enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
+            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6, kMetaWords = 8 };
+
+// counters[] (u64), reset by the router's scan every forward
+enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
+               kCntTcGather = 4, kCntTcAll = 5, kCntRoutedH = 6, kCntSharedH = 7,
+               kCntWords = 8 };
+
+enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3 };
+
+// Requested path (mirrors moe_path in the public header).
+enum Mode { kModeAuto = 0, kModeDense = 1, kModeGemv = 2, kModeTc = 3, kModeTcAll = 4 };
+
+// One expert token group: up to kGroupMax consecutive slots of one expert.
+struct Group {
+  int32_t expert;  // 0..E-1 routed; E + s for shared expert s
+  int32_t slot0;   // first slot: column of H^T and row of Y
+  int32_t m;       // tokens in the group
+  int32_t xrow0;   // first row of the activations: X_perm row (routed) or token (shared)
+};
+
+struct Dims {
+  int d, F, Fs, E, S, k, T, renorm;
+  int F_max;          // max(F, Fs)
+  int fw;             // 32-bit words per neuron bitmap row: F_max / 32 (rounded up)
+  int slots_routed;   // routed slot capacity (multiple of kSlotAlign)
+  int slots_total;    // routed + shared slots = leading dimension of H^T
+  int T_pad;          // tokens rounded up to kSlotAlign (per shared expert)
+  int groups_max;
+  int mode;           // Mode
+  int gemv_max;       // AUTO: GEMV for groups with m <= gemv_max
+  float gather_density;
+  int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
+};
+
+struct Workspace {
+  int* status;                  // [1] device error word
+  int* meta;                    // [kMetaWords]
+  unsigned long long* counters; // [kCntWords]
+  int* topk_idx;                // [Tmax*kmax]
+  float* topk_w;                // [Tmax*kmax]
+  int* slot_of;                 // [Tmax*kmax]
+  int* perm;                    // [slots_routed] token of each routed slot, -1 for padding
+  Group* groups;                // [groups_max]
+  int* group_path;              // [groups_max]
+  uint32_t* union_bits;         // [groups_max][fw]
+  int* union_rows;              // [groups_max][F_max]
+  int* union_cnt;               // [groups_max]
+  int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
+  int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
+  uint32_t* act_bits;           // [slots_total][fw] or null (debug off)
+  void* xperm;                  // [slots_routed][d] activations gathered by slot
+  void* ht;                     // [F_max][slots_total] masked h, transposed
+  float* y;                     // [slots_total][d] per-slot expert outputs
+};
+
+// ------------------------------------------------------------ gate + up (tcgen05)
+struct GateUpTcParams {
+  CUtensorMap tm_wg, tm_wu;    // [E*F][d], box {64, 128}
+  CUtensorMap tm_wgs, tm_wus;  // [S*Fs][d], box {64, 128}
+  CUtensorMap tm_xperm;        // [slots_routed][d], box {64, 16}
+  CUtensorMap tm_x;            // [T][d], box {64, 16}
+  Dims dm;
+  Workspace ws;
+  float tau, tau_shared;
+  int dense;                   // 1: no threshold
+  int n_max;                   // largest MMA N of this launch (multiple of 16, <= 256)
+  int stages;
+  int nbuf;                    // TMEM accumulator buffers (1 or 2)
+  uint32_t tmem_cols;          // allocated TMEM columns
+};
+
+// ------------------------------------------------------------ down (tcgen05)
+struct DownTcParams {
+  CUtensorMap tm_wd_row, tm_wd_blk;    // [E*F][d]: box {64,1} and {64,64}
+  CUtensorMap tm_wds_row, tm_wds_blk;  // [S*Fs][d]
+  CUtensorMap tm_ht_row, tm_ht_blk;    // [F_max][slots_total]: box {64,1} and {64,64}
+  Dims dm;
+  Workspace ws;
+  int n_max;        // largest MMA N of this launch
+  int stages;
+  uint32_t tmem_cols;
+  int b_bytes;      // B bytes per stage
+};
+
+cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, const void* Wr,
+                         const float* bias, bool bf16, cudaStream_t st);
+cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
+                           cudaStream_t st);
+cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);
+size_t gate_up_tc_smem_bytes(int n_max, int stages);
+cudaError_t launch_gate_up_simt(const Dims& dm, const Workspace& ws, const float* x,
+                                const float* Wg, const float* Wu, const float* Wgs,
+                                const float* Wus, float tau, float tau_shared, int dense,
+                                cudaStream_t st);
+cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st);
+cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
+                             const void* Wds, bool bf16, int n_sms, cudaStream_t st);
+cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st);
+size_t down_tc_smem_bytes(int b_bytes, int stages);
+cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
+                           cudaStream_t st);
+cudaError_t launch_debug_gather(const Dims& dm, const Workspace& ws, int32_t* topk_idx,
+                                float* topk_w, uint32_t* bits, uint32_t* bits_shared,
+                                cudaStream_t st);
+
+}  // namespace moe

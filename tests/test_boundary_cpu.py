@@ -1,0 +1,135 @@
+"""Host-only checks of the C-ABI boundary: the library builds and loads,
+exports every entry point include/moe_sparse.h declares, and rejects bad
+descriptors and arguments synchronously without touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from intra_expert_activation_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_sparse.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from intra_expert_activation_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_sparse_\w+)\s*\(", src)))
+
+
+def good_desc(**kw):
+    d = dict(d_model=512, d_ff=384, n_experts=4, top_k_max=2, max_tokens=64, renormalize=1,
+             n_shared=0, d_ff_shared=0, dtype=_lib.MOE_BF16, path=0, debug=0, device=0,
+             gemv_max_tokens=0, gather_max_density=0.0)
+    d.update(kw)
+    return _lib.moe_sparse_desc(**d)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe_sparse.h but not exported"
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_only_the_abi_is_exported():
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {s for s in syms if s.startswith("moe_")}
+    assert ours == set(declared_functions())
+
+
+def test_struct_sizes_match_header():
+    assert ctypes.sizeof(_lib.moe_sparse_desc) == 14 * 4
+    assert ctypes.sizeof(_lib.moe_stats) == 10 * 8
+
+
+def test_valid_desc_accepted(lib):
+    assert lib.moe_sparse_validate_desc(ctypes.byref(good_desc())) == _lib.MOE_OK
+    f32 = good_desc(dtype=_lib.MOE_F32, d_model=256, d_ff=512)
+    assert lib.moe_sparse_validate_desc(ctypes.byref(f32)) == _lib.MOE_OK
+    shared = good_desc(n_shared=2, d_ff_shared=256)
+    assert lib.moe_sparse_validate_desc(ctypes.byref(shared)) == _lib.MOE_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d_model=0), _lib.MOE_ERR_INVALID),
+    (dict(d_model=320), _lib.MOE_ERR_UNSUPPORTED),           # bf16 needs d % 256
+    (dict(d_ff=100), _lib.MOE_ERR_UNSUPPORTED),              # bf16 needs d_ff % 128
+    (dict(n_experts=300), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(top_k_max=5), _lib.MOE_ERR_INVALID),               # > n_experts
+    (dict(max_tokens=-1), _lib.MOE_ERR_INVALID),
+    (dict(max_tokens=70000), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(dtype=7), _lib.MOE_ERR_INVALID),
+    (dict(path=9), _lib.MOE_ERR_INVALID),
+    (dict(n_shared=1, d_ff_shared=0), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(n_shared=9, d_ff_shared=128), _lib.MOE_ERR_INVALID),
+    (dict(dtype=_lib.MOE_F32, d_model=256, d_ff=512, path=3), _lib.MOE_ERR_UNSUPPORTED),
+    (dict(gather_max_density=1.5), _lib.MOE_ERR_INVALID),
+    (dict(gemv_max_tokens=-2), _lib.MOE_ERR_INVALID),
+])
+def test_bad_desc_rejected(lib, kw, code):
+    d = good_desc(**kw)
+    assert lib.moe_sparse_validate_desc(ctypes.byref(d)) == code
+    assert lib.moe_sparse_last_error(None)
+    ctx = ctypes.c_void_p()
+    assert lib.moe_sparse_init(ctypes.byref(d), ctypes.byref(ctx)) == code
+    assert not ctx.value
+
+
+def test_null_desc_and_ctx(lib):
+    assert lib.moe_sparse_validate_desc(None) == _lib.MOE_ERR_INVALID
+    ctx = ctypes.c_void_p()
+    assert lib.moe_sparse_init(None, ctypes.byref(ctx)) == _lib.MOE_ERR_INVALID
+    assert lib.moe_sparse_forward(None, None, 1, None, None, None, None, None, 0.0, 1, None,
+                                  None) == _lib.MOE_ERR_INVALID
+    assert lib.moe_sparse_get_stats(None, None, None) == _lib.MOE_ERR_INVALID
+    assert lib.moe_sparse_destroy(None) == _lib.MOE_OK
+
+
+def test_workspace_bytes_scale_with_tokens(lib):
+    small = ctypes.c_size_t()
+    big = ctypes.c_size_t()
+    assert lib.moe_sparse_workspace_bytes(ctypes.byref(good_desc(max_tokens=16)),
+                                          ctypes.byref(small)) == _lib.MOE_OK
+    assert lib.moe_sparse_workspace_bytes(ctypes.byref(good_desc(max_tokens=4096)),
+                                          ctypes.byref(big)) == _lib.MOE_OK
+    assert 0 < small.value < big.value
+    # h^T, X_perm and Y dominate: at least P * (2*d + 4*d) bytes
+    assert big.value >= 4096 * 2 * (2 * 512 + 4 * 512)
+
+
+def test_stage_names(lib):
+    names = [lib.moe_sparse_stage_name(i).decode() for i in range(len(_lib.STAGES))]
+    assert tuple(names) == _lib.STAGES
+    assert lib.moe_sparse_stage_name(len(_lib.STAGES)) is None
+
+
+def test_init_without_gpu_fails_cleanly(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    ctx = ctypes.c_void_p()
+    st = lib.moe_sparse_init(ctypes.byref(good_desc()), ctypes.byref(ctx))
+    assert st == _lib.MOE_ERR_CUDA
+    assert not ctx.value
+    assert lib.moe_sparse_last_error(None)
+
+
+def test_binding_refuses_missing_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.load()

@@ -1,0 +1,234 @@
+"""GPU parity of the C-ABI layer against the CPU oracle, on every synthetic
+workload at its full size, on small layers that span several tiles with
+ragged tails, with each down-projection path forced, and on edge cases."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from moe_inputs import LayerShape, make_tokens, make_weights
+from oracle import moe_oracle as om
+from _parity import (DeviceWeights, compare, make_layer, oracle_forward, run_gpu, tau_of,
+                     workload_tokens, workload_weights)
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["auto", "dense", "sparse_gemv", "sparse_tc", "sparse_tc_allrows"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    yield
+    torch.cuda.synchronize()
+
+
+def _calibrated(dw, x, q, shared_q=None):
+    ref0 = oracle_forward(dw, x, 0.0, 0.0)
+    tau = om.calibrate_tau(om.routed_abs_h(ref0), q)
+    ts = om.calibrate_tau(om.shared_abs_h(ref0), shared_q if shared_q is not None else q) \
+        if ref0.h_shared is not None else 0.0
+    return tau, ts
+
+
+def _check(layer, dw, x, tau, ts, dtype, dense=False, top_k=None):
+    gpu = run_gpu(layer, dw, x, tau, ts, top_k=top_k)
+    ref = oracle_forward(dw, x, tau, ts, dense=dense, top_k=top_k)
+    info = compare(gpu, ref, tau, ts, dtype, dense=dense)
+    assert layer.status() == 0
+    return gpu, ref, info
+
+
+# ----------------------------------------------------------------- fp32 layer
+
+@pytest.fixture(scope="module")
+def tiny():
+    return workload_weights("tiny_f32")
+
+
+@pytest.mark.parametrize("path", ["auto", "dense", "sparse_gemv"])
+def test_tiny_f32_full(tiny, path):
+    wl, dw = tiny
+    tau, _ = tau_of("tiny_f32", 0.7)
+    x = workload_tokens(wl, 16)
+    layer = make_layer(wl.shape, 16, path=path)
+    gpu, ref, info = _check(layer, dw, x, tau, 0.0, "f32", dense=(path == "dense"))
+    if path != "dense":
+        st = gpu["stats"]
+        assert st["n_routed_h"] == 16 * 2 * 512
+        meas = 1.0 - st["n_routed_active"] / st["n_routed_h"]
+        assert abs(meas - om.measured_sparsity(np.abs(ref.h), tau)) <= 2.0 / st["n_routed_h"] \
+            + info["active_mismatch_in_band"] / st["n_routed_h"]
+
+
+@pytest.mark.parametrize("T", [1, 5, 13, 16])
+def test_tiny_f32_ragged_batches(tiny, T):
+    wl, dw = tiny
+    tau, _ = tau_of("tiny_f32", 0.7)
+    layer = make_layer(wl.shape, 16)
+    _check(layer, dw, workload_tokens(wl, T), tau, 0.0, "f32")
+
+
+def test_tiny_f32_shared_and_smaller_k():
+    sh = LayerShape(d_model=256, n_experts=6, top_k=3, d_ff=160, renormalize=False, n_shared=2,
+                    d_ff_shared=96, dtype="f32")
+    dw = DeviceWeights(make_weights(sh, 11))
+    x = make_tokens(256, 21, 11, "f32")
+    tau, ts = _calibrated(dw, x, 0.6, 0.4)
+    layer = make_layer(sh, 32)
+    _check(layer, dw, x, tau, ts, "f32")
+    _check(layer, dw, x, tau, ts, "f32", top_k=2)
+
+
+# ------------------------------------------------- small bf16 layers, all paths
+
+SMALL = LayerShape(d_model=512, n_experts=4, top_k=2, d_ff=384, renormalize=True, dtype="bf16")
+SMALL_SHARED = LayerShape(d_model=768, n_experts=5, top_k=2, d_ff=256, renormalize=False,
+                          n_shared=1, d_ff_shared=384, dtype="bf16")
+
+
+@pytest.fixture(scope="module")
+def small():
+    return DeviceWeights(make_weights(SMALL, 21))
+
+
+@pytest.fixture(scope="module")
+def small_shared():
+    return DeviceWeights(make_weights(SMALL_SHARED, 22))
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 37, 100, 300, 777])
+@pytest.mark.parametrize("path", PATHS)
+def test_small_bf16_paths(small, T, path):
+    x = make_tokens(SMALL.d_model, T, 21, "bf16")
+    tau, _ = _calibrated(small, x, 0.7)
+    layer = make_layer(SMALL, 1024, path=path)
+    _check(layer, small, x, tau, 0.0, "bf16", dense=(path == "dense"))
+
+
+@pytest.mark.parametrize("T", [2, 45, 260])
+@pytest.mark.parametrize("path", ["auto", "dense", "sparse_gemv", "sparse_tc"])
+def test_small_bf16_shared(small_shared, T, path):
+    x = make_tokens(SMALL_SHARED.d_model, T, 22, "bf16")
+    tau, ts = _calibrated(small_shared, x, 0.7, 0.5)
+    layer = make_layer(SMALL_SHARED, 512, path=path)
+    _check(layer, small_shared, x, tau, ts, "bf16", dense=(path == "dense"))
+
+
+def test_sparse_tau0_equals_dense(small):
+    x = make_tokens(SMALL.d_model, 37, 21, "bf16")
+    a = run_gpu(make_layer(SMALL, 64, path="auto"), small, x, 0.0)
+    b = run_gpu(make_layer(SMALL, 64, path="dense"), small, x, 0.0)
+    err = np.linalg.norm(a["out"] - b["out"]) / np.linalg.norm(b["out"])
+    assert err <= 1e-6
+
+
+def test_tau_infinity_gives_zero(small):
+    x = make_tokens(SMALL.d_model, 9, 21, "bf16")
+    gpu = run_gpu(make_layer(SMALL, 16, path="auto"), small, x, math.inf)
+    assert np.all(gpu["out"] == 0.0)
+    assert gpu["stats"]["n_routed_active"] == 0
+
+
+def test_tau_infinity_leaves_shared_only(small_shared):
+    x = make_tokens(SMALL_SHARED.d_model, 11, 22, "bf16")
+    _, ts = _calibrated(small_shared, x, 0.7, 0.5)
+    layer = make_layer(SMALL_SHARED, 16)
+    _check(layer, small_shared, x, math.inf, ts, "bf16")
+
+
+def test_empty_batch_is_a_noop(small):
+    layer = make_layer(SMALL, 16)
+    out = torch.full((0, SMALL.d_model), 7.0, dtype=torch.bfloat16, device="cuda")
+    x = torch.empty((0, SMALL.d_model), dtype=torch.bfloat16, device="cuda")
+    layer.forward(x, small.W_router, small.W_gate, small.W_up, small.W_down, 0.1, 2, out=out)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+
+
+def test_max_tokens_and_rejections(small):
+    layer = make_layer(SMALL, 40)
+    x = make_tokens(SMALL.d_model, 40, 21, "bf16")
+    tau, _ = _calibrated(small, x, 0.7)
+    _check(layer, small, x, tau, 0.0, "bf16")
+    big = make_tokens(SMALL.d_model, 41, 21, "bf16").cuda()
+    with pytest.raises(Exception, match="T out of range"):
+        layer.forward(big, small.W_router, small.W_gate, small.W_up, small.W_down, tau, 2)
+    with pytest.raises(Exception, match="top_k"):
+        layer.forward(big[:4], small.W_router, small.W_gate, small.W_up, small.W_down, tau, 3)
+
+
+def test_deterministic(small):
+    x = make_tokens(SMALL.d_model, 100, 21, "bf16")
+    layer = make_layer(SMALL, 128)
+    a = run_gpu(layer, small, x, 0.2)["out"]
+    b = run_gpu(layer, small, x, 0.2)["out"]
+    assert np.array_equal(a, b)
+
+
+def test_timing_and_stats(small):
+    x = make_tokens(SMALL.d_model, 64, 21, "bf16").cuda()
+    layer = make_layer(SMALL, 64)
+    layer.set_timing(4)
+    layer.forward(x, small.W_router, small.W_gate, small.W_up, small.W_down, 0.3, 2)
+    t = layer.timing()
+    assert set(t) >= {"route", "gate_up", "combine"}
+    assert all(v >= 0 for v in t.values()) and t["gate_up"] > 0
+    st = layer.stats()
+    assert st["n_groups"] >= 1 and st["n_experts_touched"] >= 1
+
+
+# ------------------------------------------------------------ full workloads
+
+@pytest.fixture(scope="module")
+def mixtral():
+    return workload_weights("mixtral_decode")
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 64])
+def test_mixtral_decode(mixtral, T):
+    wl, dw = mixtral
+    tau, _ = tau_of("mixtral_decode", 0.7)
+    layer = make_layer(wl.shape, 64)
+    _check(layer, dw, workload_tokens(wl, T), tau, 0.0, "bf16")
+
+
+@pytest.mark.parametrize("path", ["dense", "sparse_gemv", "sparse_tc", "sparse_tc_allrows"])
+def test_mixtral_decode_paths(mixtral, path):
+    wl, dw = mixtral
+    tau, _ = tau_of("mixtral_decode", 0.7)
+    layer = make_layer(wl.shape, 64, path=path)
+    _check(layer, dw, workload_tokens(wl, 32), tau, 0.0, "bf16", dense=(path == "dense"))
+
+
+def test_many_small_experts():
+    wl, dw = workload_weights("many_small_experts")
+    tau, _ = tau_of("many_small_experts", 0.8)
+    layer = make_layer(wl.shape, 256)
+    gpu, ref, info = _check(layer, dw, workload_tokens(wl, 256), tau, 0.0, "bf16")
+    counts = np.bincount(ref.router.topk_idx.ravel(), minlength=128)
+    assert counts.max() >= 3 * max(counts.mean(), 1)  # the bias skews the load
+
+
+def test_shared_routed_prefill():
+    wl, dw = workload_weights("shared_routed_prefill")
+    tau, ts = tau_of("shared_routed_prefill", 0.6)
+    layer = make_layer(wl.shape, 4096)
+    _check(layer, dw, workload_tokens(wl, 4096), tau, ts, "bf16")
+
+
+@pytest.fixture(scope="module")
+def sweep():
+    return workload_weights("mixtral_sweep")
+
+
+@pytest.mark.parametrize("T", [1, 16, 128, 512])
+@pytest.mark.parametrize("q", [0.0, 0.5, 0.7, 0.9])
+def test_mixtral_sweep(sweep, T, q):
+    wl, dw = sweep
+    tau, _ = tau_of("mixtral_sweep", q)
+    layer = make_layer(wl.shape, 512)
+    _check(layer, dw, workload_tokens(wl, T), tau, 0.0, "bf16")
