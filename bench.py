@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager API calls instead of replaying a captured CUDA graph")
     return ap.parse_args()
 
 
@@ -82,19 +84,33 @@ class Clocks:
 
     def __init__(self, device: int):
         self.proc = None
-        try:
-            uuid = str(torch.cuda.get_device_properties(device).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
-        except Exception:
-            self.proc = None
+        self.error = None
+        props = torch.cuda.get_device_properties(device)
+        cands = []
+        uuid = str(getattr(props, "uuid", "") or "")
+        if uuid:
+            cands.append(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+        if hasattr(props, "pci_bus_id"):
+            cands.append(f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:"
+                         f"{getattr(props, 'pci_device_id', 0):02X}.0")
+        for sel in cands:
+            try:
+                probe = subprocess.run(["nvidia-smi", "--query-gpu=index", "--format=csv,noheader",
+                                        "-i", sel], capture_output=True, text=True, timeout=20)
+            except Exception as exc:  # no nvidia-smi
+                self.error = str(exc)
+                return
+            if probe.returncode == 0 and probe.stdout.strip():
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                     "-lms", "200", "-i", sel], stdout=subprocess.PIPE,
+                    stderr=subprocess.DEVNULL, text=True)
+                return
+            self.error = (probe.stderr or probe.stdout).strip()[:200]
 
     def stop(self):
         if self.proc is None:
-            return None
+            return {"error": self.error or "nvidia-smi unavailable"}
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -223,10 +239,25 @@ def run_ours(args, world, rank, local):
 
     stream = torch.cuda.current_stream(dev)
 
-    def timed(L, ring):
-        for _ in range(args.warmup):
+    def capture(L):
+        """One step of forwards captured into a CUDA graph (the library's
+        forward allocates nothing and never synchronises, so it captures)."""
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
             step(L)
-        L.set_timing(ring)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            step(L)
+        torch.cuda.synchronize(dev)
+        return g
+
+    def timed(L, graph=None):
+        """Pass A: K steps with nothing between the kernels (no events)."""
+        for _ in range(args.warmup):
+            graph.replay() if graph is not None else step(L)
         torch.cuda.synchronize(dev)
         barrier(world)
         torch.cuda.synchronize(dev)
@@ -234,21 +265,40 @@ def run_ours(args, world, rank, local):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
-            step(L)
+            graph.replay() if graph is not None else step(L)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
-        ms = e0.elapsed_time(e1)
-        launches = L.launch_count() - n0
-        per = L.timing_all(ring) if ring else []
+        per_step = (L.launch_count() - n0) // args.steps if graph is None else None
+        return e0.elapsed_time(e1), per_step
+
+    def kernel_times(L):
+        """Pass B: the same K steps, eager, with per-stage CUDA events recorded
+        by the library on the forward's stream around every kernel."""
+        L.set_timing(args.steps * len(tokens))
+        torch.cuda.synchronize(dev)
+        for _ in range(args.steps):
+            step(L)
+        torch.cuda.synchronize(dev)
+        per = L.timing_all(args.steps * len(tokens))
         L.set_timing(0)
-        return ms, launches, per
+        return per
 
     sparse = make("auto")
+    for _ in range(args.warmup):
+        step(sparse)
+    torch.cuda.synchronize(dev)
+    # launches per step, counted on an eager step
+    n0 = sparse.launch_count()
+    step(sparse)
+    launches_per_step = sparse.launch_count() - n0
+    g_sparse = None if args.eager else capture(sparse)
     clocks = Clocks(local)
-    ms_sparse, launches, per_fwd = timed(sparse, args.steps * len(tokens))
+    ms_sparse, _ = timed(sparse, g_sparse)
     clk = clocks.stop()
     ms_sparse = max_over_ranks(world, ms_sparse, local)
+    launches = launches_per_step * args.steps
+    per_fwd = kernel_times(sparse)
     tok_step = sum(tokens)
     value = tok_step * args.steps * world / (ms_sparse / 1e3)
 
@@ -264,10 +314,15 @@ def run_ours(args, world, rank, local):
     per_dense = []
     if not args.no_dense:
         dense = make("dense")
-        ms_dense, _, per_dense = timed(dense, args.steps * len(tokens))
+        for _ in range(args.warmup):
+            step(dense)
+        g_dense = None if args.eager else capture(dense)
+        ms_dense, _ = timed(dense, g_dense)
         ms_dense = max_over_ranks(world, ms_dense, local)
+        per_dense = kernel_times(dense)
         dense_line = {"value": tok_step * args.steps * world / (ms_dense / 1e3),
                       "ms_per_step": ms_dense / args.steps}
+        del g_dense
         dense.close()
 
     # per-kernel times, grouped by batch (forwards cycle through `tokens`)
@@ -383,9 +438,12 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": steps_launches,
+            "launch": "eager" if args.eager else "cuda_graph",
+            "kernel_times": "second timed pass of the same steps with per-stage CUDA events",
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    del g_sparse
     sparse.close()
     return 0
 

@@ -104,7 +104,7 @@ typedef struct {
   int32_t debug;              /* 1: keep per-pair active bitmaps for moe_sparse_get_debug */
   int32_t device;             /* CUDA device ordinal */
   int32_t gemv_max_tokens;    /* AUTO: groups with <= this many tokens use the GEMV path (0: 4) */
-  float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: 0.9) */
+  float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: never) */
 } moe_sparse_desc;
 
 typedef struct {

@@ -17,8 +17,76 @@ namespace moe {
 namespace {
 
 constexpr int kScanThreads = 256;
+constexpr int kListMax = 2048;
+
+// Sort a list of group ids ascending in place (ids are distinct): each
+// entry's position is the number of smaller entries.
+__device__ void sort_list(int* list, int n, int* tmp) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int v = __ldcg(list + i);
+    int r = 0;
+    for (int j = 0; j < n; ++j) r += __ldcg(list + j) < v;
+    tmp[r] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) list[i] = tmp[i];
+  __syncthreads();
+}
+
+// Last union_scan CTA: order the path lists by group id, and lay out the
+// GEMV work items: unit = (group, pass of MT tokens), item = (unit, split of
+// the union rows). Splits aim at about two items per CTA of the GEMV grid,
+// with kGemvRowsMin..kGemvRowsMax rows per item.
+__device__ void scan_finish(const Dims& dm, Workspace& ws) {
+  __shared__ int tmp[kListMax];
+  __shared__ int s_units[kListMax];
+  __shared__ int s_rows[kListMax];
+  __shared__ int total_units;
+  const int n_gemv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
+  const int n_tc = min(__ldcg(ws.meta + kMetaTcCount), kListMax);
+  sort_list(ws.gemv_list, n_gemv, tmp);
+  sort_list(ws.tc_list, n_tc, tmp);
+  const int mt = dm.no_tc ? 8 : kGemvTokens;
+  for (int i = threadIdx.x; i < n_gemv; i += blockDim.x) {
+    const int g = __ldcg(ws.gemv_list + i);
+    s_units[i] = (ws.groups[g].m + mt - 1) / mt;
+    s_rows[i] = __ldcg(ws.union_cnt + g);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int u = 0;
+    for (int i = 0; i < n_gemv; ++i) u += s_units[i];
+    total_units = u;
+  }
+  __syncthreads();
+  const int target = max(1, 4 * dm.n_sms / max(total_units, 1));
+  for (int i = threadIdx.x; i < n_gemv; i += blockDim.x) {
+    const int cnt = s_rows[i];
+    const int s_min = max(1, (cnt + kGemvRowsMax - 1) / kGemvRowsMax);
+    const int s_max = max(s_min, cnt / kGemvRowsMin);
+    tmp[i] = min(max(target, s_min), s_max);  // splits of every unit of group i
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* item_off = ws.gemv_item_off;
+    int* unit_off = ws.gemv_item_off + dm.groups_max + 1;
+    int units = 0, items = 0;
+    for (int i = 0; i < n_gemv; ++i) {
+      unit_off[i] = units;
+      item_off[i] = items;
+      units += s_units[i];
+      items += s_units[i] * tmp[i];
+    }
+    unit_off[n_gemv] = units;
+    item_off[n_gemv] = items;
+    ws.meta[kMetaGemvItems] = items;
+    ws.meta[kMetaGemvUnits] = units;
+    ws.meta[kMetaScanDone] = 0;
+  }
+}
 
 __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Workspace ws) {
+  grid_dep_wait();
   const int g = blockIdx.x;
   if (g >= __ldcg(ws.meta + kMetaGroups)) return;
   const Group gr = ws.groups[g];
@@ -64,6 +132,7 @@ __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Works
     __syncthreads();
   }
 
+  __shared__ int is_last;
   if (threadIdx.x == 0) {
     const int cnt = carry;
     const int m = gr.m;
@@ -92,7 +161,25 @@ __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Works
               static_cast<unsigned long long>(path == kPathTcAll ? F_e : cnt));
     atomicAdd(ws.counters + (path == kPathGemv ? kCntGemv
                              : path == kPathTcGather ? kCntTcGather : kCntTcAll), 1ull);
+    is_last = path == kPathGemv;  // reused below: zero this group's Y rows
   }
+  __syncthreads();
+  if (is_last) {
+    // GEMV splits add into Y: start from zero
+    float4* yz = reinterpret_cast<float4*>(ws.y + static_cast<size_t>(gr.slot0) * dm.d);
+    const int n4 = gr.m * dm.d / 4;
+    for (int q = threadIdx.x; q < n4; q += blockDim.x) yz[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int ticket = atomicAdd(ws.meta + kMetaScanDone, 1);
+    is_last = ticket == __ldcg(ws.meta + kMetaGroups) - 1;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  scan_finish(dm, ws);
 }
 
 template <typename TX>
@@ -111,6 +198,7 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 
 template <typename TX>
 __global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX* out) {
+  grid_dep_wait();
   const int t = blockIdx.x;
   const int d = dm.d, k = dm.k;
   __shared__ int slot[16];
@@ -143,6 +231,7 @@ __global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX*
 
 __global__ void debug_gather_kernel(Dims dm, Workspace ws, int32_t* topk_idx, float* topk_w,
                                     uint32_t* bits, uint32_t* bits_shared) {
+  grid_dep_wait();
   const int P = dm.T * dm.k;
   const int fwr = (dm.F + 31) / 32, fws = (dm.Fs + 31) / 32;
   const int stride = gridDim.x * blockDim.x;
@@ -171,19 +260,16 @@ __global__ void debug_gather_kernel(Dims dm, Workspace ws, int32_t* topk_idx, fl
 }  // namespace
 
 cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st) {
-  union_scan_kernel<<<dm.groups_max, kScanThreads, 0, st>>>(dm, ws);
-  return cudaGetLastError();
+  return launch_k(union_scan_kernel, dm.groups_max, kScanThreads, 0, st, dm, ws);
 }
 
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
                            cudaStream_t st) {
   const int threads = dm.d / 4 >= 256 ? 256 : ((dm.d / 4 + 31) / 32) * 32;
   if (bf16)
-    combine_kernel<__nv_bfloat16>
-        <<<dm.T, threads, 0, st>>>(dm, ws, static_cast<__nv_bfloat16*>(out));
-  else
-    combine_kernel<float><<<dm.T, threads, 0, st>>>(dm, ws, static_cast<float*>(out));
-  return cudaGetLastError();
+    return launch_k(combine_kernel<__nv_bfloat16>, dm.T, threads, 0, st, dm, ws,
+                    static_cast<__nv_bfloat16*>(out));
+  return launch_k(combine_kernel<float>, dm.T, threads, 0, st, dm, ws, static_cast<float*>(out));
 }
 
 cudaError_t launch_debug_gather(const Dims& dm, const Workspace& ws, int32_t* topk_idx,

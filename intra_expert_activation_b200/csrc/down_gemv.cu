@@ -10,35 +10,42 @@
 // cost is the bytes of the rows it reads ["Fused Up-Down Projection": only
 // the active neurons' weights are fetched].
 //
-// Work unit: (group, slice of d_model columns), handled by one thread-block
-// cluster of kCluster CTAs that split the union rows evenly; each warp walks
-// its rows with an 8-deep unrolled stream of 16-byte loads (one 512-byte row
-// segment per warp load), keeps fp32 partial sums in registers, the CTA sums
-// its warps through shared memory, and rank 0 sums the CTAs of the cluster
-// through distributed shared memory in rank order (deterministic) and writes
-// Y[slot][columns]. Clusters walk units with a static stride.
-#include <cooperative_groups.h>
-
+// Work: a unit is (group, pass of up to MT tokens); its union rows are cut
+// into splits, and a work item is one split of one unit over all d_model
+// columns. Persistent CTAs of 16 warps (one per SM) stride over the items. A
+// CTA first stages the item's row ids and the tokens' h values in shared
+// memory; then each warp owns one 512-byte column slice and streams the
+// item's rows through its own ring of shared-memory stages with cp.async
+// (16 bytes per lane per row; kStages x kBatch rows in flight per warp, with
+// no registers held by data in flight), and multiplies each landed row
+// segment by the tokens' h values into fp32 registers. Each lane copies and
+// later reads back exactly its own 16 bytes, so a wait on the lane's own copy
+// group is all the synchronisation the ring needs. An item that is a whole
+// unit stores its result into Y[slot][columns]; a split adds its partial into
+// Y (zeroed by the union scan) with vector fp32 atomics, so the splits of a
+// unit are summed in arrival order: results agree to fp32 rounding, not
+// bitwise, between runs on this path.
 #include "common.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace moe {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCluster = 8;
-constexpr int kUnroll = 8;
-constexpr int kRowChunk = 2048;  // union positions staged in shared memory at a time
+constexpr int kBatch = 8;    // rows per stage
+constexpr int kStages = 3;   // stages per warp ring
+constexpr int kWarpRing = kStages * kBatch * 32 * 16;  // bytes per warp ring
 
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 template <typename TW>
@@ -96,143 +103,173 @@ __device__ __forceinline__ void load_h(const TW* p, int mt, float (&h)[MT]) {
     if (i >= mt) h[i] = 0.f;
 }
 
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 template <typename TW, int MT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
     down_gemv_kernel(Dims dm, Workspace ws, const TW* __restrict__ Wd,
                      const TW* __restrict__ Wds) {
   constexpr int VEC = Vec<TW>::N;
   constexpr int SW = 32 * VEC;  // columns per slice: one 512-byte row segment
-  __shared__ float red[kWarps][MT][SW];
-  __shared__ float part[MT][SW];
-  __shared__ int srows[kRowChunk];
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* rings = smem;                                          // [kWarps][kWarpRing]
+  int* srow = reinterpret_cast<int*>(smem + kWarps * kWarpRing);  // [kGemvRowsMax]
+  float* sh = reinterpret_cast<float*>(srow + kGemvRowsMax);      // [kGemvRowsMax][MT]
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int cid = blockIdx.x / kCluster;
-  const int ncl = gridDim.x / kCluster;
+  grid_dep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int n_slices = d / SW;
-  const int n_units = __ldcg(ws.meta + kMetaGemvCount) * n_slices;
+  const int n_phase = n_slices >= kWarps ? 1 : kWarps / n_slices;  // warps per slice
+  const int n_tasks = n_slices * n_phase;
+  const int n_list = __ldcg(ws.meta + kMetaGemvCount);
+  const int n_items = __ldcg(ws.meta + kMetaGemvItems);
+  const int* item_off = ws.gemv_item_off;
+  const int* unit_off = ws.gemv_item_off + dm.groups_max + 1;
   const size_t ld = static_cast<size_t>(dm.slots_total);
   const TW* ht = static_cast<const TW*>(ws.ht);
+  uint8_t* ring = rings + warp * kWarpRing;
+  const uint32_t ring_s = smem_u32(ring) + lane * 16;
 
-  for (int u = cid; u < n_units; u += ncl) {
-    const int g = __ldcg(ws.gemv_list + u / n_slices);
-    const int c0 = (u % n_slices) * SW;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    // listed group i with item_off[i] <= item < item_off[i + 1]
+    int lo_i = 0, hi_i = n_list;
+    while (hi_i - lo_i > 1) {
+      const int mid = (lo_i + hi_i) >> 1;
+      if (__ldcg(item_off + mid) <= item) lo_i = mid; else hi_i = mid;
+    }
+    const int i = lo_i;
+    const int g = __ldcg(ws.gemv_list + i);
     const Group gr = ws.groups[g];
+    const int units_i = __ldcg(unit_off + i + 1) - __ldcg(unit_off + i);
+    const int splits = (__ldcg(item_off + i + 1) - __ldcg(item_off + i)) / units_i;
+    const int local = item - __ldcg(item_off + i);
+    const int split = local % splits, pass = local / splits;
+    const int tp = pass * MT;
+    const int mt = min(MT, gr.m - tp);
+    const int cnt = __ldcg(ws.union_cnt + g);
+    const int lo = static_cast<int>(static_cast<long long>(split) * cnt / splits);
+    const int n = static_cast<int>(static_cast<long long>(split + 1) * cnt / splits) - lo;
+
+    // stage the item's rows and h values (fp32, zero past mt)
+    const int* rows = ws.union_rows + static_cast<size_t>(g) * dm.F_max + lo;
+    const TW* hcol = ht + gr.slot0 + tp;
+    for (int r = threadIdx.x; r < n; r += kThreads) {
+      const int j = __ldcg(rows + r);
+      srow[r] = j;
+      float hv[MT];
+      load_h<TW, MT>(hcol + static_cast<size_t>(j) * ld, mt, hv);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) sh[r * MT + t] = hv[t];
+    }
+    __syncthreads();
+
     const bool shared = gr.expert >= dm.E;
     const int F_e = shared ? dm.Fs : dm.F;
-    const TW* W = shared ? Wds + static_cast<size_t>(gr.expert - dm.E) * F_e * d
-                         : Wd + static_cast<size_t>(gr.expert) * F_e * d;
-    W += c0 + lane * VEC;
-    const int cnt = __ldcg(ws.union_cnt + g);
-    const int* rows = ws.union_rows + static_cast<size_t>(g) * dm.F_max;
-    const int lo = static_cast<int>(static_cast<long long>(rank) * cnt / kCluster);
-    const int hi = static_cast<int>(static_cast<long long>(rank + 1) * cnt / kCluster);
-
-    for (int tp = 0; tp < gr.m; tp += MT) {
-      const int mt = min(MT, gr.m - tp);
-      const TW* hcol = ht + gr.slot0 + tp;
+    const TW* Wbase = shared ? Wds + static_cast<size_t>(gr.expert - dm.E) * F_e * d
+                             : Wd + static_cast<size_t>(gr.expert) * F_e * d;
+    float* y = ws.y + static_cast<size_t>(gr.slot0 + tp) * d;
+    for (int task = warp; task < n_tasks; task += kWarps) {
+      const int slice = task % n_slices, phase = task / n_slices;
+      const int col = slice * SW + lane * VEC;
+      const TW* W = Wbase + col;
+      // this warp's rows: p = phase + n_phase * q, q < nq
+      const int nq = n > phase ? (n - phase + n_phase - 1) / n_phase : 0;
+      const int nb = (nq + kBatch - 1) / kBatch;
+      auto issue = [&](int b) {
+        if (b < nb) {
+          const uint32_t dst = ring_s + (b % kStages) * (kBatch * 512);
+#pragma unroll
+          for (int r = 0; r < kBatch; ++r) {
+            const int q = b * kBatch + r;
+            if (q < nq)
+              cp_async16(dst + r * 512, W + static_cast<size_t>(srow[phase + n_phase * q]) * d);
+          }
+        }
+        cp_async_commit();
+      };
       float acc[MT][VEC];
 #pragma unroll
       for (int t = 0; t < MT; ++t)
 #pragma unroll
         for (int v = 0; v < VEC; ++v) acc[t][v] = 0.f;
-
-      for (int base = lo; base < hi; base += kRowChunk) {
-        const int n = min(kRowChunk, hi - base);
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kThreads) srows[i] = __ldcg(rows + base + i);
-        __syncthreads();
-        int i = warp;
-        for (; i + kWarps * (kUnroll - 1) < n; i += kWarps * kUnroll) {
-          uint4 wv[kUnroll];
-          float hv[kUnroll][MT];
 #pragma unroll
-          for (int r = 0; r < kUnroll; ++r) {
-            const int j = srows[i + kWarps * r];
-            wv[r] = ld_stream(W + static_cast<size_t>(j) * d);
-            load_h<TW, MT>(hcol + static_cast<size_t>(j) * ld, mt, hv[r]);
-          }
+      for (int b = 0; b < kStages - 1; ++b) issue(b);
+      for (int b = 0; b < nb; ++b) {
+        issue(b + kStages - 1);
+        cp_async_wait<kStages - 1>();
+        const uint8_t* src = ring + (b % kStages) * (kBatch * 512) + lane * 16;
 #pragma unroll
-          for (int r = 0; r < kUnroll; ++r) {
+        for (int r = 0; r < kBatch; ++r) {
+          const int q = b * kBatch + r;
+          if (q < nq) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(src + r * 512);
             float w[VEC];
-            Vec<TW>::unpack(wv[r], w);
+            Vec<TW>::unpack(wv, w);
+            const float* hq = sh + (phase + n_phase * q) * MT;
 #pragma unroll
-            for (int t = 0; t < MT; ++t)
+            for (int t = 0; t < MT; ++t) {
+              const float h = hq[t];
 #pragma unroll
-              for (int v = 0; v < VEC; ++v) acc[t][v] = fmaf(hv[r][t], w[v], acc[t][v]);
+              for (int v = 0; v < VEC; ++v) acc[t][v] = fmaf(h, w[v], acc[t][v]);
+            }
           }
         }
-        for (; i < n; i += kWarps) {
-          const int j = srows[i];
-          const uint4 wv = ld_stream(W + static_cast<size_t>(j) * d);
-          float hv[MT];
-          load_h<TW, MT>(hcol + static_cast<size_t>(j) * ld, mt, hv);
-          float w[VEC];
-          Vec<TW>::unpack(wv, w);
+      }
+      cp_async_wait<0>();
+      const bool whole = splits == 1 && n_phase == 1;
 #pragma unroll
-          for (int t = 0; t < MT; ++t)
+      for (int t = 0; t < MT; ++t) {
+        if (t < mt) {
+          float* yt = y + static_cast<size_t>(t) * d + col;
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[t][v] = fmaf(hv[t], w[v], acc[t][v]);
+          for (int v = 0; v < VEC; v += 4) {
+            if (whole)
+              *reinterpret_cast<float4*>(yt + v) =
+                  make_float4(acc[t][v], acc[t][v + 1], acc[t][v + 2], acc[t][v + 3]);
+            else
+              red_add_v4(yt + v, acc[t][v], acc[t][v + 1], acc[t][v + 2], acc[t][v + 3]);
+          }
         }
       }
-
-      // CTA: sum the warps (fixed order)
-#pragma unroll
-      for (int t = 0; t < MT; ++t)
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) red[warp][t][lane * VEC + v] = acc[t][v];
-      __syncthreads();
-      for (int e = threadIdx.x; e < MT * SW; e += kThreads) {
-        const int t = e / SW, c = e % SW;
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += red[w][t][c];
-        part[t][c] = s;
-      }
-      // cluster: rank 0 sums the CTAs in rank order
-      cluster.sync();
-      if (rank == 0) {
-        float* y = ws.y + static_cast<size_t>(gr.slot0 + tp) * d + c0;
-        for (int e = threadIdx.x; e < mt * SW; e += kThreads) {
-          const int t = e / SW, c = e % SW;
-          float s = 0.f;
-#pragma unroll
-          for (int r = 0; r < kCluster; ++r) s += cluster.map_shared_rank(&part[0][0], r)[t * SW + c];
-          y[static_cast<size_t>(t) * d + c] = s;
-        }
-      }
-      cluster.sync();
     }
+    __syncthreads();
   }
 }
 
 }  // namespace
 
+size_t down_gemv_smem_bytes(bool bf16) {
+  const int mt = bf16 ? kGemvTokens : 8;
+  return static_cast<size_t>(kWarps) * kWarpRing + sizeof(int) * kGemvRowsMax +
+         sizeof(float) * kGemvRowsMax * mt;
+}
+
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
                              const void* Wds, bool bf16, int n_sms, cudaStream_t st) {
-  int n_clusters = (2 * n_sms + kCluster - 1) / kCluster;
-  if (n_clusters < 1) n_clusters = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_clusters * kCluster);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(down_gemv_kernel<__nv_bfloat16, kGemvTokens>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)down_gemv_smem_bytes(true));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(down_gemv_kernel<float, 8>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)down_gemv_smem_bytes(false));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = n_sms;  // one 16-warp CTA per SM
   if (bf16)
-    return cudaLaunchKernelEx(&cfg, down_gemv_kernel<__nv_bfloat16, 4>, dm, ws,
-                              static_cast<const __nv_bfloat16*>(Wd),
-                              static_cast<const __nv_bfloat16*>(Wds));
-  return cudaLaunchKernelEx(&cfg, down_gemv_kernel<float, 8>, dm, ws,
-                            static_cast<const float*>(Wd), static_cast<const float*>(Wds));
+    return launch_k(down_gemv_kernel<__nv_bfloat16, kGemvTokens>, grid, kThreads,
+                    down_gemv_smem_bytes(true), st, dm, ws,
+                    static_cast<const __nv_bfloat16*>(Wd), static_cast<const __nv_bfloat16*>(Wds));
+  return launch_k(down_gemv_kernel<float, 8>, grid, kThreads, down_gemv_smem_bytes(false), st,
+                  dm, ws, static_cast<const float*>(Wd), static_cast<const float*>(Wds));
 }
 
 }  // namespace moe

@@ -87,6 +87,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
+  // TMEM is taken only once the previous kernel has completed, so a CTA of
+  // this kernel never holds TMEM while waiting on another kernel
+  grid_dep_wait();
   if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
   tc_fence_before();
   __syncthreads();
@@ -262,8 +265,7 @@ cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStr
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  down_tc_kernel<<<grid, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_k(down_tc_kernel, grid, kThreads, smem, st, p);
 }
 
 }  // namespace moe

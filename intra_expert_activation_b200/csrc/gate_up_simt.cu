@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kThreads)
                         float tau_shared, int dense) {
   __shared__ uint32_t tok_bits[kGroupMax];
   __shared__ uint32_t uni;
+  grid_dep_wait();
   const int n_rg = __ldcg(ws.meta + kMetaRoutedGroups);
   const int n_g = __ldcg(ws.meta + kMetaGroups);
   const int blk_r = dm.F / 32;
@@ -107,9 +108,8 @@ cudaError_t launch_gate_up_simt(const Dims& dm, const Workspace& ws, const float
                                 cudaStream_t st) {
   const int units_max = dm.groups_max * (dm.F_max / 32);
   const int grid = units_max < 4096 ? units_max : 4096;
-  gate_up_simt_kernel<<<grid, kThreads, 0, st>>>(dm, ws, x, Wg, Wu, Wgs, Wus, tau, tau_shared,
-                                                 dense);
-  return cudaGetLastError();
+  return launch_k(gate_up_simt_kernel, grid, kThreads, 0, st, dm, ws, x, Wg, Wu, Wgs, Wus, tau,
+                  tau_shared, dense);
 }
 
 }  // namespace moe

@@ -7,7 +7,32 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
+
+// Every kernel is launched with programmatic stream serialization: its CTAs
+// may be scheduled while the previous kernel on the stream drains, and they
+// call grid_dep_wait() (griddepcontrol.wait) before touching global memory,
+// so the launch latency overlaps the predecessor's tail. MOE_PDL=0 in the
+// environment turns it off.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 constexpr uint32_t kSpinLimit = 4u << 20;  // ~1 s of polling with backoff
 constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT
@@ -18,10 +43,15 @@ constexpr int kSlotAlign = 8;       // expert slot ranges start at multiples of 
 constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
 constexpr int kDownSlice = 128;     // d_model columns per down TC tile (M)
 constexpr int kKBlock = 64;         // K elements per pipeline stage (128 B of bf16)
+constexpr int kRouteTokens = 16;    // tokens per router CTA
+constexpr int kGemvRowsMax = 768;   // union rows per GEMV work item at most
+constexpr int kGemvRowsMin = 32;    // ... and at least (unless the union is smaller)
+constexpr int kGemvTokens = 4;      // tokens per GEMV unit (bf16); fp32 uses 8
 
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
-            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6, kMetaWords = 8 };
+            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
+            kMetaScanDone = 7, kMetaGemvItems = 8, kMetaGemvUnits = 9, kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
@@ -53,6 +83,7 @@ struct Dims {
   int gemv_max;       // AUTO: GEMV for groups with m <= gemv_max
   float gather_density;
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
+  int n_sms;          // streaming multiprocessors of the device
 };
 
 struct Workspace {
@@ -62,6 +93,10 @@ struct Workspace {
   int* topk_idx;                // [Tmax*kmax]
   float* topk_w;                // [Tmax*kmax]
   int* slot_of;                 // [Tmax*kmax]
+  int* rank_cta;                // [Tmax*kmax] rank of a pair among its CTA's pairs of that expert
+  int* hist;                    // [router CTAs][E] per-CTA expert counts, then CTA base offsets
+  int* expert_off;              // [E+1] first slot of each expert (multiple of kSlotAlign)
+  int* expert_cnt;              // [E] routed pairs per expert
   int* perm;                    // [slots_routed] token of each routed slot, -1 for padding
   Group* groups;                // [groups_max]
   int* group_path;              // [groups_max]
@@ -70,6 +105,8 @@ struct Workspace {
   int* union_cnt;               // [groups_max]
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
   int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
+  int* gemv_item_off;           // [groups_max+1] first GEMV work item of each listed group
+
   uint32_t* act_bits;           // [slots_total][fw] or null (debug off)
   void* xperm;                  // [slots_routed][d] activations gathered by slot
   void* ht;                     // [F_max][slots_total] masked h, transposed

@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -16,6 +17,16 @@
 
 using moe::Dims;
 using moe::Workspace;
+
+namespace moe {
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+}  // namespace moe
 
 namespace {
 
@@ -73,13 +84,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 struct Layout {
   Dims cap;
-  size_t off[24];
+  size_t off[32];
   size_t total;
 };
 
-enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bActBits, bXperm, bHt, bY,
-           bCount };
+enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
+           bExpCnt, bPerm, bGroups, bGroupPath,
+           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bGemvItemOff, bActBits,
+           bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   if (!d) { err = "desc is NULL"; return MOE_ERR_INVALID; }
@@ -111,6 +123,12 @@ moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   if (d->gemv_max_tokens < 0 || d->gemv_max_tokens > 256) { err = "gemv_max_tokens must be in 0..256"; return MOE_ERR_INVALID; }
   if (!(d->gather_max_density >= 0.f && d->gather_max_density <= 1.f)) { err = "gather_max_density must be in [0, 1]"; return MOE_ERR_INVALID; }
   if ((long long)d->max_tokens * d->top_k_max > (1ll << 22)) { err = "max_tokens * top_k_max > 2^22"; return MOE_ERR_UNSUPPORTED; }
+  {
+    const long long P = (long long)d->max_tokens * d->top_k_max;
+    const long long groups = P / 256 + std::min<long long>(d->n_experts, P) +
+                             (long long)d->n_shared * ((d->max_tokens + 255) / 256) + 1;
+    if (groups > 2048) { err = "too many expert token groups (max_tokens * top_k_max too large)"; return MOE_ERR_UNSUPPORTED; }
+  }
   return MOE_OK;
 }
 
@@ -137,7 +155,7 @@ Layout make_layout(const moe_sparse_desc* d) {
                  c.S * ((c.T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
   c.mode = d->path;
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
-  c.gather_density = d->gather_max_density > 0.f ? d->gather_max_density : 0.9f;
+  c.gather_density = d->gather_max_density;
   c.no_tc = bf16 ? 0 : 1;
 
   const size_t es = bf16 ? 2 : 4;
@@ -148,6 +166,10 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bTopkIdx] = sizeof(int) * P;
   sz[bTopkW] = sizeof(float) * P;
   sz[bSlotOf] = sizeof(int) * P;
+  sz[bRankCta] = sizeof(int) * P;
+  sz[bHist] = sizeof(int) * (size_t)((c.T + 1) / 2) * c.E;  // at most ceil(T/2) router CTAs
+  sz[bExpOff] = sizeof(int) * (c.E + 1);
+  sz[bExpCnt] = sizeof(int) * c.E;
   sz[bPerm] = sizeof(int) * c.slots_routed;
   sz[bGroups] = sizeof(moe::Group) * c.groups_max;
   sz[bGroupPath] = sizeof(int) * c.groups_max;
@@ -156,6 +178,7 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bUnionCnt] = sizeof(int) * c.groups_max;
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
+  sz[bGemvItemOff] = sizeof(int) * 2 * (size_t)(c.groups_max + 1);
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;
   sz[bXperm] = es * (size_t)c.slots_routed * c.d;
   sz[bHt] = es * (size_t)c.F_max * c.slots_total;
@@ -295,6 +318,7 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   c->lay = make_layout(desc);
   c->bf16 = desc->dtype == MOE_BF16;
   c->n_sms = sms;
+  c->lay.cap.n_sms = sms;
   e = cudaMalloc(&c->mem, c->lay.total);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -319,6 +343,10 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.topk_idx = reinterpret_cast<int*>(b + o[bTopkIdx]);
   w.topk_w = reinterpret_cast<float*>(b + o[bTopkW]);
   w.slot_of = reinterpret_cast<int*>(b + o[bSlotOf]);
+  w.rank_cta = reinterpret_cast<int*>(b + o[bRankCta]);
+  w.hist = reinterpret_cast<int*>(b + o[bHist]);
+  w.expert_off = reinterpret_cast<int*>(b + o[bExpOff]);
+  w.expert_cnt = reinterpret_cast<int*>(b + o[bExpCnt]);
   w.perm = reinterpret_cast<int*>(b + o[bPerm]);
   w.groups = reinterpret_cast<moe::Group*>(b + o[bGroups]);
   w.group_path = reinterpret_cast<int*>(b + o[bGroupPath]);
@@ -327,6 +355,7 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.union_cnt = reinterpret_cast<int*>(b + o[bUnionCnt]);
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
+  w.gemv_item_off = reinterpret_cast<int*>(b + o[bGemvItemOff]);
   w.act_bits = desc->debug ? reinterpret_cast<uint32_t*>(b + o[bActBits]) : nullptr;
   w.xperm = b + o[bXperm];
   w.ht = b + o[bHt];
@@ -506,11 +535,15 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     p.n_max = n_max;
     p.b_bytes = std::max(8192, (n_max + 63) / 64 * 8192);
     p.tmem_cols = pow2_at_least(2u * n_max);
+    // small groups (decode): two CTAs per SM so that a unit's epilogue and
+    // the next unit's loads overlap across CTAs; large groups: one CTA
+    const int ctas_per_sm = n_max <= 64 ? 2 : 1;
+    const size_t budget = ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
     const size_t stage_bytes = 16384 + (size_t)p.b_bytes;
-    p.stages = (int)std::min<size_t>(8, (225 * 1024 - 2048) / stage_bytes);
+    p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
     const size_t smem = moe::down_tc_smem_bytes(p.b_bytes, p.stages);
     const int units_max = dm.groups_max * (cap.d / moe::kDownSlice);
-    const int grid = std::max(1, std::min(units_max, c->n_sms));
+    const int grid = std::max(1, std::min(units_max, ctas_per_sm * c->n_sms));
     e = moe::launch_down_tc(p, grid, smem, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_tc launch");
     stage_ran[5] = true;

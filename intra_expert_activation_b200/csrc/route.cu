@@ -1,88 +1,136 @@
-// Router: logits, softmax over all experts, top-k (+ renormalisation), then a
+// Router: logits, softmax over all experts, top-k (+ renormalisation), and a
 // deterministic stable counting sort of the routed (token, expert) pairs into
 // per-expert slot ranges and expert token groups. The pages keep the dense
 // model's router as it is [gist.science EN "Uncovering Intra-expert
 // Activation Sparsity for Efficient Mixture-of-Expert Model Execution",
 // Technical Summary > Methodology > System Implementation in vLLM].
 //
-// route_kernel: one CTA per 32 tokens. Logits are fp32 dot products over
-// shared-memory tiles of x and W_router (sequential in d, so every call gives
-// the same bits). One warp per token then picks the top-k by logit (equal
-// logits: lower expert index), and the softmax weights. The last CTA to
-// finish (atomic ticket after a fence) runs the scan for the whole batch.
-//
-// permute_kernel: X_perm[slot] = x[perm[slot]] (zero rows for padding slots).
+// route_kernel, one CTA per `tpc` tokens (2 at decode, kRouteTokens at
+// prefill):
+//   logits   warp tasks (token, expert): the lanes stride d with batches of
+//            16-byte loads of the x row and the W_router row and reduce with
+//            a butterfly (fp32, a fixed summation order);
+//   top-k    one warp per token: the k largest logits, equal logits to the
+//            lower expert index; softmax weights, renormalised or not;
+//   ranks    each pair's rank among the CTA's pairs of the same expert in
+//            pair order (warp match + per-warp counts) and the CTA's
+//            histogram hist[cta][e];
+//   finish   the last CTA to finish (atomic ticket after a fence) turns the
+//            histograms into per-CTA base offsets with a segmented scan over
+//            CTAs, pads each expert's slot range to kSlotAlign, and writes the
+//            expert token groups.
+// permute_kernel, one warp per pair: slot = expert_off[e] + base[cta][e] +
+//   rank, so slots are ordered by (token, choice) within each expert; it
+//   records perm / slot_of and copies the x row to X_perm[slot]; extra warps
+//   zero the padding slots.
 #include "common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kRouteTokens = 32;
-constexpr int kRouteThreads = 256;
-constexpr int kRouteChunk = 32;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 constexpr int kMaxExperts = 256;
-constexpr int kPad = kRouteChunk + 1;
-
-template <typename TX>
-__device__ __forceinline__ float ldf(const TX* p) {
-  return to_f32<TX>(*p);
-}
 
 // Total order used by the top-k: larger logit first, then lower index.
 __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
-__device__ void route_scan(const Dims& dm, const Workspace& ws, int* smem_i) {
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int E = dm.E, k = dm.k, T = dm.T;
-  const int P = T * k;
-  int* cnt = smem_i;                     // [E]
-  int* poff = cnt + kMaxExperts;         // [E+1]
-  int* run = poff + kMaxExperts + 1;     // [E]
-  int* wcnt = run + kMaxExperts;         // [8][E]
+template <typename TX>
+struct XVec;
+template <>
+struct XVec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(b[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+};
+template <>
+struct XVec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float (&f)[4]) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+};
 
-  for (int e = tid; e < E; e += blockDim.x) { cnt[e] = 0; run[e] = 0; }
-  for (int i = tid; i < 8 * kMaxExperts; i += blockDim.x) wcnt[i] = 0;
-  __syncthreads();
-  for (int p = tid; p < P; p += blockDim.x) atomicAdd(&cnt[__ldcg(ws.topk_idx + p)], 1);
+// Last CTA: histograms -> base offsets, expert slot ranges, token groups.
+__device__ void route_finish(const Dims& dm, const Workspace& ws, int n_cta) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int poff[kMaxExperts + 1];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int E = dm.E, T = dm.T, k = dm.k;
+  int e_pow2 = 1;
+  while (e_pow2 < E) e_pow2 <<= 1;
+  const int parts = kThreads / e_pow2 < 32 ? kThreads / e_pow2 : 32;  // lanes per expert
+  const int e = tid / parts, part = tid % parts;
+  const bool live = e < E && tid < e_pow2 * parts;
+  const int c0 = static_cast<int>((long long)part * n_cta / parts);
+  const int c1 = static_cast<int>((long long)(part + 1) * n_cta / parts);
+  int s = 0;
+  if (live)
+    for (int c = c0; c < c1; ++c) s += __ldcg(ws.hist + (size_t)c * E + e);
+  // segmented inclusive scan over the `parts` lanes of one expert
+  int incl = s;
+  for (int o = 1; o < parts; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o, parts);
+    if ((lane % parts) >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, (lane / parts) * parts + parts - 1);
+  if (live) {
+    int run = incl - s;
+    for (int c = c0; c < c1; ++c) {
+      int* h = ws.hist + (size_t)c * E + e;
+      const int v = __ldcg(h);
+      *h = run;
+      run += v;
+    }
+    if (part == 0) cnt[e] = total;
+  }
   __syncthreads();
 
   if (tid == 0) {
     int touched = 0;
     poff[0] = 0;
-    for (int e = 0; e < E; ++e) {
-      const int me = cnt[e];
+    for (int x = 0; x < E; ++x) {
+      const int me = cnt[x];
       touched += me > 0;
-      poff[e + 1] = poff[e] + (me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+      poff[x + 1] = poff[x] + (me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
     }
     int ng = 0;
-    for (int e = 0; e < E; ++e) {
-      const int me = cnt[e];
+    for (int x = 0; x < E; ++x) {
+      const int me = cnt[x];
       if (me == 0) continue;
       const int n_g = (me + kGroupMax - 1) / kGroupMax;
       int gsz = (me + n_g - 1) / n_g;
       gsz = (gsz + 63) / 64 * 64;
       for (int g = 0; g * gsz < me && ng < dm.groups_max; ++g) {
         Group gr;
-        gr.expert = e;
-        gr.slot0 = poff[e] + g * gsz;
+        gr.expert = x;
+        gr.slot0 = poff[x] + g * gsz;
         gr.m = min(gsz, me - g * gsz);
         gr.xrow0 = gr.slot0;
         ws.groups[ng++] = gr;
       }
     }
     ws.meta[kMetaRoutedGroups] = ng;
-    for (int s = 0; s < dm.S; ++s) {
+    for (int sh = 0; sh < dm.S; ++sh) {
       const int n_g = (T + kGroupMax - 1) / kGroupMax;
       int gsz = (T + n_g - 1) / n_g;
       gsz = (gsz + 63) / 64 * 64;
       for (int g = 0; g * gsz < T && ng < dm.groups_max; ++g) {
         Group gr;
-        gr.expert = E + s;
-        gr.slot0 = dm.slots_routed + s * dm.T_pad + g * gsz;
+        gr.expert = E + sh;
+        gr.slot0 = dm.slots_routed + sh * dm.T_pad + g * gsz;
         gr.m = min(gsz, T - g * gsz);
         gr.xrow0 = g * gsz;
         ws.groups[ng++] = gr;
@@ -95,106 +143,79 @@ __device__ void route_scan(const Dims& dm, const Workspace& ws, int* smem_i) {
     ws.meta[kMetaTcCount] = 0;
   }
   __syncthreads();
-
-  // padding slots of each expert's range hold no token
-  for (int e = warp; e < E; e += blockDim.x / 32)
-    for (int s = poff[e] + cnt[e] + lane; s < poff[e + 1]; s += 32) ws.perm[s] = -1;
-
-  // stable scatter, pairs in (token, choice) order
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = 0; base < P; base += blockDim.x) {
-    const int p = base + tid;
-    const int e = p < P ? __ldcg(ws.topk_idx + p) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (e >= 0 && rank == 0) wcnt[warp * kMaxExperts + e] = __popc(peers);
-    __syncthreads();
-    if (e >= 0) {
-      int off = run[e] + rank;
-      for (int w = 0; w < warp; ++w) off += wcnt[w * kMaxExperts + e];
-      const int slot = poff[e] + off;
-      ws.perm[slot] = p / k;
-      ws.slot_of[p] = slot;
-    }
-    __syncthreads();
-    for (int e2 = tid; e2 < E; e2 += blockDim.x) {
-      int tot = 0;
-      for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
-        tot += wcnt[w * kMaxExperts + e2];
-        wcnt[w * kMaxExperts + e2] = 0;
-      }
-      run[e2] += tot;
-    }
-    __syncthreads();
-  }
-
+  for (int x = tid; x <= E; x += kThreads) ws.expert_off[x] = poff[x];
+  for (int x = tid; x < E; x += kThreads) ws.expert_cnt[x] = cnt[x];
   if (tid < kCntWords) ws.counters[tid] = 0ull;
   __syncthreads();
   if (tid == 0) {
-    ws.counters[kCntRoutedH] = (unsigned long long)P * (unsigned long long)dm.F;
+    ws.counters[kCntRoutedH] = (unsigned long long)T * k * (unsigned long long)dm.F;
     ws.counters[kCntSharedH] =
         (unsigned long long)dm.S * (unsigned long long)T * (unsigned long long)dm.Fs;
     ws.meta[kMetaDone] = 0;  // ticket counter for the next forward
   }
 }
 
+// Dot product of one token row with one router row, lanes over d in chunks
+// of 32 x VEC elements, loads issued in batches of kBatch chunks.
 template <typename TX>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(Dims dm, Workspace ws, const TX* x,
-                                                              const TX* Wr, const float* bias) {
-  __shared__ float xs[kRouteTokens * kPad];
-  __shared__ float wsm[kMaxExperts * kPad];  // reused for logits and the scan
+__device__ __forceinline__ float row_dot(const TX* a, const TX* b, int d, int lane) {
+  constexpr int VEC = XVec<TX>::N;
+  constexpr int kBatch = 8;
+  float acc = 0.f;
+  for (int c0 = lane * VEC; c0 < d; c0 += 32 * VEC * kBatch) {
+    float av[kBatch][VEC], bv[kBatch][VEC];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int c = c0 + i * 32 * VEC;
+      if (c < d) {
+        XVec<TX>::load(a + c, av[i]);
+        XVec<TX>::load(b + c, bv[i]);
+      } else {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) av[i][v] = bv[i][v] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc = fmaf(av[i][v], bv[i][v], acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+template <typename TX>
+__global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, const TX* x,
+                                                         const TX* Wr, const float* bias,
+                                                         int tpc) {
+  __shared__ float lg[kRouteTokens][kMaxExperts + 1];
+  __shared__ int sel[kRouteTokens * 16];
+  __shared__ int wcnt[kWarps][kMaxExperts];
   __shared__ int is_last;
 
-  const int tid = threadIdx.x;
-  const int tok0 = blockIdx.x * kRouteTokens;
+  grid_dep_wait();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = dm.E, d = dm.d, T = dm.T, k = dm.k;
-  const int tt = tid >> 3, eg = tid & 7;
-  const int nq = (E + 7) / 8;
+  const int tok0 = blockIdx.x * tpc;
+  const int tb = min(tpc, T - tok0);
 
-  float acc[kMaxExperts / 8];
-#pragma unroll
-  for (int q = 0; q < kMaxExperts / 8; ++q) acc[q] = 0.f;
-
-  for (int d0 = 0; d0 < d; d0 += kRouteChunk) {
-    for (int i = tid; i < kRouteTokens * kRouteChunk; i += kRouteThreads) {
-      const int t = i / kRouteChunk, c = i % kRouteChunk;
-      const int tok = tok0 + t;
-      xs[t * kPad + c] = tok < T ? ldf(x + (size_t)tok * d + d0 + c) : 0.f;
-    }
-    for (int i = tid; i < E * kRouteChunk; i += kRouteThreads) {
-      const int e = i / kRouteChunk, c = i % kRouteChunk;
-      wsm[e * kPad + c] = ldf(Wr + (size_t)e * d + d0 + c);
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kRouteChunk; ++c) {
-      const float xv = xs[tt * kPad + c];
-#pragma unroll
-      for (int q = 0; q < kMaxExperts / 8; ++q)
-        if (q < nq) acc[q] = fmaf(xv, wsm[(eg + 8 * q) * kPad + c], acc[q]);
-    }
-    __syncthreads();
-  }
-
-  // logits [32][E+1] in the (now free) W tile
-  float* lg = wsm;
-  const int lgp = E + 1;
-#pragma unroll
-  for (int q = 0; q < kMaxExperts / 8; ++q) {
-    const int e = eg + 8 * q;
-    if (q < nq && e < E) lg[tt * lgp + e] = acc[q] + (bias ? bias[e] : 0.f);
+  // ---- logits: warp tasks (token, expert), lanes over d
+  for (int task = warp; task < tb * E; task += kWarps) {
+    const int t = task / E, e = task % E;
+    const float a = row_dot<TX>(x + (size_t)(tok0 + t) * d, Wr + (size_t)e * d, d, lane);
+    if (lane == 0) lg[t][e] = a + (bias ? bias[e] : 0.f);
   }
   __syncthreads();
 
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int t = warp; t < kRouteTokens; t += kRouteThreads / 32) {
+  // ---- top-k and weights: one warp per token
+  for (int t = warp; t < tb; t += kWarps) {
     const int tok = tok0 + t;
-    if (tok >= T) break;
     float v[kMaxExperts / 32];
 #pragma unroll
     for (int j = 0; j < kMaxExperts / 32; ++j) {
       const int e = lane + 32 * j;
-      v[j] = e < E ? lg[t * lgp + e] : -INFINITY;
+      v[j] = e < E ? lg[t][e] : -INFINITY;
     }
     float mx = -INFINITY;
 #pragma unroll
@@ -234,10 +255,32 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Dims dm, Workspace
     if (lane < k) {
       ws.topk_idx[tok * k + lane] = my_e;
       ws.topk_w[tok * k + lane] = dm.renorm ? my_p / psum : my_p;
+      sel[t * k + lane] = my_e;
     }
   }
+  for (int i = tid; i < kWarps * kMaxExperts; i += kThreads) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
 
-  // the last CTA to finish builds the slot layout for the whole batch
+  // ---- stable ranks within the CTA and the CTA's histogram (pairs in order)
+  const int np = tb * k;  // <= kRouteTokens * 16 = kThreads
+  const int e = tid < np ? sel[tid] : -1;
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && rank == 0) wcnt[warp][e] = __popc(peers);
+  __syncthreads();
+  if (e >= 0) {
+    int r = rank;
+    for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+    ws.rank_cta[tok0 * k + tid] = r;
+  }
+  for (int x2 = tid; x2 < E; x2 += kThreads) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += wcnt[w][x2];
+    ws.hist[(size_t)blockIdx.x * E + x2] = c;
+  }
+
+  // ---- the last CTA to finish builds the slot layout for the whole batch
   __syncthreads();
   if (tid == 0) {
     __threadfence();
@@ -247,55 +290,72 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Dims dm, Workspace
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  route_scan(dm, ws, reinterpret_cast<int*>(wsm));
+  route_finish(dm, ws, gridDim.x);
 }
 
 template <typename TX>
-__global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, const TX* x) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, const TX* x,
+                                                      int tpc) {
+  grid_dep_wait();
+  const int item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= __ldcg(ws.meta + kMetaSlotsUsed)) return;
-  const int tok = ws.perm[warp];
+  const int k = dm.k, E = dm.E, P = dm.T * dm.k;
   constexpr int kVec = 16 / sizeof(TX);
   const int nv = dm.d / kVec;
-  uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)warp * dm.d);
-  if (tok < 0) {
-    for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-    return;
+  if (item < P) {
+    const int t = item / k;
+    const int e = __ldcg(ws.topk_idx + item);
+    const int cta = t / tpc;
+    const int slot = __ldcg(ws.expert_off + e) + __ldcg(ws.hist + (size_t)cta * E + e) +
+                     __ldcg(ws.rank_cta + item);
+    if (lane == 0) {
+      ws.perm[slot] = t;
+      ws.slot_of[item] = slot;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * dm.d);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * dm.d);
+    for (int i = lane; i < nv; i += 32) dst[i] = __ldg(src + i);
+  } else if (item < P + E) {
+    const int e = item - P;
+    const int s0 = __ldcg(ws.expert_off + e) + __ldcg(ws.expert_cnt + e);
+    const int s1 = __ldcg(ws.expert_off + e + 1);
+    for (int s = s0; s < s1; ++s) {
+      if (lane == 0) ws.perm[s] = -1;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)s * dm.d);
+      for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+    }
   }
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * dm.d);
-  for (int i = lane; i < nv; i += 32) dst[i] = __ldg(src + i);
 }
 
 }  // namespace
 
-static_assert(sizeof(float) * kMaxExperts * kPad >=
-                  sizeof(int) * (3 * kMaxExperts + 1 + 8 * kMaxExperts),
-              "scan scratch must fit in the W tile");
+// Tokens per router CTA: few at decode so that the (token, expert) dot
+// products spread over many SMs, more at prefill to keep the per-CTA
+// histograms short.
+int route_tokens_per_cta(int T) { return T <= 256 ? 2 : kRouteTokens; }
 
 cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, const void* Wr,
                          const float* bias, bool bf16, cudaStream_t st) {
-  const int grid = (dm.T + kRouteTokens - 1) / kRouteTokens;
+  const int tpc = route_tokens_per_cta(dm.T);
+  const int grid = (dm.T + tpc - 1) / tpc;
   if (bf16)
-    route_kernel<__nv_bfloat16><<<grid, kRouteThreads, 0, st>>>(
-        dm, ws, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
-        bias);
-  else
-    route_kernel<float><<<grid, kRouteThreads, 0, st>>>(
-        dm, ws, static_cast<const float*>(x), static_cast<const float*>(Wr), bias);
-  return cudaGetLastError();
+    return launch_k(route_kernel<__nv_bfloat16>, grid, kThreads, 0, st, dm, ws,
+                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
+                    bias, tpc);
+  return launch_k(route_kernel<float>, grid, kThreads, 0, st, dm, ws,
+                  static_cast<const float*>(x), static_cast<const float*>(Wr), bias, tpc);
 }
 
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st) {
-  const int rows = dm.slots_routed;
-  const int grid = (rows + 7) / 8;
+  const int items = dm.T * dm.k + dm.E;
+  const int grid = (items + 7) / 8;
+  const int tpc = route_tokens_per_cta(dm.T);
   if (bf16)
-    permute_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(dm, ws,
-                                                        static_cast<const __nv_bfloat16*>(x));
-  else
-    permute_kernel<float><<<grid, 256, 0, st>>>(dm, ws, static_cast<const float*>(x));
-  return cudaGetLastError();
+    return launch_k(permute_kernel<__nv_bfloat16>, grid, 256, 0, st, dm, ws,
+                    static_cast<const __nv_bfloat16*>(x), tpc);
+  return launch_k(permute_kernel<float>, grid, 256, 0, st, dm, ws, static_cast<const float*>(x),
+                  tpc);
 }
 
 }  // namespace moe

@@ -37,7 +37,7 @@ def _calibrated(dw, x, q, shared_q=None):
 def _check(layer, dw, x, tau, ts, dtype, dense=False, top_k=None):
     gpu = run_gpu(layer, dw, x, tau, ts, top_k=top_k)
     ref = oracle_forward(dw, x, tau, ts, dense=dense, top_k=top_k)
-    info = compare(gpu, ref, tau, ts, dtype, dense=dense)
+    info = compare(gpu, ref, tau, ts, dtype, dw=dw, dense=dense)
     assert layer.status() == 0
     return gpu, ref, info
 
