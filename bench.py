@@ -284,6 +284,33 @@ def run_ours(args, world, rank, local):
         L.set_timing(0)
         return per
 
+    def per_batch_us(L):
+        """Layer latency per decode batch: K replays of a graph of one forward."""
+        res = []
+        for x, o in zip(xs, outs):
+            def one():
+                L.forward(x, W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau,
+                          sh.top_k, router_bias=W["router_bias"], out=o)
+            one()
+            torch.cuda.synchronize(dev)
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                one()
+            for _ in range(args.warmup):
+                g.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            res.append(1e3 * a.elapsed_time(b) / args.steps)
+            del g
+        return res
+
     sparse = make("auto")
     for _ in range(args.warmup):
         step(sparse)
@@ -299,6 +326,7 @@ def run_ours(args, world, rank, local):
     ms_sparse = max_over_ranks(world, ms_sparse, local)
     launches = launches_per_step * args.steps
     per_fwd = kernel_times(sparse)
+    lat_sparse = per_batch_us(sparse)
     tok_step = sum(tokens)
     value = tok_step * args.steps * world / (ms_sparse / 1e3)
 
@@ -312,6 +340,7 @@ def run_ours(args, world, rank, local):
 
     dense_line = None
     per_dense = []
+    lat_dense = [None] * len(tokens)
     if not args.no_dense:
         dense = make("dense")
         for _ in range(args.warmup):
@@ -320,6 +349,7 @@ def run_ours(args, world, rank, local):
         ms_dense, _ = timed(dense, g_dense)
         ms_dense = max_over_ranks(world, ms_dense, local)
         per_dense = kernel_times(dense)
+        lat_dense = per_batch_us(dense)
         dense_line = {"value": tok_step * args.steps * world / (ms_dense / 1e3),
                       "ms_per_step": ms_dense / args.steps}
         del g_dense
@@ -355,6 +385,10 @@ def run_ours(args, world, rank, local):
         sp = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
         per_T.append({
             "T": T, "sparsity": round(sp, 4), "experts_touched": touched,
+            "layer_us_graph": round(lat_sparse[i], 2),
+            "dense_layer_us_graph": None if lat_dense[i] is None else round(lat_dense[i], 2),
+            "speedup_vs_dense_graph": None if lat_dense[i] is None else
+            round(lat_dense[i] / lat_sparse[i], 3),
             "down_rows_read": st["down_rows_read"],
             "down_rows_dense": touched * sh.d_ff,
             "groups": {"gemv": st["n_groups_gemv"], "tc_gather": st["n_groups_tc_gather"],

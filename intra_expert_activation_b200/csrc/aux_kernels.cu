@@ -1,12 +1,11 @@
 // Small kernels between the big ones:
-//  union_scan   per expert token group: compact the active-row union bitmap
-//               into an ordered row list, and choose the down-projection path
-//               from the group's token count and union size (the pages'
-//               sparse/dense switch by batch size [gist.science EN "Uncovering
-//               Intra-expert Activation Sparsity for Efficient
-//               Mixture-of-Expert Model Execution", Technical Summary >
-//               Methodology > System Implementation in vLLM > "Dynamic
-//               Switching"], taken per group on the device).
+//  union_scan   (gathered tensor-core mode only) per expert token group:
+//               compact the active-row union bitmap into an ordered row list
+//               and mark groups of <= kGatherMaxTokens tokens for the gathered
+//               path [gist.science EN "Uncovering Intra-expert Activation
+//               Sparsity for Efficient Mixture-of-Expert Model Execution",
+//               Technical Summary > Methodology > System Implementation in
+//               vLLM > "Fused Up-Down Projection"].
 //  combine      out[t] = sum_i w[t,i] * Y[slot(t,i)] + sum_s Y[shared slot(s,t)],
 //               in a fixed order.
 //  debug_gather routing and active bitmaps of the last forward in pair order.
@@ -17,74 +16,6 @@ namespace moe {
 namespace {
 
 constexpr int kScanThreads = 256;
-constexpr int kListMax = 2048;
-
-// Sort a list of group ids ascending in place (ids are distinct): each
-// entry's position is the number of smaller entries.
-__device__ void sort_list(int* list, int n, int* tmp) {
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int v = __ldcg(list + i);
-    int r = 0;
-    for (int j = 0; j < n; ++j) r += __ldcg(list + j) < v;
-    tmp[r] = v;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) list[i] = tmp[i];
-  __syncthreads();
-}
-
-// Last union_scan CTA: order the path lists by group id, and lay out the
-// GEMV work items: unit = (group, pass of MT tokens), item = (unit, split of
-// the union rows). Splits aim at about two items per CTA of the GEMV grid,
-// with kGemvRowsMin..kGemvRowsMax rows per item.
-__device__ void scan_finish(const Dims& dm, Workspace& ws) {
-  __shared__ int tmp[kListMax];
-  __shared__ int s_units[kListMax];
-  __shared__ int s_rows[kListMax];
-  __shared__ int total_units;
-  const int n_gemv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
-  const int n_tc = min(__ldcg(ws.meta + kMetaTcCount), kListMax);
-  sort_list(ws.gemv_list, n_gemv, tmp);
-  sort_list(ws.tc_list, n_tc, tmp);
-  const int mt = dm.no_tc ? 8 : kGemvTokens;
-  for (int i = threadIdx.x; i < n_gemv; i += blockDim.x) {
-    const int g = __ldcg(ws.gemv_list + i);
-    s_units[i] = (ws.groups[g].m + mt - 1) / mt;
-    s_rows[i] = __ldcg(ws.union_cnt + g);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int u = 0;
-    for (int i = 0; i < n_gemv; ++i) u += s_units[i];
-    total_units = u;
-  }
-  __syncthreads();
-  const int target = max(1, 4 * dm.n_sms / max(total_units, 1));
-  for (int i = threadIdx.x; i < n_gemv; i += blockDim.x) {
-    const int cnt = s_rows[i];
-    const int s_min = max(1, (cnt + kGemvRowsMax - 1) / kGemvRowsMax);
-    const int s_max = max(s_min, cnt / kGemvRowsMin);
-    tmp[i] = min(max(target, s_min), s_max);  // splits of every unit of group i
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int* item_off = ws.gemv_item_off;
-    int* unit_off = ws.gemv_item_off + dm.groups_max + 1;
-    int units = 0, items = 0;
-    for (int i = 0; i < n_gemv; ++i) {
-      unit_off[i] = units;
-      item_off[i] = items;
-      units += s_units[i];
-      items += s_units[i] * tmp[i];
-    }
-    unit_off[n_gemv] = units;
-    item_off[n_gemv] = items;
-    ws.meta[kMetaGemvItems] = items;
-    ws.meta[kMetaGemvUnits] = units;
-    ws.meta[kMetaScanDone] = 0;
-  }
-}
-
 __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Workspace ws) {
   grid_dep_wait();
   const int g = blockIdx.x;
@@ -132,54 +63,16 @@ __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Works
     __syncthreads();
   }
 
-  __shared__ int is_last;
   if (threadIdx.x == 0) {
+    // gathered rows for groups of <= kGatherMaxTokens tokens, all rows above
     const int cnt = carry;
-    const int m = gr.m;
-    int path;
-    if (dm.no_tc || dm.mode == kModeGemv) {
-      path = kPathGemv;
-    } else if (dm.mode == kModeDense) {
-      path = m <= dm.gemv_max ? kPathGemv : kPathTcAll;
-    } else if (dm.mode == kModeTc) {
-      path = m <= kGatherMaxTokens ? kPathTcGather : kPathTcAll;
-    } else if (dm.mode == kModeTcAll) {
-      path = kPathTcAll;
-    } else {
-      if (m <= dm.gemv_max)
-        path = kPathGemv;
-      else if (m <= kGatherMaxTokens && cnt <= dm.gather_density * F_e)
-        path = kPathTcGather;
-      else
-        path = kPathTcAll;
-    }
+    const int path = gr.m <= kGatherMaxTokens ? kPathTcGather : kPathTcAll;
     ws.union_cnt[g] = cnt;
     ws.group_path[g] = path;
-    const int li = atomicAdd(ws.meta + (path == kPathGemv ? kMetaGemvCount : kMetaTcCount), 1);
-    (path == kPathGemv ? ws.gemv_list : ws.tc_list)[li] = g;
     atomicAdd(ws.counters + kCntDownRows,
               static_cast<unsigned long long>(path == kPathTcAll ? F_e : cnt));
-    atomicAdd(ws.counters + (path == kPathGemv ? kCntGemv
-                             : path == kPathTcGather ? kCntTcGather : kCntTcAll), 1ull);
-    is_last = path == kPathGemv;  // reused below: zero this group's Y rows
+    if (path == kPathTcGather) atomicAdd(ws.counters + kCntTcGather, 1ull);
   }
-  __syncthreads();
-  if (is_last) {
-    // GEMV splits add into Y: start from zero
-    float4* yz = reinterpret_cast<float4*>(ws.y + static_cast<size_t>(gr.slot0) * dm.d);
-    const int n4 = gr.m * dm.d / 4;
-    for (int q = threadIdx.x; q < n4; q += blockDim.x) yz[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const int ticket = atomicAdd(ws.meta + kMetaScanDone, 1);
-    is_last = ticket == __ldcg(ws.meta + kMetaGroups) - 1;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  scan_finish(dm, ws);
 }
 
 template <typename TX>

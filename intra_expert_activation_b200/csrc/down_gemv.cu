@@ -1,6 +1,6 @@
 // Down projection on CUDA cores for expert token groups with few tokens
 // (decode): stream only the W_down rows in the group's active-neuron union
-// with 128-bit loads and multiply them by the tokens' h values.
+// and multiply them by the tokens' h values.
 //
 // This is the low-batch side of the pages' batch-size switch [gist.science
 // EN "Uncovering Intra-expert Activation Sparsity for Efficient
@@ -10,35 +10,42 @@
 // cost is the bytes of the rows it reads ["Fused Up-Down Projection": only
 // the active neurons' weights are fetched].
 //
-// Work: a unit is (group, pass of up to MT tokens); its union rows are cut
-// into splits, and a work item is one split of one unit over all d_model
-// columns. Persistent CTAs of 16 warps (one per SM) stride over the items. A
-// CTA first stages the item's row ids and the tokens' h values in shared
-// memory; then each warp owns one 512-byte column slice and streams the
-// item's rows through its own ring of shared-memory stages with cp.async
-// (16 bytes per lane per row; kStages x kBatch rows in flight per warp, with
-// no registers held by data in flight), and multiplies each landed row
-// segment by the tokens' h values into fp32 registers. Each lane copies and
-// later reads back exactly its own 16 bytes, so a wait on the lane's own copy
-// group is all the synchronisation the ring needs. An item that is a whole
-// unit stores its result into Y[slot][columns]; a split adds its partial into
-// Y (zeroed by the union scan) with vector fp32 atomics, so the splits of a
-// unit are summed in arrival order: results agree to fp32 rounding, not
-// bitwise, between runs on this path.
+// Work: a unit is (group, pass of up to MT tokens); its neuron range is cut
+// into splits of whole union-bitmap words, and a work item is one split of
+// one unit over all d_model columns, described by a GemvItem the router
+// wrote. One CTA per SM: 16 streaming warps and one scheduler warp. The
+// scheduler takes the next item from an atomic queue and compacts its
+// union-bitmap words into an ordered row list (double-buffered) while the
+// streaming warps work on the current item, so items are balanced
+// dynamically and their set-up is hidden. Each streaming warp owns one
+// 512-byte column slice and streams the item's rows through its own ring of
+// shared-memory stages with cp.async: per row 16 bytes of W_down per lane and
+// the tokens' h values (one lane), kStages x kBatch rows in flight per warp
+// with no registers held by data in flight; landed segments are multiplied
+// by h with packed fp32x2 FMAs. An item that is a whole unit stores its
+// result into Y[slot][columns]; a split adds its partial into Y (zeroed by the
+// router) with vector fp32 atomics, so the splits of a unit are summed in
+// arrival order: results agree to fp32 rounding, not bitwise, between runs on
+// this path.
 #include "common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
+constexpr int kStreamWarps = 16;
+constexpr int kThreads = (kStreamWarps + 1) * 32;  // + the scheduler warp
 constexpr int kBatch = 8;    // rows per stage
 constexpr int kStages = 3;   // stages per warp ring
-constexpr int kWarpRing = kStages * kBatch * 32 * 16;  // bytes per warp ring
+constexpr int kHBytes = 32;  // h bytes kept per row (MT x element: 8 for bf16, 32 for fp32)
+constexpr int kStageBytes = kBatch * 512 + kBatch * kHBytes;
+constexpr int kWarpRing = kStages * kStageBytes;  // bytes per warp ring
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
@@ -48,193 +55,238 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename TW>
-struct Vec;
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ static void unpack(const uint4& u, float (&f)[8]) {
-    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 t = __bfloat1622float2(b[i]);
-      f[2 * i] = t.x;
-      f[2 * i + 1] = t.y;
-    }
-  }
-};
-template <>
-struct Vec<float> {
-  static constexpr int N = 4;
-  __device__ static void unpack(const uint4& u, float (&f)[4]) {
-    f[0] = __uint_as_float(u.x);
-    f[1] = __uint_as_float(u.y);
-    f[2] = __uint_as_float(u.z);
-    f[3] = __uint_as_float(u.w);
-  }
-};
-
-// h of MT consecutive slots of one neuron row of H^T; entries past mt are 0.
-template <typename TW, int MT>
-__device__ __forceinline__ void load_h(const TW* p, int mt, float (&h)[MT]) {
-  if constexpr (sizeof(TW) == 2) {
-    static_assert(MT == 4 || MT == 8, "bf16 h vector");
-    if constexpr (MT == 4) {
-      const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
-      const float2 a = __bfloat1622float2(b[0]), c = __bfloat1622float2(b[1]);
-      h[0] = a.x; h[1] = a.y; h[2] = c.x; h[3] = c.y;
-    } else {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-      float f[8];
-      Vec<__nv_bfloat16>::unpack(u, f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) h[i] = f[i];
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < MT; i += 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(p + i));
-      h[i] = v.x; h[i + 1] = v.y; h[i + 2] = v.z; h[i + 3] = v.w;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < MT; ++i)
-    if (i >= mt) h[i] = 0.f;
-}
-
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
                "f"(d)
                : "memory");
 }
 
+// Packed pair of fp32 values and d = a * b + d on both lanes of the pair.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
+// A landed 16-byte weight segment as packed fp32 pairs.
+template <typename TW>
+struct Seg;
+template <>
+struct Seg<__nv_bfloat16> {
+  static constexpr int VEC = 8, NP = 4;
+  __device__ static void pairs(const uint4& u, uint64_t (&w)[4]) {
+    const uint32_t q[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)  // bf16 pair -> (low << 16, high & 0xffff0000) as fp32
+      w[i] = pack2(__uint_as_float(q[i] << 16), __uint_as_float(q[i] & 0xffff0000u));
+  }
+};
+template <>
+struct Seg<float> {
+  static constexpr int VEC = 4, NP = 2;
+  __device__ static void pairs(const uint4& u, uint64_t (&w)[2]) {
+    w[0] = pack2(__uint_as_float(u.x), __uint_as_float(u.y));
+    w[1] = pack2(__uint_as_float(u.z), __uint_as_float(u.w));
+  }
+};
+
+// Token t's h of a row as landed in the ring, broadcast to a packed pair.
+template <typename TW>
+__device__ __forceinline__ uint64_t h_pair(const uint8_t* p, int t) {
+  float h;
+  if constexpr (sizeof(TW) == 2)
+    h = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(p)[t]) << 16);
+  else
+    h = reinterpret_cast<const float*>(p)[t];
+  return pack2(h, h);
+}
+
+struct Staged {
+  GemvItem it;
+  int item;  // index, or >= n_items when the queue is empty
+  int n;     // rows
+};
+
+// One streaming warp: rows of the staged item through its cp.async ring,
+// MTE tokens accumulated in packed fp32 pairs; stores or adds mt results.
+template <typename TW, int MT, int MTE>
+__device__ __forceinline__ void stream_rows(const char* Wb, const char* hb, float* y, int d,
+                                            uint32_t w_stride, uint32_t h_stride,
+                                            const int* srow, int n, int rstride, int mt,
+                                            bool whole,
+                                            uint8_t* ring, uint32_t ring_s, int lane) {
+  constexpr int NP = Seg<TW>::NP;
+  constexpr int HB = MT * static_cast<int>(sizeof(TW));
+  const int nb = (n + kBatch - 1) / kBatch;
+  auto issue = [&](int b) {
+    if (b < nb) {
+      const uint32_t st = ring_s + (b % kStages) * kStageBytes;
+      const int q0 = b * kBatch;
+      const int cnt = min(kBatch, n - q0);
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) {
+        if (r < cnt) {
+          const uint32_t j = static_cast<uint32_t>(srow[(q0 + r) * rstride]);
+          cp_async16(st + r * 512 + lane * 16, Wb + j * w_stride);
+          const uint32_t hdst = st + kBatch * 512 + r * kHBytes;
+          if constexpr (HB == 8) {
+            if (lane == 0) cp_async8(hdst, hb + j * h_stride);
+          } else {
+            if (lane * 16 < HB) cp_async16(hdst + lane * 16, hb + j * h_stride + lane * 16);
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  uint64_t acc[MTE][NP];
+#pragma unroll
+  for (int t = 0; t < MTE; ++t)
+#pragma unroll
+    for (int v = 0; v < NP; ++v) acc[t][v] = 0ull;
+#pragma unroll
+  for (int b = 0; b < kStages - 1; ++b) issue(b);
+  for (int b = 0; b < nb; ++b) {
+    issue(b + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();  // the h slots were copied by other lanes
+    const uint8_t* st = ring + (b % kStages) * kStageBytes;
+    const int cnt = min(kBatch, n - b * kBatch);
+#pragma unroll
+    for (int r = 0; r < kBatch; ++r) {
+      if (r < cnt) {
+        uint64_t w[NP];
+        Seg<TW>::pairs(*reinterpret_cast<const uint4*>(st + r * 512 + lane * 16), w);
+        const uint8_t* hp = st + kBatch * 512 + r * kHBytes;
+#pragma unroll
+        for (int t = 0; t < MTE; ++t) {
+          const uint64_t h2 = h_pair<TW>(hp, t);
+#pragma unroll
+          for (int v = 0; v < NP; ++v) fma2(acc[t][v], h2, w[v]);
+        }
+      }
+    }
+    __syncwarp();  // every lane has read the stage before it is refilled
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int t = 0; t < MTE; ++t) {
+    if (t < mt) {
+      float* yt = y + static_cast<size_t>(t) * d;
+#pragma unroll
+      for (int v = 0; v < NP; v += 2) {
+        const float2 a = unpack2(acc[t][v]), c = unpack2(acc[t][v + 1]);
+        if (whole)
+          *reinterpret_cast<float4*>(yt + 2 * v) = make_float4(a.x, a.y, c.x, c.y);
+        else
+          red_add_v4(yt + 2 * v, a.x, a.y, c.x, c.y);
+      }
+    }
+  }
+}
+
 template <typename TW, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     down_gemv_kernel(Dims dm, Workspace ws, const TW* __restrict__ Wd,
                      const TW* __restrict__ Wds) {
-  constexpr int VEC = Vec<TW>::N;
+  constexpr int VEC = Seg<TW>::VEC;
   constexpr int SW = 32 * VEC;  // columns per slice: one 512-byte row segment
+  static_assert(MT * sizeof(TW) <= kHBytes, "h slot");
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* rings = smem;                                          // [kWarps][kWarpRing]
-  int* srow = reinterpret_cast<int*>(smem + kWarps * kWarpRing);  // [kGemvRowsMax]
-  float* sh = reinterpret_cast<float*>(srow + kGemvRowsMax);      // [kGemvRowsMax][MT]
+  uint8_t* rings = smem;                                             // [16][kWarpRing]
+  int* srow = reinterpret_cast<int*>(smem + kStreamWarps * kWarpRing);  // [2][kGemvRowsMax]
+  __shared__ Staged staged[2];
 
   grid_dep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int n_slices = d / SW;
-  const int n_phase = n_slices >= kWarps ? 1 : kWarps / n_slices;  // warps per slice
+  const int n_phase = n_slices >= kStreamWarps ? 1 : kStreamWarps / n_slices;  // warps per slice
   const int n_tasks = n_slices * n_phase;
-  const int n_list = __ldcg(ws.meta + kMetaGemvCount);
   const int n_items = __ldcg(ws.meta + kMetaGemvItems);
-  const int* item_off = ws.gemv_item_off;
-  const int* unit_off = ws.gemv_item_off + dm.groups_max + 1;
   const size_t ld = static_cast<size_t>(dm.slots_total);
   const TW* ht = static_cast<const TW*>(ws.ht);
-  uint8_t* ring = rings + warp * kWarpRing;
-  const uint32_t ring_s = smem_u32(ring) + lane * 16;
 
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    // listed group i with item_off[i] <= item < item_off[i + 1]
-    int lo_i = 0, hi_i = n_list;
-    while (hi_i - lo_i > 1) {
-      const int mid = (lo_i + hi_i) >> 1;
-      if (__ldcg(item_off + mid) <= item) lo_i = mid; else hi_i = mid;
+  // scheduler warp: take the next item and stage its rows into buffer b
+  auto fetch = [&](int b) {
+    int idx = 0;
+    if (lane == 0) idx = atomicAdd(ws.meta + kMetaGemvNext, 1);
+    idx = __shfl_sync(0xffffffffu, idx, 0);
+    if (idx >= n_items) {
+      if (lane == 0) staged[b].item = n_items;
+      return;
     }
-    const int i = lo_i;
-    const int g = __ldcg(ws.gemv_list + i);
-    const Group gr = ws.groups[g];
-    const int units_i = __ldcg(unit_off + i + 1) - __ldcg(unit_off + i);
-    const int splits = (__ldcg(item_off + i + 1) - __ldcg(item_off + i)) / units_i;
-    const int local = item - __ldcg(item_off + i);
-    const int split = local % splits, pass = local / splits;
-    const int tp = pass * MT;
-    const int mt = min(MT, gr.m - tp);
-    const int cnt = __ldcg(ws.union_cnt + g);
-    const int lo = static_cast<int>(static_cast<long long>(split) * cnt / splits);
-    const int n = static_cast<int>(static_cast<long long>(split + 1) * cnt / splits) - lo;
-
-    // stage the item's rows and h values (fp32, zero past mt)
-    const int* rows = ws.union_rows + static_cast<size_t>(g) * dm.F_max + lo;
-    const TW* hcol = ht + gr.slot0 + tp;
-    for (int r = threadIdx.x; r < n; r += kThreads) {
-      const int j = __ldcg(rows + r);
-      srow[r] = j;
-      float hv[MT];
-      load_h<TW, MT>(hcol + static_cast<size_t>(j) * ld, mt, hv);
+    const GemvItem it = ws.gemv_items[idx];
+    const int nw = it.w1 - it.w0;  // <= kGemvWordsMax <= 32
+    const uint32_t bits =
+        lane < nw ? __ldcg(ws.union_bits + static_cast<size_t>(it.g) * dm.fw + it.w0 + lane) : 0u;
+    const int c = __popc(bits);
+    int incl = c;
 #pragma unroll
-      for (int t = 0; t < MT; ++t) sh[r * MT + t] = hv[t];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    __syncthreads();
+    int* rows = srow + b * kGemvRowsMax;
+    int pos = incl - c;
+    uint32_t bb = bits;
+    const int base = 32 * (it.w0 + lane);
+    while (bb) {
+      rows[pos++] = base + __ffs(bb) - 1;
+      bb &= bb - 1;
+    }
+    if (lane == 31) {
+      staged[b].it = it;
+      staged[b].n = incl;
+      staged[b].item = idx;
+      atomicAdd(ws.counters + kCntDownRows, static_cast<unsigned long long>(incl));
+    }
+  };
 
-    const bool shared = gr.expert >= dm.E;
-    const int F_e = shared ? dm.Fs : dm.F;
-    const TW* Wbase = shared ? Wds + static_cast<size_t>(gr.expert - dm.E) * F_e * d
-                             : Wd + static_cast<size_t>(gr.expert) * F_e * d;
-    float* y = ws.y + static_cast<size_t>(gr.slot0 + tp) * d;
-    for (int task = warp; task < n_tasks; task += kWarps) {
-      const int slice = task % n_slices, phase = task / n_slices;
-      const int col = slice * SW + lane * VEC;
-      const TW* W = Wbase + col;
-      // this warp's rows: p = phase + n_phase * q, q < nq
-      const int nq = n > phase ? (n - phase + n_phase - 1) / n_phase : 0;
-      const int nb = (nq + kBatch - 1) / kBatch;
-      auto issue = [&](int b) {
-        if (b < nb) {
-          const uint32_t dst = ring_s + (b % kStages) * (kBatch * 512);
-#pragma unroll
-          for (int r = 0; r < kBatch; ++r) {
-            const int q = b * kBatch + r;
-            if (q < nq)
-              cp_async16(dst + r * 512, W + static_cast<size_t>(srow[phase + n_phase * q]) * d);
-          }
-        }
-        cp_async_commit();
-      };
-      float acc[MT][VEC];
-#pragma unroll
-      for (int t = 0; t < MT; ++t)
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[t][v] = 0.f;
-#pragma unroll
-      for (int b = 0; b < kStages - 1; ++b) issue(b);
-      for (int b = 0; b < nb; ++b) {
-        issue(b + kStages - 1);
-        cp_async_wait<kStages - 1>();
-        const uint8_t* src = ring + (b % kStages) * (kBatch * 512) + lane * 16;
-#pragma unroll
-        for (int r = 0; r < kBatch; ++r) {
-          const int q = b * kBatch + r;
-          if (q < nq) {
-            const uint4 wv = *reinterpret_cast<const uint4*>(src + r * 512);
-            float w[VEC];
-            Vec<TW>::unpack(wv, w);
-            const float* hq = sh + (phase + n_phase * q) * MT;
-#pragma unroll
-            for (int t = 0; t < MT; ++t) {
-              const float h = hq[t];
-#pragma unroll
-              for (int v = 0; v < VEC; ++v) acc[t][v] = fmaf(h, w[v], acc[t][v]);
-            }
-          }
-        }
-      }
-      cp_async_wait<0>();
-      const bool whole = splits == 1 && n_phase == 1;
-#pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        if (t < mt) {
-          float* yt = y + static_cast<size_t>(t) * d + col;
-#pragma unroll
-          for (int v = 0; v < VEC; v += 4) {
-            if (whole)
-              *reinterpret_cast<float4*>(yt + v) =
-                  make_float4(acc[t][v], acc[t][v + 1], acc[t][v + 2], acc[t][v + 3]);
-            else
-              red_add_v4(yt + v, acc[t][v], acc[t][v + 1], acc[t][v + 2], acc[t][v + 3]);
-          }
-        }
+  if (warp == kStreamWarps) fetch(0);
+  __syncthreads();
+  for (int cur = 0;; cur ^= 1) {
+    if (staged[cur].item >= n_items) break;
+    if (warp == kStreamWarps) {
+      fetch(cur ^ 1);
+    } else {
+      const GemvItem it = staged[cur].it;
+      const int n = staged[cur].n;
+      const int* rows = srow + cur * kGemvRowsMax;
+      const bool shared = it.expert >= dm.E;
+      const int F_e = shared ? dm.Fs : dm.F;
+      const TW* Wbase = shared ? Wds + static_cast<size_t>(it.expert - dm.E) * F_e * d
+                               : Wd + static_cast<size_t>(it.expert) * F_e * d;
+      float* y = ws.y + static_cast<size_t>(it.slot) * d;
+      const bool whole = it.whole && n_phase == 1;
+      const uint32_t w_stride = d * sizeof(TW), h_stride = ld * sizeof(TW);
+      uint8_t* ring = rings + warp * kWarpRing;
+      const uint32_t ring_s = smem_u32(ring);
+      for (int task = warp; task < n_tasks; task += kStreamWarps) {
+        const int slice = task % n_slices, phase = task / n_slices;
+        const int col = slice * SW + lane * VEC;
+        // this warp's rows: phase, phase + n_phase, ...
+        const int* wrows = rows + phase;
+        const int nq = n > phase ? (n - phase + n_phase - 1) / n_phase : 0;
+        const char* Wb = reinterpret_cast<const char*>(Wbase + col);
+        const char* hb = reinterpret_cast<const char*>(ht + it.slot);
+        if (it.mt <= 1)
+          stream_rows<TW, MT, 1>(Wb, hb, y + col, d, w_stride, h_stride, wrows, nq, n_phase,
+                                 it.mt, whole, ring, ring_s, lane);
+        else if (it.mt <= 2 && MT > 2)
+          stream_rows<TW, MT, 2>(Wb, hb, y + col, d, w_stride, h_stride, wrows, nq, n_phase,
+                                 it.mt, whole, ring, ring_s, lane);
+        else
+          stream_rows<TW, MT, MT>(Wb, hb, y + col, d, w_stride, h_stride, wrows, nq, n_phase,
+                                  it.mt, whole, ring, ring_s, lane);
       }
     }
     __syncthreads();
@@ -243,10 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t down_gemv_smem_bytes(bool bf16) {
-  const int mt = bf16 ? kGemvTokens : 8;
-  return static_cast<size_t>(kWarps) * kWarpRing + sizeof(int) * kGemvRowsMax +
-         sizeof(float) * kGemvRowsMax * mt;
+size_t down_gemv_smem_bytes(bool) {
+  return static_cast<size_t>(kStreamWarps) * kWarpRing + 2 * sizeof(int) * kGemvRowsMax;
 }
 
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
@@ -263,7 +313,7 @@ cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = n_sms;  // one 16-warp CTA per SM
+  const int grid = n_sms;  // one CTA per SM
   if (bf16)
     return launch_k(down_gemv_kernel<__nv_bfloat16, kGemvTokens>, grid, kThreads,
                     down_gemv_smem_bytes(true), st, dm, ws,

@@ -44,24 +44,36 @@ constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
 constexpr int kDownSlice = 128;     // d_model columns per down TC tile (M)
 constexpr int kKBlock = 64;         // K elements per pipeline stage (128 B of bf16)
 constexpr int kRouteTokens = 16;    // tokens per router CTA
-constexpr int kGemvRowsMax = 768;   // union rows per GEMV work item at most
-constexpr int kGemvRowsMin = 32;    // ... and at least (unless the union is smaller)
+constexpr int kGemvWordsMax = 24;   // bitmap words (32 neurons each) per GEMV work item
+constexpr int kGemvRowsMax = 32 * kGemvWordsMax;
+constexpr int kListMax = 2048;      // expert token groups per forward at most
 constexpr int kGemvTokens = 4;      // tokens per GEMV unit (bf16); fp32 uses 8
 
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
             kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
-            kMetaScanDone = 7, kMetaGemvItems = 8, kMetaGemvUnits = 9, kMetaWords = 16 };
+            kMetaGemvItems = 8, kMetaGemvNext = 9, kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
-               kCntTcGather = 4, kCntTcAll = 5, kCntRoutedH = 6, kCntSharedH = 7,
+               kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
                kCntWords = 8 };
 
 enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3 };
 
 // Requested path (mirrors moe_path in the public header).
 enum Mode { kModeAuto = 0, kModeDense = 1, kModeGemv = 2, kModeTc = 3, kModeTcAll = 4 };
+
+// One GEMV work item: a split of a group's union rows for one pass of tokens.
+struct GemvItem {
+  int32_t g;       // group
+  int32_t expert;  // expert of the group (E + s for shared expert s)
+  int32_t slot;    // first slot of the pass (group slot0 + pass * MT)
+  int32_t mt;      // tokens in the pass
+  int32_t w0, w1;  // union bitmap words [w0, w1): neurons 32*w0 .. 32*w1-1
+  int32_t whole;   // 1: the item is the whole unit (plain store), 0: atomic add
+  int32_t pad;
+};
 
 // One expert token group: up to kGroupMax consecutive slots of one expert.
 struct Group {
@@ -84,6 +96,7 @@ struct Dims {
   float gather_density;
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device
+  int gemv_items_max; // capacity of gemv_items
 };
 
 struct Workspace {
@@ -105,7 +118,8 @@ struct Workspace {
   int* union_cnt;               // [groups_max]
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
   int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
-  int* gemv_item_off;           // [groups_max+1] first GEMV work item of each listed group
+  GemvItem* gemv_items;         // [gemv_items_max] work items of the GEMV path
+  int* y_zero;                  // [E+1] 1: expert's Y rows (last: shared experts') start at zero
 
   uint32_t* act_bits;           // [slots_total][fw] or null (debug off)
   void* xperm;                  // [slots_routed][d] activations gathered by slot
@@ -144,6 +158,8 @@ struct DownTcParams {
 
 cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, const void* Wr,
                          const float* bias, bool bf16, cudaStream_t st);
+// True when one CTA does routing and the permute copies (launch_permute is then skipped).
+bool route_is_small(const Dims& dm);
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st);
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);

@@ -90,8 +90,8 @@ struct Layout {
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bGemvItemOff, bActBits,
-           bXperm, bHt, bY, bCount };
+           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bGemvItems, bYZero,
+           bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   if (!d) { err = "desc is NULL"; return MOE_ERR_INVALID; }
@@ -157,6 +157,15 @@ Layout make_layout(const moe_sparse_desc* d) {
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
   c.gather_density = d->gather_max_density;
   c.no_tc = bf16 ? 0 : 1;
+  {
+    // GEMV items: each unit has max(target, ceil(words / kGemvWordsMax)) splits at
+    // most, and units * target <= max(units, 2 * SMs) (SMs <= 1024 assumed here)
+    const int mt = bf16 ? moe::kGemvTokens : 8;
+    const long long units = ((long long)P + (long long)c.S * c.T) / mt + c.groups_max;
+    const long long per_unit = (c.F_max / 32 + moe::kGemvWordsMax - 1) / moe::kGemvWordsMax;
+    c.gemv_items_max =
+        (int)std::min<long long>(units * per_unit + std::max(units, 2048ll), INT32_MAX);
+  }
 
   const size_t es = bf16 ? 2 : 4;
   size_t sz[bCount];
@@ -178,7 +187,8 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bUnionCnt] = sizeof(int) * c.groups_max;
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
-  sz[bGemvItemOff] = sizeof(int) * 2 * (size_t)(c.groups_max + 1);
+  sz[bGemvItems] = sizeof(moe::GemvItem) * (size_t)c.gemv_items_max;
+  sz[bYZero] = sizeof(int) * (c.E + 1);
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;
   sz[bXperm] = es * (size_t)c.slots_routed * c.d;
   sz[bHt] = es * (size_t)c.F_max * c.slots_total;
@@ -355,7 +365,8 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.union_cnt = reinterpret_cast<int*>(b + o[bUnionCnt]);
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
-  w.gemv_item_off = reinterpret_cast<int*>(b + o[bGemvItemOff]);
+  w.gemv_items = reinterpret_cast<moe::GemvItem*>(b + o[bGemvItems]);
+  w.y_zero = reinterpret_cast<int*>(b + o[bYZero]);
   w.act_bits = desc->debug ? reinterpret_cast<uint32_t*>(b + o[bActBits]) : nullptr;
   w.xperm = b + o[bXperm];
   w.ht = b + o[bHt];
@@ -464,9 +475,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   if (e != cudaSuccess) return cuda_fail(c, e, "route launch");
   stage_ran[0] = true;
   mark(1);
-  e = moe::launch_permute(dm, c->ws, x, c->bf16, st);
-  if (e != cudaSuccess) return cuda_fail(c, e, "permute launch");
-  stage_ran[1] = true;
+  if (!moe::route_is_small(dm)) {
+    e = moe::launch_permute(dm, c->ws, x, c->bf16, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "permute launch");
+    stage_ran[1] = true;
+  }
   mark(2);
 
   const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
@@ -506,9 +519,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   if (e != cudaSuccess) return cuda_fail(c, e, "gate_up launch");
   stage_ran[2] = true;
   mark(3);
-  e = moe::launch_union_scan(dm, c->ws, st);
-  if (e != cudaSuccess) return cuda_fail(c, e, "union_scan launch");
-  stage_ran[3] = true;
+  if (c->desc.path == MOE_PATH_SPARSE_TC) {  // only the gathered path needs row lists
+    e = moe::launch_union_scan(dm, c->ws, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "union_scan launch");
+    stage_ran[3] = true;
+  }
   mark(4);
 
   const int mode = c->desc.path;
@@ -601,7 +616,7 @@ moe_status moe_sparse_get_stats(moe_sparse_ctx* c, moe_stats* s, void* stream) {
   s->n_groups = meta[moe::kMetaGroups];
   s->n_groups_gemv = (int64_t)cnt[moe::kCntGemv];
   s->n_groups_tc_gather = (int64_t)cnt[moe::kCntTcGather];
-  s->n_groups_tc_allrows = (int64_t)cnt[moe::kCntTcAll];
+  s->n_groups_tc_allrows = (int64_t)(cnt[moe::kCntTc] - cnt[moe::kCntTcGather]);
   s->n_experts_touched = meta[moe::kMetaExpertsTouched];
   return MOE_OK;
 }
