@@ -190,6 +190,37 @@ MOE_API const char* moe_sparse_stage_name(int32_t i);
 /* Last error message of ctx (or of the last failed init if ctx is NULL). */
 MOE_API const char* moe_sparse_last_error(const moe_sparse_ctx* ctx);
 
+/* Routing only, for callers that must not allocate device memory (code that
+ * runs while a CUDA graph is being captured, plug-ins living inside another
+ * framework's fixed memory plan, serving loops that reserve all memory up
+ * front). The paper has no counterpart: it is an allocation-free variant of
+ * the forward's router kernel, not a step of the method.
+ * It computes what moe_sparse_forward's router computes for x [T][d_model]
+ * and W_router [n_experts][d_model] (device pointers, dtype, 16-byte aligned;
+ * router_bias [n_experts] float32 or NULL) into caller DEVICE buffers:
+ *   topk_idx [T][top_k] int32, topk_w [T][top_k] float32 (as in get_debug);
+ *   expert_offsets [n_experts+1]: pairs of expert e hold positions
+ *     expert_offsets[e] .. expert_offsets[e+1]-1 (no padding);
+ *   slot_of [T*top_k]: position of pair p = t*top_k + i; perm [T*top_k]: token
+ *     at each position; within an expert, positions follow pair order.
+ * Its scratch is a 1 MiB array in device memory that every GPU which loads the
+ * library holds until exit, so it allocates nothing and launches one kernel
+ * (plus a 256-byte cudaMemsetAsync that clears its completion counter).
+ * Limits: T <= 4096, n_experts <= 256, top_k <= 16, d_model a multiple of 256
+ * (bf16) or 128 (fp32); larger sizes return MOE_ERR_UNSUPPORTED with a message.
+ * The first call on a device looks the scratch address up (set-up): make that
+ * first call before any stream capture. All calls share the one scratch array,
+ * so calls whose kernels overlap on the GPU (different streams, or different
+ * host threads on one device) race and must be serialised by the caller.
+ * Runs on the current device, enqueued on stream. */
+MOE_API moe_status moe_sparse_route_noalloc(const void* x, int32_t T, int32_t d_model,
+                                            const void* W_router, const float* router_bias,
+                                            int32_t n_experts, int32_t top_k,
+                                            int32_t renormalize, int32_t dtype,
+                                            int32_t* topk_idx, float* topk_w,
+                                            int32_t* expert_offsets, int32_t* slot_of,
+                                            int32_t* perm, void* stream);
+
 /* Frees the workspace and the context. NULL is accepted. */
 MOE_API moe_status moe_sparse_destroy(moe_sparse_ctx* ctx);
 

@@ -76,6 +76,8 @@ SIGNATURES = {
     "moe_sparse_launch_count": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int64)]),
     "moe_sparse_stage_name": (ctypes.c_char_p, [_i32]),
     "moe_sparse_last_error": (ctypes.c_char_p, [_vp]),
+    "moe_sparse_route_noalloc": (ctypes.c_int, [_vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
+                                                _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_sparse_destroy": (ctypes.c_int, [_vp]),
 }
 

@@ -19,6 +19,7 @@ using moe::Dims;
 using moe::Workspace;
 
 namespace moe {
+void set_last_error(const std::string& msg);
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("MOE_PDL");
@@ -216,6 +217,8 @@ struct DeviceGuard {
 };
 
 }  // namespace
+
+void moe::set_last_error(const std::string& msg) { g_init_error = msg; }
 
 struct moe_sparse_ctx {
   moe_sparse_desc desc;
