@@ -41,6 +41,11 @@ from moe_inputs import WORKLOADS, make_tokens, make_weights  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and effective HBM GB/s vs own dense path, 0-90% sparsity"
 FALLBACK_HBM_GBS = 6650.0
+# DRAM traffic / algorithmic bytes of gate_up_tc_kernel from one ncu capture of a smaller
+# launch of the same kernel (decode batch T=8, 7 experts touched): traffic grows with the
+# touched experts, so a launch's traffic is this ratio times its algorithmic bytes
+# (profiles/gate_up_tc.mixtral_decode_T8.md). None once the kernel has changed since.
+GATE_UP_TRAFFIC_RATIO = 1.0049
 
 
 def parse():
@@ -405,6 +410,9 @@ def run_ours(args, world, rank, local):
 
     peak, peak_kind = peaks()
     g_ach = gate_bytes_tot / (gate_ms_tot * 1e-3) / 1e9 if gate_ms_tot else 0.0
+    n_gate_launches = args.steps * len(tokens)
+    g_traffic = None if GATE_UP_TRAFFIC_RATIO is None else \
+        round(GATE_UP_TRAFFIC_RATIO * gate_bytes_tot / n_gate_launches)
     d_ach = down_bytes_tot / (down_ms_tot * 1e-3) / 1e9 if down_ms_tot else 0.0
     steps_launches = launches
 
@@ -461,7 +469,9 @@ def run_ours(args, world, rank, local):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"kernel": "gate_up_tc", "bound": "hbm", "achieved": round(g_ach, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(g_ach / peak, 4),
-                         "traffic": None, "peak_kind": peak_kind},
+                         "traffic": g_traffic,
+                         "algorithmic_bytes": round(gate_bytes_tot / n_gate_launches),
+                         "peak_kind": peak_kind},
             "roofline_down": {"kernel": "down (GEMV / TC, rows actually read)", "bound": "hbm",
                               "achieved": round(d_ach, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(d_ach / peak, 4), "peak_kind": peak_kind},
