@@ -242,7 +242,10 @@ __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(uint32_t M, uint32_t
 
 // ---------------------------------------------------------------- misc
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU(g) = g / (1 + e^-g) with the fast exponential and division intrinsics
+// (a few ulp of fp32; the threshold band is 1e-3 of tau). For g below about
+// -88, e^-g overflows to +inf and the quotient is -0.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);

@@ -37,7 +37,7 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 constexpr uint32_t kSpinLimit = 4u << 20;  // ~1 s of polling with backoff
 constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT
 
-constexpr int kGroupMax = 256;      // tokens per expert token group (gate/up tile N)
+constexpr int kGroupMax = 128;      // tokens per expert token group (gate/up tile N)
 constexpr int kGatherMaxTokens = 64;  // groups on the gathered TC path hold <= 64 tokens
 constexpr int kSlotAlign = 8;       // expert slot ranges start at multiples of 8 slots
 constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
@@ -107,7 +107,7 @@ struct Workspace {
   float* topk_w;                // [Tmax*kmax]
   int* slot_of;                 // [Tmax*kmax]
   int* rank_cta;                // [Tmax*kmax] rank of a pair among its CTA's pairs of that expert
-  int* hist;                    // [router CTAs][E] per-CTA expert counts, then CTA base offsets
+  int* hist;                    // [E][router CTAs] per-CTA expert counts, then CTA base offsets
   int* expert_off;              // [E+1] first slot of each expert (multiple of kSlotAlign)
   int* expert_cnt;              // [E] routed pairs per expert
   int* perm;                    // [slots_routed] token of each routed slot, -1 for padding

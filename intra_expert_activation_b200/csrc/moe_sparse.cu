@@ -126,8 +126,8 @@ moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   if ((long long)d->max_tokens * d->top_k_max > (1ll << 22)) { err = "max_tokens * top_k_max > 2^22"; return MOE_ERR_UNSUPPORTED; }
   {
     const long long P = (long long)d->max_tokens * d->top_k_max;
-    const long long groups = P / 256 + std::min<long long>(d->n_experts, P) +
-                             (long long)d->n_shared * ((d->max_tokens + 255) / 256) + 1;
+    const long long groups = P / 128 + std::min<long long>(d->n_experts, P) +
+                             (long long)d->n_shared * ((d->max_tokens + 127) / 128) + 1;
     if (groups > 2048) { err = "too many expert token groups (max_tokens * top_k_max too large)"; return MOE_ERR_UNSUPPORTED; }
   }
   return MOE_OK;

@@ -14,11 +14,11 @@
 //            lower expert index; softmax weights, renormalised or not;
 //   ranks    each pair's rank among the CTA's pairs of the same expert in
 //            pair order (warp match + per-warp counts) and the CTA's
-//            histogram hist[cta][e];
+//            histogram hist[e][cta];
 //   finish   the last CTA to finish (atomic ticket after a fence) turns the
-//            histograms into per-CTA base offsets with a segmented scan over
-//            CTAs, pads each expert's slot range to kSlotAlign, and writes the
-//            expert token groups.
+//            histograms into per-CTA base offsets with one scan per expert
+//            over the CTAs, pads each expert's slot range to kSlotAlign, and
+//            lays out the token groups, their paths and the GEMV work.
 // permute_kernel, one warp per pair: slot = expert_off[e] + base[cta][e] +
 //   rank, so slots are ordered by (token, choice) within each expert; it
 //   records perm / slot_of and copies the x row to X_perm[slot]; extra warps
@@ -44,6 +44,16 @@ struct XVec;
 template <>
 struct XVec<__nv_bfloat16> {
   static constexpr int N = 8;
+  __device__ static void load_shared(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(b[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
   __device__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
     const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -58,6 +68,10 @@ struct XVec<__nv_bfloat16> {
 template <>
 struct XVec<float> {
   static constexpr int N = 4;
+  __device__ static void load_shared(const float* p, float (&f)[4]) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
   __device__ static void load(const float* p, float (&f)[4]) {
     const float4 v = __ldg(reinterpret_cast<const float4*>(p));
     f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
@@ -83,34 +97,40 @@ __device__ void route_finish(const Dims& dm, const Workspace& ws, int n_cta, int
                              int* s_b) {
   __shared__ int cnt[kMaxExperts];
   __shared__ int poff[kMaxExperts + 1];
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = dm.E;
-  int e_pow2 = 1;
-  while (e_pow2 < E) e_pow2 <<= 1;
-  const int parts = kThreads / e_pow2 < 32 ? kThreads / e_pow2 : 32;  // lanes per expert
-  const int e = tid / parts, part = tid % parts;
-  const bool live = e < E && tid < e_pow2 * parts;
-  const int c0 = static_cast<int>((long long)part * n_cta / parts);
-  const int c1 = static_cast<int>((long long)(part + 1) * n_cta / parts);
-  int s = 0;
-  if (live)
-    for (int c = c0; c < c1; ++c) s += __ldcg(ws.hist + (size_t)c * E + e);
-  // segmented inclusive scan over the `parts` lanes of one expert
-  int incl = s;
-  for (int o = 1; o < parts; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o, parts);
-    if ((lane % parts) >= o) incl += v;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, (lane / parts) * parts + parts - 1);
-  if (live) {
-    int run = incl - s;
-    for (int c = c0; c < c1; ++c) {
-      int* h = ws.hist + (size_t)c * E + e;
-      const int v = __ldcg(h);
-      *h = run;
-      run += v;
+  // per expert: exclusive scan of its CTA counts (contiguous, expert-major);
+  // each lane takes 8 consecutive CTAs of a 256-CTA chunk, so a chunk is one
+  // load round trip
+  for (int e = warp; e < E; e += blockDim.x / 32) {
+    int* h = ws.hist + static_cast<size_t>(e) * n_cta;
+    int carry = 0;
+    for (int c0 = 0; c0 < n_cta; c0 += 256) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane * 8 + i;
+        v[i] = c < n_cta ? __ldcg(h + c) : 0;
+      }
+      int sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += v[i];
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      int run = carry + incl - sum;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = c0 + lane * 8 + i;
+        if (c < n_cta) h[c] = run;
+        run += v[i];
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (part == 0) cnt[e] = total;
+    if (lane == 0) cnt[e] = carry;
   }
   if (tid < kCntWords) ws.counters[tid] = 0ull;
   __syncthreads();
@@ -166,7 +186,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
       if (me > 0) {
         const int n_g = (me + kGroupMax - 1) / kGroupMax;
         int gsz = (me + n_g - 1) / n_g;
-        gsz = (gsz + 63) / 64 * 64;
+        gsz = (gsz + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
         for (int g = 0; g * gsz < me; ++g) {
           const int m = min(gsz, me - g * gsz);
           zero |= group_path_of(dm, m) == kPathGemv;
@@ -180,7 +200,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     for (int sh = 0; sh < dm.S; ++sh) {
       const int n_g = (T + kGroupMax - 1) / kGroupMax;
       int gsz = (T + n_g - 1) / n_g;
-      gsz = (gsz + 63) / 64 * 64;
+      gsz = (gsz + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
       for (int g = 0; g * gsz < T; ++g) {
         const int m = min(gsz, T - g * gsz);
         zero_s |= group_path_of(dm, m) == kPathGemv;
@@ -337,7 +357,7 @@ __device__ __forceinline__ void topk_token(const Dims& dm, const Workspace& ws, 
 template <typename TX>
 __global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, const TX* x,
                                                          const TX* Wr, const float* bias,
-                                                         int tpc) {
+                                                         int tpc, int stage_x) {
   __shared__ float lg[kRouteTokens][kMaxExperts + 1];
   __shared__ int sel[kRouteTokens * 16];
   __shared__ int wcnt[kWarps][kMaxExperts];
@@ -349,11 +369,62 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, 
   const int tok0 = blockIdx.x * tpc;
   const int tb = min(tpc, T - tok0);
 
-  // ---- logits: warp tasks (token, expert), lanes over d
-  for (int task = warp; task < tb * E; task += kWarps) {
-    const int t = task / E, e = task % E;
-    const float a = row_dot<TX>(x + (size_t)(tok0 + t) * d, Wr + (size_t)e * d, d, lane);
-    if (lane == 0) lg[t][e] = a + (bias ? bias[e] : 0.f);
+  if (stage_x) {
+    // ---- logits with the CTA's x rows in shared memory: a warp owns an
+    // expert and all of the CTA's tokens, so one W_router load feeds tb tokens
+    extern __shared__ __align__(16) uint8_t xs_raw[];
+    float* xs = reinterpret_cast<float*>(xs_raw);  // [tb][d] as fp32
+    constexpr int VEC = XVec<TX>::N;
+    const int nvec = tb * d / VEC;
+    for (int i = tid; i < nvec; i += kThreads) {
+      float v[VEC];
+      XVec<TX>::load(x + (size_t)tok0 * d + (size_t)i * VEC, v);
+#pragma unroll
+      for (int q = 0; q < VEC; q += 4)
+        *reinterpret_cast<float4*>(xs + (size_t)i * VEC + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+    }
+    __syncthreads();
+    for (int e = warp; e < E; e += kWarps) {
+      float acc[kRouteTokens];
+#pragma unroll
+      for (int t = 0; t < kRouteTokens; ++t) acc[t] = 0.f;
+      const TX* wr = Wr + (size_t)e * d;
+      for (int c = lane * VEC; c < d; c += 32 * VEC) {
+        float w[VEC];
+        XVec<TX>::load(wr + c, w);
+#pragma unroll
+        for (int t = 0; t < kRouteTokens; ++t) {
+          if (t < tb) {
+            const float* xr = xs + (size_t)t * d + c;
+#pragma unroll
+            for (int v = 0; v < VEC; v += 4) {
+              const float4 xv = *reinterpret_cast<const float4*>(xr + v);
+              acc[t] = fmaf(xv.x, w[v], acc[t]);
+              acc[t] = fmaf(xv.y, w[v + 1], acc[t]);
+              acc[t] = fmaf(xv.z, w[v + 2], acc[t]);
+              acc[t] = fmaf(xv.w, w[v + 3], acc[t]);
+            }
+          }
+        }
+      }
+      const float b = bias ? bias[e] : 0.f;
+#pragma unroll
+      for (int t = 0; t < kRouteTokens; ++t) {
+        if (t < tb) {
+          float a = acc[t];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          if (lane == 0) lg[t][e] = a + b;
+        }
+      }
+    }
+  } else {
+    // ---- logits: warp tasks (token, expert), lanes over d
+    for (int task = warp; task < tb * E; task += kWarps) {
+      const int t = task / E, e = task % E;
+      const float a = row_dot<TX>(x + (size_t)(tok0 + t) * d, Wr + (size_t)e * d, d, lane);
+      if (lane == 0) lg[t][e] = a + (bias ? bias[e] : 0.f);
+    }
   }
   __syncthreads();
 
@@ -379,7 +450,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, 
     int c = 0;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) c += wcnt[w][x2];
-    ws.hist[(size_t)blockIdx.x * E + x2] = c;
+    ws.hist[(size_t)x2 * gridDim.x + blockIdx.x] = c;
   }
 
   // ---- the last CTA to finish builds the slot layout for the whole batch
@@ -404,6 +475,7 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
   const int item = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int k = dm.k, E = dm.E, P = dm.T * dm.k;
+  const int n_cta = (dm.T + tpc - 1) / tpc;
   constexpr int kVec = 16 / sizeof(TX);
   const int nv = dm.d / kVec;
   const int nz = dm.d / 4;  // float4 per Y row
@@ -411,7 +483,7 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
     const int t = item / k;
     const int e = __ldcg(ws.topk_idx + item);
     const int cta = t / tpc;
-    const int slot = __ldcg(ws.expert_off + e) + __ldcg(ws.hist + (size_t)cta * E + e) +
+    const int slot = __ldcg(ws.expert_off + e) + __ldcg(ws.hist + (size_t)e * n_cta + cta) +
                      __ldcg(ws.rank_cta + item);
     if (lane == 0) {
       ws.perm[slot] = t;
@@ -529,7 +601,12 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 // Tokens per router CTA: few at decode so that the (token, expert) dot
 // products spread over many SMs, more at prefill to keep the per-CTA
 // histograms short.
-int route_tokens_per_cta(int T) { return T <= 256 ? 2 : kRouteTokens; }
+int route_tokens_per_cta(const Dims& dm) {
+  if (dm.T <= 256) return 2;
+  int tpc = kRouteTokens;  // rows staged as fp32 in shared memory: at most 192 KB
+  while (tpc > 2 && (size_t)tpc * dm.d * 4 > 192 * 1024) tpc >>= 1;
+  return tpc;
+}
 
 bool route_is_small(const Dims& dm) { return dm.T <= kSmallTokens; }
 
@@ -543,21 +620,36 @@ cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, con
     return launch_k(route_small_kernel<float>, 1, kSmallThreads, 0, st, dm, ws,
                     static_cast<const float*>(x), static_cast<const float*>(Wr), bias);
   }
-  const int tpc = route_tokens_per_cta(dm.T);
+  const int tpc = route_tokens_per_cta(dm);
   const int grid = (dm.T + tpc - 1) / tpc;
+  // with 16 tokens per CTA, stage their rows in shared memory when they fit
+  const size_t xbytes = (size_t)tpc * dm.d * 4;
+  const int stage_x = tpc > 2 && xbytes <= 192 * 1024;
+  const size_t smem = stage_x ? xbytes : 0;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               192 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   if (bf16)
-    return launch_k(route_kernel<__nv_bfloat16>, grid, kThreads, 0, st, dm, ws,
+    return launch_k(route_kernel<__nv_bfloat16>, grid, kThreads, smem, st, dm, ws,
                     static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
-                    bias, tpc);
-  return launch_k(route_kernel<float>, grid, kThreads, 0, st, dm, ws,
-                  static_cast<const float*>(x), static_cast<const float*>(Wr), bias, tpc);
+                    bias, tpc, stage_x);
+  return launch_k(route_kernel<float>, grid, kThreads, smem, st, dm, ws,
+                  static_cast<const float*>(x), static_cast<const float*>(Wr), bias, tpc,
+                  stage_x);
 }
 
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st) {
   const int items = dm.T * dm.k + dm.E + dm.S * dm.T;
   const int grid = (items + 7) / 8;
-  const int tpc = route_tokens_per_cta(dm.T);
+  const int tpc = route_tokens_per_cta(dm);
   if (bf16)
     return launch_k(permute_kernel<__nv_bfloat16>, grid, 256, 0, st, dm, ws,
                     static_cast<const __nv_bfloat16*>(x), tpc);
