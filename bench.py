@@ -27,7 +27,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
+import threading
 import sys
 import time
 
@@ -81,57 +81,54 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons of this process's GPU, read through
+    NVML every 5 ms by a background thread while the timed region runs
+    (read-only queries; nothing is set)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device: int):
-        self.proc = None
+        self.samples = []
         self.error = None
-        props = torch.cuda.get_device_properties(device)
-        cands = []
-        uuid = str(getattr(props, "uuid", "") or "")
-        if uuid:
-            cands.append(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
-        if hasattr(props, "pci_bus_id"):
-            cands.append(f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:"
-                         f"{getattr(props, 'pci_device_id', 0):02X}.0")
-        for sel in cands:
-            try:
-                probe = subprocess.run(["nvidia-smi", "--query-gpu=index", "--format=csv,noheader",
-                                        "-i", sel], capture_output=True, text=True, timeout=20)
-            except Exception as exc:  # no nvidia-smi
-                self.error = str(exc)
-                return
-            if probe.returncode == 0 and probe.stdout.strip():
-                self.proc = subprocess.Popen(
-                    ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                     "-lms", "200", "-i", sel], stdout=subprocess.PIPE,
-                    stderr=subprocess.DEVNULL, text=True)
-                return
-            self.error = (probe.stderr or probe.stdout).strip()[:200]
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # no NVML on this machine
+            self.error = f"NVML: {exc}"[:200]
+            return
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception as exc:
+                    self.error = f"NVML: {exc}"[:200]
+                    return
+                self.samples.append((sm, rs))
+                self._stop.wait(0.005)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"error": self.error or "nvidia-smi unavailable"}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return {"error": self.error or "no clock samples"}
+        reasons = sorted(n for n, bit in self.REASONS.items()
+                         if any(rs & bit for _, rs in self.samples))
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "NVML, 5 ms"}
 
 
 def dist_init(args):

@@ -68,7 +68,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // about a second: sets *abort, records MOE_ERR_DEVICE_TIMEOUT and returns
 // false, so that no kernel can hang the GPU on a lost arrival.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, int tight = 0) {
+  // optionally first a tight run of probes (each may suspend the thread
+  // briefly in hardware), for waits that are short and on the critical path;
+  // then probes with growing sleeps up to the limit
+  for (int i = 0; i < tight; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -83,9 +88,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // One lane of the warp waits; the outcome is broadcast, so the warp never
 // diverges around a later __syncwarp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, int tight = 0) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, tight) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

@@ -95,7 +95,10 @@ __global__ void __launch_bounds__(kThreads)
     }
     if (nact) atomicAdd(ws.counters + (shared ? kCntSharedActive : kCntRoutedActive), nact);
     __syncthreads();
-    if (threadIdx.x == 0) ws.union_bits[static_cast<size_t>(g) * dm.fw + blk] = uni;
+    if (threadIdx.x == 0) {
+      ws.union_bits[static_cast<size_t>(g) * dm.fw + blk] = uni;
+      if (uni) atomicAdd(ws.union_cnt + g, __popc(uni));
+    }
     __syncthreads();
   }
 }

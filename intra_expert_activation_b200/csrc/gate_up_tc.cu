@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 0) {
         p.ws.union_bits[static_cast<size_t>(g) * fw + word] = uni;
+        if (uni) atomicAdd(p.ws.union_cnt + g, __popc(uni));
         atomicAdd(p.ws.counters + (ui.shared ? kCntSharedActive : kCntRoutedActive), nact);
       }
       tc_fence_before();

@@ -35,6 +35,7 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
 }
 
 constexpr uint32_t kSpinLimit = 4u << 20;  // ~1 s of polling with backoff
+constexpr int kErrDeviceInvalid = 1;       // == MOE_ERR_INVALID: an internal consistency check failed
 constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT
 
 constexpr int kGroupMax = 128;      // tokens per expert token group (gate/up tile N)
@@ -44,15 +45,12 @@ constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
 constexpr int kDownSlice = 128;     // d_model columns per down TC tile (M)
 constexpr int kKBlock = 64;         // K elements per pipeline stage (128 B of bf16)
 constexpr int kRouteTokens = 16;    // tokens per router CTA
-constexpr int kGemvWordsMax = 24;   // bitmap words (32 neurons each) per GEMV work item
-constexpr int kGemvRowsMax = 32 * kGemvWordsMax;
 constexpr int kListMax = 2048;      // expert token groups per forward at most
 constexpr int kGemvTokens = 4;      // tokens per GEMV unit (bf16); fp32 uses 8
 
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
-            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
-            kMetaGemvItems = 8, kMetaGemvNext = 9, kMetaWords = 16 };
+            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6, kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
@@ -63,17 +61,6 @@ enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3
 
 // Requested path (mirrors moe_path in the public header).
 enum Mode { kModeAuto = 0, kModeDense = 1, kModeGemv = 2, kModeTc = 3, kModeTcAll = 4 };
-
-// One GEMV work item: a split of a group's union rows for one pass of tokens.
-struct GemvItem {
-  int32_t g;       // group
-  int32_t expert;  // expert of the group (E + s for shared expert s)
-  int32_t slot;    // first slot of the pass (group slot0 + pass * MT)
-  int32_t mt;      // tokens in the pass
-  int32_t w0, w1;  // union bitmap words [w0, w1): neurons 32*w0 .. 32*w1-1
-  int32_t whole;   // 1: the item is the whole unit (plain store), 0: atomic add
-  int32_t pad;
-};
 
 // One expert token group: up to kGroupMax consecutive slots of one expert.
 struct Group {
@@ -96,7 +83,6 @@ struct Dims {
   float gather_density;
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device
-  int gemv_items_max; // capacity of gemv_items
 };
 
 struct Workspace {
@@ -115,10 +101,10 @@ struct Workspace {
   int* group_path;              // [groups_max]
   uint32_t* union_bits;         // [groups_max][fw]
   int* union_rows;              // [groups_max][F_max]
-  int* union_cnt;               // [groups_max]
+  int* union_cnt;               // [groups_max] rows in each group's union (cleared by the router,
+                                //   accumulated by the gate/up epilogue)
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
   int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
-  GemvItem* gemv_items;         // [gemv_items_max] work items of the GEMV path
   int* y_zero;                  // [E+1] 1: expert's Y rows (last: shared experts') start at zero
 
   uint32_t* act_bits;           // [slots_total][fw] or null (debug off)

@@ -91,7 +91,7 @@ struct Layout {
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bGemvItems, bYZero,
+           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero,
            bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
@@ -158,15 +158,6 @@ Layout make_layout(const moe_sparse_desc* d) {
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
   c.gather_density = d->gather_max_density;
   c.no_tc = bf16 ? 0 : 1;
-  {
-    // GEMV items: each unit has max(target, ceil(words / kGemvWordsMax)) splits at
-    // most, and units * target <= max(units, 2 * SMs) (SMs <= 1024 assumed here)
-    const int mt = bf16 ? moe::kGemvTokens : 8;
-    const long long units = ((long long)P + (long long)c.S * c.T) / mt + c.groups_max;
-    const long long per_unit = (c.F_max / 32 + moe::kGemvWordsMax - 1) / moe::kGemvWordsMax;
-    c.gemv_items_max =
-        (int)std::min<long long>(units * per_unit + std::max(units, 2048ll), INT32_MAX);
-  }
 
   const size_t es = bf16 ? 2 : 4;
   size_t sz[bCount];
@@ -188,7 +179,6 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bUnionCnt] = sizeof(int) * c.groups_max;
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
-  sz[bGemvItems] = sizeof(moe::GemvItem) * (size_t)c.gemv_items_max;
   sz[bYZero] = sizeof(int) * (c.E + 1);
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;
   sz[bXperm] = es * (size_t)c.slots_routed * c.d;
@@ -368,7 +358,6 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.union_cnt = reinterpret_cast<int*>(b + o[bUnionCnt]);
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
-  w.gemv_items = reinterpret_cast<moe::GemvItem*>(b + o[bGemvItems]);
   w.y_zero = reinterpret_cast<int*>(b + o[bYZero]);
   w.act_bits = desc->debug ? reinterpret_cast<uint32_t*>(b + o[bActBits]) : nullptr;
   w.xperm = b + o[bXperm];

@@ -5,11 +5,12 @@
 // Activation Sparsity for Efficient Mixture-of-Expert Model Execution",
 // Technical Summary > Methodology > System Implementation in vLLM].
 //
-// route_kernel, one CTA per `tpc` tokens (2 at decode, kRouteTokens at
+// route_kernel, one CTA per `tpc` tokens (2 at decode, up to kRouteTokens at
 // prefill):
-//   logits   warp tasks (token, expert): the lanes stride d with batches of
-//            16-byte loads of the x row and the W_router row and reduce with
-//            a butterfly (fp32, a fixed summation order);
+//   logits   the CTA's x rows are copied to shared memory; a warp takes 4
+//            experts (and, with few experts, a slice of d) and keeps tpc x 4
+//            fp32 sums in registers while its lanes stride d in 16-byte
+//            vectors; butterfly reductions, a fixed summation order;
 //   top-k    one warp per token: the k largest logits, equal logits to the
 //            lower expert index; softmax weights, renormalised or not;
 //   ranks    each pair's rank among the CTA's pairs of the same expert in
@@ -39,13 +40,13 @@ __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
+// 16-byte vectors of x / W_router rows, widened to fp32 (exactly).
 template <typename TX>
 struct XVec;
 template <>
 struct XVec<__nv_bfloat16> {
   static constexpr int N = 8;
-  __device__ static void load_shared(const __nv_bfloat16* p, float (&f)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+  __device__ static void unpack(const uint4& u, float (&f)[8]) {
     const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -54,27 +55,25 @@ struct XVec<__nv_bfloat16> {
       f[2 * i + 1] = t.y;
     }
   }
+  __device__ static void load_shared(const __nv_bfloat16* p, float (&f)[8]) {
+    unpack(*reinterpret_cast<const uint4*>(p), f);
+  }
   __device__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 t = __bfloat1622float2(b[i]);
-      f[2 * i] = t.x;
-      f[2 * i + 1] = t.y;
-    }
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), f);
   }
 };
 template <>
 struct XVec<float> {
   static constexpr int N = 4;
+  __device__ static void unpack(const uint4& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
   __device__ static void load_shared(const float* p, float (&f)[4]) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    unpack(*reinterpret_cast<const uint4*>(p), f);
   }
   __device__ static void load(const float* p, float (&f)[4]) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), f);
   }
 };
 
@@ -87,187 +86,243 @@ __device__ __forceinline__ int group_path_of(const Dims& dm, int m) {
   return m <= dm.gemv_max ? kPathGemv : kPathTcAll;  // auto and dense
 }
 
-// Last CTA: histograms -> base offsets, expert slot ranges, token groups, the
-// path of every group, the GEMV work items. s_a / s_b are free shared
-// scratch of at least 2 * kListMax + 1 and kListMax ints.
-__device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt, int* poff,
-                             int* s_a, int* s_b);
+// Last CTA: histograms -> base offsets, expert slot ranges, token groups and
+// the path of every group.
+__device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt, int* poff);
 
-__device__ void route_finish(const Dims& dm, const Workspace& ws, int n_cta, int* s_a,
-                             int* s_b) {
+__device__ void route_finish(const Dims& dm, const Workspace& ws, int n_cta) {
   __shared__ int cnt[kMaxExperts];
   __shared__ int poff[kMaxExperts + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = dm.E;
-  // per expert: exclusive scan of its CTA counts (contiguous, expert-major);
-  // each lane takes 8 consecutive CTAs of a 256-CTA chunk, so a chunk is one
-  // load round trip
-  for (int e = warp; e < E; e += blockDim.x / 32) {
-    int* h = ws.hist + static_cast<size_t>(e) * n_cta;
-    int carry = 0;
+  // per expert: exclusive scan of its CTA counts (contiguous, expert-major).
+  // A warp takes kEb experts at a time and each lane 8 consecutive CTAs of a
+  // 256-CTA chunk, so the loads of kEb experts' chunks are in flight together
+  constexpr int kEb = 4;
+  const int nw = blockDim.x / 32;
+  for (int e0 = warp * kEb; e0 < E; e0 += nw * kEb) {
+    int carry[kEb] = {};
     for (int c0 = 0; c0 < n_cta; c0 += 256) {
-      int v[8];
+      int v[kEb][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = c0 + lane * 8 + i;
-        v[i] = c < n_cta ? __ldcg(h + c) : 0;
+      for (int j = 0; j < kEb; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = c0 + lane * 8 + i;
+          v[j][i] = (e0 + j < E && c < n_cta) ? __ldcg(ws.hist + (size_t)(e0 + j) * n_cta + c) : 0;
+        }
+#pragma unroll
+      for (int j = 0; j < kEb; ++j) {
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum += v[j][i];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        int run = carry[j] + incl - sum;
+        if (e0 + j < E) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int c = c0 + lane * 8 + i;
+            if (c < n_cta) ws.hist[(size_t)(e0 + j) * n_cta + c] = run;
+            run += v[j][i];
+          }
+        }
+        carry[j] += __shfl_sync(0xffffffffu, incl, 31);
       }
-      int sum = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sum += v[i];
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      int run = carry + incl - sum;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = c0 + lane * 8 + i;
-        if (c < n_cta) h[c] = run;
-        run += v[i];
-      }
-      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) cnt[e] = carry;
+    if (lane < kEb && e0 + lane < E) {
+      int cv = carry[0];
+#pragma unroll
+      for (int j = 1; j < kEb; ++j)
+        if (lane == j) cv = carry[j];
+      cnt[e0 + lane] = cv;
+    }
   }
   if (tid < kCntWords) ws.counters[tid] = 0ull;
   __syncthreads();
-  build_layout(dm, ws, cnt, poff, s_a, s_b);
+  build_layout(dm, ws, cnt, poff);
+}
+
+// Exclusive prefix sums over the CTA of N ints per thread, in thread order
+// (v becomes the prefix, total the CTA-wide sums). sm: (32 + 1) * N ints.
+// Every thread of the CTA calls it.
+template <int N>
+__device__ __forceinline__ void block_exclusive_scan(int (&v)[N], int (&total)[N], int* sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int inc[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) inc[j] = v[j];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int u = __shfl_up_sync(0xffffffffu, inc[j], o);
+      if (lane >= o) inc[j] += u;
+    }
+  if (lane == 31)
+#pragma unroll
+    for (int j = 0; j < N; ++j) sm[warp * N + j] = inc[j];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int w = lane < nw ? sm[lane * N + j] : 0;
+      int wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += u;
+      }
+      if (lane < nw) sm[lane * N + j] = wi - w;
+      if (lane == 31) sm[32 * N + j] = wi;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    v[j] = sm[warp * N + j] + inc[j] - v[j];
+    total[j] = sm[32 * N + j];
+  }
+  __syncthreads();
+}
+
+// How one entry's tokens are cut into groups. An entry is a routed expert
+// (q < E, its me = cnt[q] pairs) or a shared expert (q >= E, all T tokens):
+// ng groups of gsz tokens (a multiple of kSlotAlign; the last one has
+// m_last), each at most kGroupMax.
+struct EntryCut {
+  int me, ng, gsz, m_last, F_e, path_full, path_last;
+};
+
+__device__ __forceinline__ EntryCut entry_cut(const Dims& dm, const int* cnt, int q) {
+  EntryCut c;
+  c.me = q < dm.E ? cnt[q] : dm.T;
+  c.F_e = q < dm.E ? dm.F : dm.Fs;
+  if (c.me <= 0) {
+    c.ng = c.gsz = c.m_last = 0;
+    c.path_full = c.path_last = kPathGemv;
+    return c;
+  }
+  const int n_g = (c.me + kGroupMax - 1) / kGroupMax;
+  c.gsz = ((c.me + n_g - 1) / n_g + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+  c.ng = (c.me + c.gsz - 1) / c.gsz;
+  c.m_last = c.me - (c.ng - 1) * c.gsz;
+  c.path_full = group_path_of(dm, c.gsz);
+  c.path_last = group_path_of(dm, c.m_last);
+  return c;
 }
 
 // From the per-expert pair counts cnt[E] (shared memory): expert slot ranges
-// poff[E+1] (shared), token groups, the path of every group, the GEMV work
-// items, counters and meta. s_a / s_b: shared scratch of 2 * kListMax + 1 and
-// kListMax ints. Called by every thread of the CTA; counters must be zero.
-__device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt, int* poff,
-                             int* s_a, int* s_b) {
-  __shared__ int n_gemv_s, n_items_s;
+// poff[E+1] (shared), token groups, the path of every group, the GEMV and TC
+// group lists, counters and meta; every group's union count is cleared for
+// the gate/up epilogue to accumulate. Called by every thread of the CTA;
+// counters must be zero. Each thread takes a run of consecutive entries
+// (routed experts, then the shared experts); prefix sums over the CTA place
+// their slots, groups and list entries, so group order is (expert, group) as
+// in a serial walk over the experts.
+__device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt, int* poff) {
+  constexpr int kPer = 2;  // entries per thread: E + S <= 264 <= 2 x 256 threads
+  __shared__ int scan_sm[33 * 8];
+  __shared__ int zero_shared;
   const int tid = threadIdx.x;
-  const int E = dm.E, T = dm.T, k = dm.k;
-  const int mt = dm.no_tc ? 8 : kGemvTokens;
-  int* gemv_g = s_a;                  // [kListMax] GEMV groups in group order
-  int* item_off = s_a + kListMax;     // [kListMax + 1]
-  int* splits = s_b;                  // [kListMax]
-  if (tid == 0) {
-    int touched = 0;
-    poff[0] = 0;
-    for (int x = 0; x < E; ++x) {
-      const int me = cnt[x];
-      touched += me > 0;
-      poff[x + 1] = poff[x] + (me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+  const int E = dm.E, T = dm.T, k = dm.k, S = dm.S;
+  const int n_ent = E + S;
+  const int per = (n_ent + blockDim.x - 1) / blockDim.x;  // <= kPer
+  const int q0 = min(tid * per, n_ent), q1 = min(q0 + per, n_ent);
+  if (tid == 0) zero_shared = 0;
+
+  // ---- pass 1: slots, groups, GEMV / TC list positions
+  enum { kSlots, kGroups, kGemv, kTc, kRoutedGroups, kTcShared, kTouched, kN };
+  int v[kN] = {}, tot[kN];
+  EntryCut cut[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int q = q0 + i;
+    if (q >= q1) continue;
+    const EntryCut c = entry_cut(dm, cnt, q);
+    cut[i] = c;
+    if (c.ng == 0) continue;
+    const int n_gemv = (c.ng - 1) * (c.path_full == kPathGemv) + (c.path_last == kPathGemv);
+    if (q < E) {
+      v[kSlots] += (c.me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+      v[kRoutedGroups] += c.ng;
+      v[kTouched] += 1;
+    } else {
+      v[kTcShared] += c.ng - n_gemv;
     }
-    int ng = 0, n_gemv = 0, n_tc = 0, units = 0;
-    unsigned long long tc_rows = 0;
-    auto add_group = [&](int expert, int slot0, int m, int xrow0, int F_e) {
-      if (ng >= dm.groups_max) return;
-      Group gr;
-      gr.expert = expert;
-      gr.slot0 = slot0;
-      gr.m = m;
-      gr.xrow0 = xrow0;
-      ws.groups[ng] = gr;
-      const int path = group_path_of(dm, m);
-      ws.group_path[ng] = path;
-      if (path == kPathGemv) {
-        gemv_g[n_gemv] = ng;
-        ws.gemv_list[n_gemv++] = ng;
-        units += (m + mt - 1) / mt;
-      } else {
-        ws.tc_list[n_tc++] = ng;
-        tc_rows += F_e;
-      }
-      ++ng;
-    };
-    for (int x = 0; x < E; ++x) {
-      const int me = cnt[x];
-      int zero = 0;
-      if (me > 0) {
-        const int n_g = (me + kGroupMax - 1) / kGroupMax;
-        int gsz = (me + n_g - 1) / n_g;
-        gsz = (gsz + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
-        for (int g = 0; g * gsz < me; ++g) {
-          const int m = min(gsz, me - g * gsz);
-          zero |= group_path_of(dm, m) == kPathGemv;
-          add_group(x, poff[x] + g * gsz, m, poff[x] + g * gsz, dm.F);
+    v[kGroups] += c.ng;
+    v[kGemv] += n_gemv;
+    v[kTc] += c.ng - n_gemv;
+  }
+  block_exclusive_scan<kN>(v, tot, scan_sm);
+
+  // ---- pass 2: write the groups and lists
+  {
+    int slot = v[kSlots], g = v[kGroups], gv = v[kGemv], tc = v[kTc];
+    for (int i = 0; i < kPer; ++i) {
+      const int q = q0 + i;
+      if (q >= q1) continue;
+      const EntryCut& c = cut[i];
+      const bool routed = q < E;
+      const int base = routed ? slot : dm.slots_routed + (q - E) * dm.T_pad;
+      if (routed) poff[q] = slot;
+      int any_gemv = 0;
+      for (int j = 0; j < c.ng; ++j, ++g) {
+        const int m = j == c.ng - 1 ? c.m_last : c.gsz;
+        const int path = j == c.ng - 1 ? c.path_last : c.path_full;
+        if (g < dm.groups_max) {
+          Group gr;
+          gr.expert = q;
+          gr.slot0 = base + j * c.gsz;
+          gr.m = m;
+          gr.xrow0 = routed ? base + j * c.gsz : j * c.gsz;
+          ws.groups[g] = gr;
+          ws.group_path[g] = path;
+          ws.union_cnt[g] = 0;
+          if (path == kPathGemv) {
+            any_gemv = 1;
+            ws.gemv_list[gv++] = g;
+          } else {
+            ws.tc_list[tc++] = g;
+          }
         }
       }
-      ws.y_zero[x] = zero;
-    }
-    ws.meta[kMetaRoutedGroups] = ng;
-    int zero_s = 0;
-    for (int sh = 0; sh < dm.S; ++sh) {
-      const int n_g = (T + kGroupMax - 1) / kGroupMax;
-      int gsz = (T + n_g - 1) / n_g;
-      gsz = (gsz + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
-      for (int g = 0; g * gsz < T; ++g) {
-        const int m = min(gsz, T - g * gsz);
-        zero_s |= group_path_of(dm, m) == kPathGemv;
-        add_group(E + sh, dm.slots_routed + sh * dm.T_pad + g * gsz, m, g * gsz, dm.Fs);
+      if (routed) {
+        ws.y_zero[q] = any_gemv;
+        slot += (c.me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
+      } else if (any_gemv) {
+        zero_shared = 1;  // benign race: every writer stores 1
       }
     }
-    ws.y_zero[E] = zero_s;
-    // GEMV items: every unit (group, pass of mt tokens) of group i is cut into
-    // splits[i] neuron ranges of whole bitmap words, about three items per SM
-    // (the GEMV kernel balances them with a queue)
-    const int target = max(1, 3 * dm.n_sms / max(units, 1));
-    int items = 0;
-    for (int i = 0; i < n_gemv; ++i) {
-      const Group gr = ws.groups[gemv_g[i]];
-      const int words = (gr.expert >= E ? dm.Fs : dm.F) / 32;
-      const int s_min = (words + kGemvWordsMax - 1) / kGemvWordsMax;
-      splits[i] = min(max(target, s_min), words);
-      item_off[i] = items;
-      items += (gr.m + mt - 1) / mt * splits[i];
-    }
-    item_off[n_gemv] = items;
-    items = min(items, dm.gemv_items_max);
-    n_gemv_s = n_gemv;
-    n_items_s = items;
-    ws.meta[kMetaGroups] = ng;
-    ws.meta[kMetaSlotsUsed] = poff[E];
-    ws.meta[kMetaExpertsTouched] = touched;
-    ws.meta[kMetaGemvCount] = n_gemv;
-    ws.meta[kMetaTcCount] = n_tc;
-    ws.meta[kMetaGemvItems] = items;
-    ws.meta[kMetaGemvNext] = 0;
-    ws.counters[kCntGemv] = n_gemv;
-    ws.counters[kCntTc] = n_tc;
-    if (dm.mode != kModeTc) ws.counters[kCntDownRows] = tc_rows;  // GEMV items add theirs
+  }
+  __syncthreads();
+  if (tid == 0) {
+    poff[E] = tot[kSlots];
+    ws.y_zero[E] = zero_shared;
+    ws.meta[kMetaRoutedGroups] = tot[kRoutedGroups];
+    ws.meta[kMetaGroups] = tot[kGroups];
+    ws.meta[kMetaSlotsUsed] = tot[kSlots];
+    ws.meta[kMetaExpertsTouched] = tot[kTouched];
+    ws.meta[kMetaGemvCount] = tot[kGemv];
+    ws.meta[kMetaTcCount] = tot[kTc];
+    ws.counters[kCntGemv] = tot[kGemv];
+    ws.counters[kCntTc] = tot[kTc];
+    if (dm.mode != kModeTc)  // the GEMV kernel adds its rows
+      ws.counters[kCntDownRows] =
+          (unsigned long long)(tot[kTc] - tot[kTcShared]) * dm.F +
+          (unsigned long long)tot[kTcShared] * dm.Fs;
     ws.counters[kCntRoutedH] = (unsigned long long)T * k * (unsigned long long)dm.F;
     ws.counters[kCntSharedH] =
-        (unsigned long long)dm.S * (unsigned long long)T * (unsigned long long)dm.Fs;
+        (unsigned long long)S * (unsigned long long)T * (unsigned long long)dm.Fs;
     ws.meta[kMetaDone] = 0;  // ticket counter for the next forward
   }
   __syncthreads();
   for (int x = tid; x <= E; x += blockDim.x) ws.expert_off[x] = poff[x];
   for (int x = tid; x < E; x += blockDim.x) ws.expert_cnt[x] = cnt[x];
-  // item descriptors: everything a GEMV CTA needs in one load
-  const int n_gemv = n_gemv_s, n_items = n_items_s;
-  for (int it = tid; it < n_items; it += blockDim.x) {
-    int lo_i = 0, hi_i = n_gemv;
-    while (hi_i - lo_i > 1) {
-      const int mid = (lo_i + hi_i) >> 1;
-      if (item_off[mid] <= it) lo_i = mid; else hi_i = mid;
-    }
-    const int g = gemv_g[lo_i];
-    const Group gr = ws.groups[g];
-    const int words = (gr.expert >= E ? dm.Fs : dm.F) / 32;
-    const int sp = splits[lo_i];
-    const int local = it - item_off[lo_i];
-    const int split = local % sp, pass = local / sp;
-    GemvItem d;
-    d.g = g;
-    d.expert = gr.expert;
-    d.slot = gr.slot0 + pass * mt;
-    d.mt = min(mt, gr.m - pass * mt);
-    d.w0 = split * words / sp;
-    d.w1 = (split + 1) * words / sp;
-    d.whole = sp == 1;
-    d.pad = 0;
-    ws.gemv_items[it] = d;
-  }
 }
 
 // Dot product of one token row with one router row, lanes over d in chunks
@@ -278,22 +333,25 @@ __device__ __forceinline__ float row_dot(const TX* a, const TX* b, int d, int la
   constexpr int kBatch = 8;
   float acc = 0.f;
   for (int c0 = lane * VEC; c0 < d; c0 += 32 * VEC * kBatch) {
-    float av[kBatch][VEC], bv[kBatch][VEC];
+    uint4 ra[kBatch], rb[kBatch];  // raw vectors: the loads of a batch are in flight together
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
       const int c = c0 + i * 32 * VEC;
       if (c < d) {
-        XVec<TX>::load(a + c, av[i]);
-        XVec<TX>::load(b + c, bv[i]);
+        ra[i] = __ldg(reinterpret_cast<const uint4*>(a + c));
+        rb[i] = __ldg(reinterpret_cast<const uint4*>(b + c));
       } else {
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) av[i][v] = bv[i][v] = 0.f;
+        ra[i] = rb[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i)
+    for (int i = 0; i < kBatch; ++i) {
+      float av[VEC], bv[VEC];
+      XVec<TX>::unpack(ra[i], av);
+      XVec<TX>::unpack(rb[i], bv);
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc = fmaf(av[i][v], bv[i][v], acc);
+      for (int v = 0; v < VEC; ++v) acc = fmaf(av[v], bv[v], acc);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -354,10 +412,84 @@ __device__ __forceinline__ void topk_token(const Dims& dm, const Workspace& ws, 
   }
 }
 
-template <typename TX>
-__global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, const TX* x,
-                                                         const TX* Wr, const float* bias,
-                                                         int tpc, int stage_x) {
+// Logits of the CTA's tb <= TPC tokens, whose rows sit in shared memory in
+// their stored type, against every expert. A warp item is (4 experts, one
+// slice of d); its lanes stride the slice in 16-byte vectors and keep TPC x 4
+// fp32 sums in registers, so one shared-memory vector of x feeds 4 experts
+// and one W_router vector feeds all TPC tokens. With fewer than 4 x kWarps
+// experts, d is split into up to kWarps / (E/4) slices so that every warp has
+// work; the slices' sums are added in slice order (fixed summation order).
+template <typename TX, int TPC>
+__device__ __forceinline__ void staged_logits(const Dims& dm, const TX* xs, const TX* Wr,
+                                              const float* bias, int tb,
+                                              float (*lg)[kMaxExperts + 1], float* part) {
+  constexpr int VEC = XVec<TX>::N;
+  constexpr int EPW = 4;
+  const int E = dm.E, d = dm.d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_eg = (E + EPW - 1) / EPW;
+  const int ks = n_eg >= kWarps ? 1 : kWarps / n_eg;
+  const int dsl = ((d / ks + VEC - 1) / VEC) * VEC;
+  for (int item = warp; item < n_eg * ks; item += kWarps) {
+    const int e0 = (item / ks) * EPW, s = item % ks;
+    const int c0 = s * dsl, c1 = min(d, c0 + dsl);
+    const TX* wrow[EPW];
+#pragma unroll
+    for (int j = 0; j < EPW; ++j) wrow[j] = Wr + (size_t)min(e0 + j, E - 1) * d;
+    float acc[TPC][EPW];
+#pragma unroll
+    for (int t = 0; t < TPC; ++t)
+#pragma unroll
+      for (int j = 0; j < EPW; ++j) acc[t][j] = 0.f;
+#pragma unroll(TPC <= 4 ? 2 : 1)
+    for (int c = c0 + lane * VEC; c < c1; c += 32 * VEC) {
+      float w[EPW][VEC];
+#pragma unroll
+      for (int j = 0; j < EPW; ++j) XVec<TX>::load(wrow[j] + c, w[j]);
+#pragma unroll
+      for (int t = 0; t < TPC; ++t) {
+        if (t < tb) {
+          float xv[VEC];
+          XVec<TX>::load_shared(xs + (size_t)t * d + c, xv);
+#pragma unroll
+          for (int j = 0; j < EPW; ++j)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[t][j] = fmaf(xv[v], w[j][v], acc[t][j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < TPC; ++t) {
+#pragma unroll
+      for (int j = 0; j < EPW; ++j) {
+        float a = acc[t][j];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        const int e = e0 + j;
+        if (lane == 0 && t < tb && e < E) {
+          if (ks == 1)
+            lg[t][e] = a + (bias ? bias[e] : 0.f);
+          else
+            part[(s * TPC + t) * E + e] = a;
+        }
+      }
+    }
+  }
+  if (ks > 1) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < tb * E; i += kThreads) {
+      const int t = i / E, e = i % E;
+      float a = 0.f;
+      for (int s = 0; s < ks; ++s) a += part[(s * TPC + t) * E + e];
+      lg[t][e] = a + (bias ? bias[e] : 0.f);
+    }
+  }
+}
+
+template <typename TX, int TPC>
+__global__ void __launch_bounds__(kThreads, 2) route_kernel(Dims dm, Workspace ws, const TX* x,
+                                                            const TX* Wr, const float* bias,
+                                                            int tpc, int stage_x) {
   __shared__ float lg[kRouteTokens][kMaxExperts + 1];
   __shared__ int sel[kRouteTokens * 16];
   __shared__ int wcnt[kWarps][kMaxExperts];
@@ -370,54 +502,17 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, 
   const int tb = min(tpc, T - tok0);
 
   if (stage_x) {
-    // ---- logits with the CTA's x rows in shared memory: a warp owns an
-    // expert and all of the CTA's tokens, so one W_router load feeds tb tokens
+    // ---- logits with the CTA's x rows copied to shared memory as stored
     extern __shared__ __align__(16) uint8_t xs_raw[];
-    float* xs = reinterpret_cast<float*>(xs_raw);  // [tb][d] as fp32
-    constexpr int VEC = XVec<TX>::N;
-    const int nvec = tb * d / VEC;
-    for (int i = tid; i < nvec; i += kThreads) {
-      float v[VEC];
-      XVec<TX>::load(x + (size_t)tok0 * d + (size_t)i * VEC, v);
-#pragma unroll
-      for (int q = 0; q < VEC; q += 4)
-        *reinterpret_cast<float4*>(xs + (size_t)i * VEC + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-    }
+    TX* xs = reinterpret_cast<TX*>(xs_raw);  // [tb][d]
+    const int nvec = tb * d * (int)sizeof(TX) / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok0 * d);
+    for (int i = tid; i < nvec; i += kThreads) reinterpret_cast<uint4*>(xs)[i] = __ldg(src + i);
     __syncthreads();
-    for (int e = warp; e < E; e += kWarps) {
-      float acc[kRouteTokens];
-#pragma unroll
-      for (int t = 0; t < kRouteTokens; ++t) acc[t] = 0.f;
-      const TX* wr = Wr + (size_t)e * d;
-      for (int c = lane * VEC; c < d; c += 32 * VEC) {
-        float w[VEC];
-        XVec<TX>::load(wr + c, w);
-#pragma unroll
-        for (int t = 0; t < kRouteTokens; ++t) {
-          if (t < tb) {
-            const float* xr = xs + (size_t)t * d + c;
-#pragma unroll
-            for (int v = 0; v < VEC; v += 4) {
-              const float4 xv = *reinterpret_cast<const float4*>(xr + v);
-              acc[t] = fmaf(xv.x, w[v], acc[t]);
-              acc[t] = fmaf(xv.y, w[v + 1], acc[t]);
-              acc[t] = fmaf(xv.z, w[v + 2], acc[t]);
-              acc[t] = fmaf(xv.w, w[v + 3], acc[t]);
-            }
-          }
-        }
-      }
-      const float b = bias ? bias[e] : 0.f;
-#pragma unroll
-      for (int t = 0; t < kRouteTokens; ++t) {
-        if (t < tb) {
-          float a = acc[t];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          if (lane == 0) lg[t][e] = a + b;
-        }
-      }
-    }
+    // the split-d partial sums (slices x E <= 32, so at most 32 x TPC
+    // floats) reuse wcnt, which is cleared only after the top-k
+    static_assert(sizeof(wcnt) >= sizeof(float) * 32 * kRouteTokens, "partials");
+    staged_logits<TX, TPC>(dm, xs, Wr, bias, tb, lg, reinterpret_cast<float*>(&wcnt[0][0]));
   } else {
     // ---- logits: warp tasks (token, expert), lanes over d
     for (int task = warp; task < tb * E; task += kWarps) {
@@ -463,9 +558,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(Dims dm, Workspace ws, 
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  static_assert(sizeof(lg) >= sizeof(int) * (2 * kListMax + 1), "finish scratch");
-  static_assert(sizeof(wcnt) >= sizeof(int) * kListMax, "finish scratch");
-  route_finish(dm, ws, gridDim.x, reinterpret_cast<int*>(&lg[0][0]), &wcnt[0][0]);
+  route_finish(dm, ws, gridDim.x);
 }
 
 template <typename TX>
@@ -516,7 +609,7 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
 }
 
 // Small batches (T <= kSmallTokens): the whole routing step in one CTA of
-// 32 warps with no cross-CTA ticket: logits, top-k, in-order stable ranks,
+// 16 warps with no cross-CTA ticket: logits, top-k, in-order stable ranks,
 // layout, and the permute copies of the x rows (and zeroing of the Y rows
 // that GEMV splits add into).
 constexpr int kSmallThreads = 512;
@@ -530,8 +623,6 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __shared__ int slot_s[kSmallTokens * 16];
   __shared__ int cnt[kMaxExperts];
   __shared__ int poff[kMaxExperts + 1];
-  __shared__ int scratch_a[2 * kListMax + 1];
-  __shared__ int scratch_b[kListMax];
 
   grid_dep_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -558,7 +649,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  build_layout(dm, ws, cnt, poff, scratch_a, scratch_b);
+  build_layout(dm, ws, cnt, poff);
   __syncthreads();
   for (int p = tid; p < P; p += kSmallThreads) {
     const int slot = poff[sel[p]] + slot_s[p];
@@ -598,17 +689,52 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 
 }  // namespace
 
-// Tokens per router CTA: few at decode so that the (token, expert) dot
-// products spread over many SMs, more at prefill to keep the per-CTA
-// histograms short.
-int route_tokens_per_cta(const Dims& dm) {
+// Tokens per router CTA: few at decode so that the batch spreads over many
+// SMs, more at prefill to keep the per-CTA histograms short; the staged rows
+// stay within kStageBytes so that two router CTAs fit on an SM.
+constexpr size_t kStageBytes = 80 * 1024;
+
+int route_tokens_per_cta(const Dims& dm, int elem_bytes) {
   if (dm.T <= 256) return 2;
-  int tpc = kRouteTokens;  // rows staged as fp32 in shared memory: at most 192 KB
-  while (tpc > 2 && (size_t)tpc * dm.d * 4 > 192 * 1024) tpc >>= 1;
+  int tpc = kRouteTokens;
+  while (tpc > 2 && (size_t)tpc * dm.d * elem_bytes > kStageBytes) tpc >>= 1;
   return tpc;
 }
 
 bool route_is_small(const Dims& dm) { return dm.T <= kSmallTokens; }
+
+namespace {
+
+template <typename TX, int TPC>
+cudaError_t launch_route_t(const Dims& dm, const Workspace& ws, const TX* x, const TX* Wr,
+                           const float* bias, int tpc, cudaStream_t st) {
+  const int grid = (dm.T + tpc - 1) / tpc;
+  const size_t xbytes = (size_t)tpc * dm.d * sizeof(TX);
+  const int stage_x = xbytes <= kStageBytes;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        route_kernel<TX, TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return launch_k(route_kernel<TX, TPC>, grid, kThreads, stage_x ? xbytes : 0, st, dm, ws, x,
+                  Wr, bias, tpc, stage_x);
+}
+
+template <typename TX>
+cudaError_t launch_route_x(const Dims& dm, const Workspace& ws, const TX* x, const TX* Wr,
+                           const float* bias, cudaStream_t st) {
+  const int tpc = route_tokens_per_cta(dm, sizeof(TX));
+  switch (tpc) {
+    case 2: return launch_route_t<TX, 2>(dm, ws, x, Wr, bias, tpc, st);
+    case 4: return launch_route_t<TX, 4>(dm, ws, x, Wr, bias, tpc, st);
+    case 8: return launch_route_t<TX, 8>(dm, ws, x, Wr, bias, tpc, st);
+    default: return launch_route_t<TX, kRouteTokens>(dm, ws, x, Wr, bias, tpc, st);
+  }
+}
+
+}  // namespace
 
 cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, const void* Wr,
                          const float* bias, bool bf16, cudaStream_t st) {
@@ -620,36 +746,18 @@ cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, con
     return launch_k(route_small_kernel<float>, 1, kSmallThreads, 0, st, dm, ws,
                     static_cast<const float*>(x), static_cast<const float*>(Wr), bias);
   }
-  const int tpc = route_tokens_per_cta(dm);
-  const int grid = (dm.T + tpc - 1) / tpc;
-  // with 16 tokens per CTA, stage their rows in shared memory when they fit
-  const size_t xbytes = (size_t)tpc * dm.d * 4;
-  const int stage_x = tpc > 2 && xbytes <= 192 * 1024;
-  const size_t smem = stage_x ? xbytes : 0;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<__nv_bfloat16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(route_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               192 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   if (bf16)
-    return launch_k(route_kernel<__nv_bfloat16>, grid, kThreads, smem, st, dm, ws,
-                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(Wr),
-                    bias, tpc, stage_x);
-  return launch_k(route_kernel<float>, grid, kThreads, smem, st, dm, ws,
-                  static_cast<const float*>(x), static_cast<const float*>(Wr), bias, tpc,
-                  stage_x);
+    return launch_route_x(dm, ws, static_cast<const __nv_bfloat16*>(x),
+                          static_cast<const __nv_bfloat16*>(Wr), bias, st);
+  return launch_route_x(dm, ws, static_cast<const float*>(x), static_cast<const float*>(Wr), bias,
+                        st);
 }
 
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st) {
   const int items = dm.T * dm.k + dm.E + dm.S * dm.T;
   const int grid = (items + 7) / 8;
-  const int tpc = route_tokens_per_cta(dm);
+  const int tpc = route_tokens_per_cta(dm, bf16 ? 2 : 4);
   if (bf16)
     return launch_k(permute_kernel<__nv_bfloat16>, grid, 256, 0, st, dm, ws,
                     static_cast<const __nv_bfloat16*>(x), tpc);
