@@ -231,6 +231,9 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
                            long long* sm_warp) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = blockDim.x / 32;
+  // the first list entries are read while the list length is still in
+  // flight (they are inside the list's capacity either way)
+  const int g_spec = tid < dm.groups_max ? __ldcg(ws.gemv_list + tid) : 0;
   const int n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
   // rows of each GEMV group (all passes); one sweep when the groups fit the
   // CTA, else a first sweep for the total
@@ -240,17 +243,18 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
     st->i = -1;
     st->rows = 0;
   }
-  __syncthreads();
   for (int sweep = one ? 1 : 0; sweep < 2; ++sweep) {
     long long carry = 0;
     for (int base = 0; base < n_gv; base += blockDim.x) {
       const int i = base + tid;
       long long v = 0;
-      int g = 0, cnt = 0;
+      int g = 0, cnt = 0, words = 0;
       if (i < n_gv) {
-        g = __ldcg(ws.gemv_list + i);
+        g = base == 0 ? g_spec : __ldcg(ws.gemv_list + i);
         cnt = __ldcg(ws.union_cnt + g);
-        v = (long long)((ws.groups[g].m + MT - 1) / MT) * cnt;
+        const Group gr = ws.groups[g];
+        v = (long long)((gr.m + MT - 1) / MT) * cnt;
+        words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
       }
       long long incl = v;
 #pragma unroll
@@ -278,6 +282,7 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
           st->p = (int)(off / cnt);
           st->g = g;
           st->row = (int)(off % cnt);
+          st->w = words;  // the group's word count, until warp 0 positions the cursor
         }
       }
       carry += chunk;
@@ -292,8 +297,7 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
   if (st->rows <= 0 || st->i < 0) return;  // uniform
   // warp 0: the bitmap word holding row st->row of group st->g
   if (warp == 0) {
-    const int g = st->g;
-    const int words = (ws.groups[g].expert >= dm.E ? dm.Fs : dm.F) / 32;
+    const int g = st->g, words = st->w;
     int skip = st->row;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const uint32_t bits =
@@ -306,13 +310,14 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
         if (lane >= o) incl += u;
       }
       const int excl = incl - c;
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      __syncwarp();  // every lane has read st->w before the owner lane rewrites it
       if (excl <= skip && skip < incl) {  // this lane's word holds the first row
         uint32_t m = bits;
         for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
         st->w = w0 + lane;
         st->m = m;
       }
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
       if (skip < total) break;
       skip -= total;
     }
@@ -451,10 +456,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NS = geo.n_stages;
   const int n_blocks = (row_bytes + kBlockBytes - 1) / kBlockBytes;
 
-  // finite zeros in every stage (rows past a run keep earlier finite rows),
-  // barriers, then the async proxy may write
-  for (int i = threadIdx.x; i < NS * geo.stage / 16; i += kThreads)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
   if (threadIdx.x == 0) {
     for (int b = 0; b < NS; ++b) {
       mbar_init(full + b, 1 + kBatch);  // expect_tx arrival + one per h-copying lane
@@ -464,76 +465,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     atomicAdd(ws.counters + kCntDownRows, static_cast<unsigned long long>(start.rows));
   }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   const uint32_t smem_s = smem_u32(smem);
 
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
+    // run-major: each run of rows (one unit) is streamed once per column
+    // block, so the bitmaps are walked once
     const size_t ld = static_cast<size_t>(dm.slots_total);
     const char* ht = static_cast<const char*>(ws.ht);
+    Walk k;
+    k.i = start.i;
+    k.p = start.p;
+    k.w = start.w;
+    k.m = start.m;
+    k.left = start.rows;
+    k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
+    k.serial = 0;
+    walk_load_group(dm, ws, k, MT);
     int s = 0;  // stages filled
     bool ok = true;
-    for (int cb = 0; cb < n_blocks && ok; ++cb) {
-      const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
-      Walk k;
-      k.i = start.i;
-      k.p = start.p;
-      k.w = start.w;
-      k.m = start.m;
-      k.left = start.rows;
-      k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
-      k.serial = 0;
-      walk_load_group(dm, ws, k, MT);
-      int n_list = 0, pos = 0;
-      for (;;) {
-        while (pos >= n_list) {
-          n_list = walk_next(dm, ws, k, list, MT, lane);
-          pos = 0;
-          if (n_list == 0) break;
-        }
-        const int b = s % NS;
-        if (s >= NS && !warp_wait(empty + b, ((s / NS) + 1) & 1, &abort_flag, ws.status, kTight)) {
-          ok = false;
-          break;
-        }
-        uint8_t* stg = smem + b * geo.stage;
-        const uint32_t stg_s = smem_s + b * geo.stage;
-        const int cnt = min(kBatch, n_list - pos);  // 0: the block's end marker
-        const int p = k.p;
-        const int slot = k.slot0 + p * MT;
-        const int mt = min(MT, k.m_tok - p * MT);
-        // stage metadata, then one arrival with the rows' transaction bytes;
-        // lanes 0..7 copy the h values of their rows with cp.async and arrive
-        // when those land (the consumers mask tokens past the pass and rows
-        // past the run)
-        if (lane == 0) {
-          *reinterpret_cast<int4*>(stg + kBatch * geo.stride + kBatch * kHBytes) =
-              make_int4(cnt > 0 ? k.serial : -1, cnt, slot, mt);
-          mbar_arrive_expect_tx(full + b, static_cast<uint32_t>(cnt * cbytes));
-        }
-        __syncwarp();
-        if (lane < kBatch) {
-          if (lane < cnt) {
-            const int j = list[pos + lane];
-            const char* hsrc = ht + ((size_t)j * ld + slot) * ES;
-            const uint32_t hdst = stg_s + kBatch * geo.stride + lane * kHBytes;
-            if constexpr (ES == 2) {
-              cp_async8(hdst, hsrc);
-            } else {
-              cp_async16(hdst, hsrc);
-              cp_async16(hdst + 16, hsrc + 16);
-            }
-            const TW* wrow = (k.expert >= dm.E ? Wds + (size_t)(k.expert - dm.E) * dm.Fs * d
-                                               : Wd + (size_t)k.expert * dm.F * d) +
-                             (size_t)j * d + cb * (kBlockBytes / ES);
-            bulk_load(stg_s + lane * geo.stride, wrow, cbytes, smem_u32(full + b));
+    for (bool last = false; ok && !last;) {
+      const int n_list = walk_next(dm, ws, k, list, MT, lane);
+      last = n_list == 0;
+      const int slot = k.slot0 + k.p * MT;
+      const int mt = min(MT, k.m_tok - k.p * MT);
+      const TW* wexp = k.expert >= dm.E ? Wds + (size_t)(k.expert - dm.E) * dm.Fs * d
+                                        : Wd + (size_t)k.expert * dm.F * d;
+      for (int cb = 0; cb < (last ? 1 : n_blocks) && ok; ++cb) {
+        const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
+        for (int pos = 0; pos < n_list || (last && pos == 0); pos += kBatch) {
+          const int b = s % NS;
+          if (s >= NS && !warp_wait(empty + b, ((s / NS) + 1) & 1, &abort_flag, ws.status, kTight)) {
+            ok = false;
+            break;
           }
-          cp_async_arrive(smem_u32(full + b));
+          uint8_t* stg = smem + b * geo.stage;
+          const uint32_t stg_s = smem_s + b * geo.stage;
+          const int cnt = last ? 0 : min(kBatch, n_list - pos);  // 0: the end marker
+          if (!last && cnt < kBatch) {
+            // rows past the run enter the mma with zero h: give them finite
+            // values (never-written shared memory may hold any bits)
+            for (int r = cnt; r < kBatch; ++r)
+              for (int o = lane * 16; o < geo.block; o += 32 * 16)
+                *reinterpret_cast<uint4*>(stg + r * geo.stride + o) = make_uint4(0u, 0u, 0u, 0u);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          }
+          // stage metadata, then one arrival with the rows' transaction
+          // bytes; lanes 0..7 copy the h values of their rows with cp.async
+          // and arrive when those land (the consumers mask tokens past the
+          // pass and rows past the run)
+          if (lane == 0) {
+            *reinterpret_cast<int4*>(stg + kBatch * geo.stride + kBatch * kHBytes) =
+                make_int4(last ? -1 : k.serial * n_blocks + cb, cnt, slot, mt | (cb << 8));
+            mbar_arrive_expect_tx(full + b, static_cast<uint32_t>(cnt * cbytes));
+          }
+          __syncwarp();
+          if (lane < kBatch) {
+            if (lane < cnt) {
+              const int j = list[pos + lane];
+              const uint32_t hdst = stg_s + kBatch * geo.stride + lane * kHBytes;
+              const char* hsrc = ht + ((size_t)j * ld + slot) * ES;
+              if constexpr (ES == 2) {
+                cp_async8(hdst, hsrc);
+              } else {
+                cp_async16(hdst, hsrc);
+                cp_async16(hdst + 16, hsrc + 16);
+              }
+              bulk_load(stg_s + lane * geo.stride,
+                        wexp + (size_t)j * d + cb * (kBlockBytes / ES), cbytes,
+                        smem_u32(full + b));
+            }
+            cp_async_arrive(smem_u32(full + b));
+          }
+          ++s;
         }
-        ++s;
-        pos += cnt;
-        if (cnt == 0) break;  // end marker sent
       }
     }
     // do not leave with copies in flight: wait (bounded) for the last stages
@@ -545,47 +551,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ consumers
     R rows;
     float* ystage = reinterpret_cast<float*>(smem + NS * geo.stage) + warp * (kYBytes / 4);
-    int s = 0;  // stages consumed
-    for (int cb = 0; cb < n_blocks; ++cb) {
+    rows.zero();
+    int cur_tag = -1, cur_slot = 0, cur_mt = 0, cur_col0 = 0;
+    for (int s = 0;; ++s) {
+      const int b = s % NS;
+      if (!warp_wait(full + b, (s / NS) & 1, &abort_flag, ws.status, kTight)) break;
+      const uint8_t* stg = smem + b * geo.stage;
+      const int4 meta = *reinterpret_cast<const int4*>(stg + kBatch * geo.stride + kBatch * kHBytes);
+      const int cb = meta.w >> 8, mt = meta.w & 255;
       const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
-      const int n_slices = (cbytes + kSliceBytes - 1) / kSliceBytes;
+      // this warp's slice of the block; with narrow blocks several warps
+      // share a slice and take alternate stages
+      const int n_slices = cbytes / kSliceBytes;
       const int n_phase = n_slices >= kConsumers ? 1 : kConsumers / n_slices;
       const int slice = warp % n_slices, phase = warp / n_slices;
-      const bool active = phase < n_phase;
-      const int col0 = (cb * kBlockBytes + slice * kSliceBytes) / ES;
-      rows.zero();
-      int cur_serial = -1, cur_slot = 0, cur_mt = 0;
-      bool ok = true;
-      for (int q = 0;; ++q, ++s) {
-        const int b = s % NS;
-        if (!warp_wait(full + b, (s / NS) & 1, &abort_flag, ws.status, kTight)) {
-          ok = false;
-          break;
+      const bool mine = phase < n_phase && (s % n_phase) == phase;
+      if (meta.x != cur_tag && (mine || meta.x < 0)) {
+        if (cur_tag >= 0) {
+          rows.flush(ws.y + (size_t)cur_slot * d + cur_col0, d, cur_mt, ystage, lane);
+          rows.zero();
         }
-        const uint8_t* stg = smem + b * geo.stage;
-        const int4 meta =
-            *reinterpret_cast<const int4*>(stg + kBatch * geo.stride + kBatch * kHBytes);
-        const bool mine = active && (q % n_phase) == phase;
-        if (meta.x != cur_serial && (mine || meta.x < 0)) {
-          if (cur_serial >= 0) {
-            rows.flush(ws.y + (size_t)cur_slot * d + col0, d, cur_mt, ystage, lane);
-            rows.zero();
-          }
-          cur_serial = meta.x;
-          cur_slot = meta.z;
-          cur_mt = meta.w;
-        }
-        if (mine && meta.y > 0)
-          rows.consume(smem_s + b * geo.stage + slice * kSliceBytes, stg + slice * kSliceBytes,
-                       geo.stride, stg + kBatch * geo.stride, meta.y, meta.w, lane);
-        __syncwarp();  // every lane has read the stage
-        if (lane == 0) mbar_arrive(empty + b);
-        if (meta.x < 0) {
-          ++s;
-          break;
-        }
+        cur_tag = meta.x;
+        cur_slot = meta.z;
+        cur_mt = mt;
+        cur_col0 = (cb * kBlockBytes + slice * kSliceBytes) / ES;
       }
-      if (!ok) break;
+      if (mine && meta.y > 0)
+        rows.consume(smem_s + b * geo.stage + slice * kSliceBytes, stg + slice * kSliceBytes,
+                     geo.stride, stg + kBatch * geo.stride, meta.y, mt, lane);
+      __syncwarp();  // every lane has read the stage
+      if (lane == 0) mbar_arrive(empty + b);
+      if (meta.x < 0) break;
     }
   }
 }
