@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # launch of the same kernel (decode batch T=8, 7 experts touched): traffic grows with the
 # touched experts, so a launch's traffic is this ratio times its algorithmic bytes
 # (profiles/gate_up_tc.mixtral_decode_T8.md). None once the kernel has changed since.
-GATE_UP_TRAFFIC_RATIO = 1.0049
+GATE_UP_TRAFFIC_RATIO = None
 
 
 def parse():
@@ -131,18 +131,20 @@ class Clocks:
                 "source": "NVML, 5 ms"}
 
 
-def dist_init(args):
+def dist_init(args=None, backend=None):
+    """One process per GPU (torchrun env); NCCL on GPUs, gloo without."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
+    if cuda:
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
+        backend = backend or ("nccl" if cuda else "gloo")
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -153,12 +155,31 @@ def barrier(world):
 
 
 def max_over_ranks(world, v: float, local: int) -> float:
+    """The slowest rank's time: every rank's number is all-reduced with MAX."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device=f"cuda:{local}")
+    dev = "cpu" if dist.get_backend() == "gloo" else f"cuda:{local}"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(tokens_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s of weak-scaling replicas: every rank runs the same
+    steps on its own batch, the job takes the slowest rank's time."""
+    return tokens_per_step * steps * world / (ms / 1e3)
+
+
+def workload_config(args, wl, tokens, tau, calib_sparsity, world) -> dict:
+    """The config block both arms print for a workload."""
+    sh = wl.shape
+    return {"workload": args.workload, "batches": tokens, "tokens_per_step": sum(tokens),
+            "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
+            "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
+            "calibrated_sparsity": round(calib_sparsity, 4),
+            "l2": "no flush: touched expert weights (>= 470 MB per forward) exceed L2",
+            "parallelism": f"replicas x{world}"}
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -177,12 +198,16 @@ def oracle_step_time(wl, tokens, tau, tau_s, w_host):
 
 
 def run_reference(args, world, rank):
+    """The oracle arm: the fp64 CPU oracle timed on the host cores, on rank 0
+    only; each step is a bounded sample of the workload's step (its T = 8
+    batch, or its smallest one)."""
     if rank != 0:
         return 0
     wl = WORKLOADS[args.workload]
-    tau, tau_s, _ = load_tau(args.workload, args.sparsity)
+    tokens = [int(t) for t in args.tokens.split(",")] if args.tokens else list(wl.tokens)
+    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity)
     w = make_weights(wl.shape, wl.weight_seed)
-    sample = [8] if 8 in wl.tokens else [min(wl.tokens)]
+    sample = [8] if 8 in tokens else [min(tokens)]
     for _ in range(args.warmup):
         oracle_step_time(wl, sample, tau, tau_s, w)
     t = sum(oracle_step_time(wl, sample, tau, tau_s, w) for _ in range(args.steps))
@@ -194,10 +219,9 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "batches": sample, "target_sparsity": args.sparsity,
-                   "tau": tau},
+        "config": workload_config(args, wl, tokens, tau, calib_sparsity, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"decode batch T={sample} of {args.workload} per step "
+                         "sample": f"each step: the decode batch T={sample} of {args.workload} "
                                    f"(fp64 numpy oracle on {cores} host threads)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -330,7 +354,7 @@ def run_ours(args, world, rank, local):
     per_fwd = kernel_times(sparse)
     lat_sparse = per_batch_us(sparse)
     tok_step = sum(tokens)
-    value = tok_step * args.steps * world / (ms_sparse / 1e3)
+    value = replica_value(tok_step, args.steps, world, ms_sparse)
 
     # per-batch statistics of the sparse path (one extra forward each, untimed)
     stats = []
@@ -352,7 +376,7 @@ def run_ours(args, world, rank, local):
         ms_dense = max_over_ranks(world, ms_dense, local)
         per_dense = kernel_times(dense)
         lat_dense = per_batch_us(dense)
-        dense_line = {"value": tok_step * args.steps * world / (ms_dense / 1e3),
+        dense_line = {"value": replica_value(tok_step, args.steps, world, ms_dense),
                       "ms_per_step": ms_dense / args.steps}
         del g_dense
         dense.close()
@@ -441,7 +465,7 @@ def run_ours(args, world, rank, local):
         barrier(world)
         ms_e2e = max_over_ranks(world, a.elapsed_time(b), local)
         nbytes = sum(x.numel() * x.element_size() for x in xs_host)
-        e2e = {"value": tok_step * args.steps * world / (ms_e2e / 1e3), "unit": "tokens/s",
+        e2e = {"value": replica_value(tok_step, args.steps, world, ms_e2e), "unit": "tokens/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
 
     cpu = None
@@ -458,12 +482,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_sparse / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
             "data": "synthetic",
-            "config": {"workload": args.workload, "batches": tokens, "tokens_per_step": tok_step,
-                       "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
-                       "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
-                       "calibrated_sparsity": round(calib_sparsity, 4),
-                       "l2": "no flush: touched expert weights (>= 470 MB per forward) exceed L2",
-                       "parallelism": f"replicas x{world}"},
+            "config": workload_config(args, wl, tokens, tau, calib_sparsity, world),
             "roofline": {"kernel": "gate_up_tc", "bound": "hbm", "achieved": round(g_ach, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(g_ach / peak, 4),
                          "traffic": g_traffic,
