@@ -25,6 +25,19 @@
 // rounding, warp-ballot the active bits of 32 neurons per token, OR them into
 // the group's active-row union, and write masked h (bf16) transposed into
 // H^T[neuron][slot]. Persistent CTAs walk units with a static stride.
+//
+// Whole units leave the SMs unevenly loaded when the unit count is not a
+// multiple of the grid (decode: a few experts x d_ff/128 tiles over 148 or
+// 296 CTAs, e.g. 896 units = 6 x 148 + 8). So after the rounds of whole
+// units, the leftover units are cut along K into at most four parts each and
+// spread over the CTAs. A cut unit is finished by the CTA that holds its last
+// K-block; the other parts' accumulators go to a per-CTA partial slot with a
+// release flag. The finishing CTA meets that unit first in its leftover
+// range, parks its own part, and sums the parts and runs the epilogue for it
+// after all its other work, when the parts are (nearly) done. Waits are
+// bounded; the parts are added in K order. (Cutting every unit's range
+// evenly instead lowered the DRAM throughput on small-d layers: the whole-
+// unit rounds keep the CTAs in step along K.)
 #include "common.cuh"
 
 namespace moe {
@@ -69,6 +82,136 @@ __device__ __forceinline__ int group_of_unit(int u, int n_rg, int tiles_r, int t
   return n_rg + (u - n_rg * tiles_r) / tiles_s;
 }
 
+// The CTA's sequence of segments: (unit, first K-block, end K-block). Whole
+// units in rounds of G (CTA c takes units c, c + G, ...) while every CTA has
+// one; the n_units mod G leftover units are then cut along K, each into at
+// most kMaxParts parts, over the first P = min(G, leftover x kMaxParts) CTAs:
+// CTA c < P takes iterations [base + Wr c / P, base + Wr (c+1) / P) of the
+// Wr = leftover x K-blocks iterations that start at base.
+constexpr int kMaxParts = 4;
+
+struct Segs {
+  int u, n_full, KB;   // whole units: next one, and how many are whole
+  long long i, end;    // leftover iterations of this CTA
+};
+
+__device__ __forceinline__ Segs segs_begin(int n_units, int KB, int split) {
+  Segs s;
+  s.KB = KB;
+  s.u = blockIdx.x;
+  s.n_full = split ? n_units / gridDim.x * gridDim.x : n_units;
+  const int left = n_units - s.n_full;
+  const int P = min((int)gridDim.x, left * kMaxParts);
+  s.i = s.end = 0;
+  if ((int)blockIdx.x < P) {
+    const long long base = (long long)s.n_full * KB, Wr = (long long)left * KB;
+    s.i = base + Wr * blockIdx.x / P;
+    s.end = base + Wr * (blockIdx.x + 1) / P;
+  }
+  return s;
+}
+
+__device__ __forceinline__ bool segs_next(Segs& s, int& u, int& kb0, int& kb1) {
+  if (s.u < s.n_full) {
+    u = s.u;
+    kb0 = 0;
+    kb1 = s.KB;
+    s.u += gridDim.x;
+    return true;
+  }
+  if (s.i >= s.end) return false;
+  u = (int)(s.i / s.KB);
+  kb0 = (int)(s.i % s.KB);
+  kb1 = (int)min((long long)s.KB, kb0 + (s.end - s.i));
+  s.i += kb1 - kb0;
+  return true;
+}
+
+// CTA holding leftover iteration i.
+__device__ __forceinline__ int cta_of_iter(long long i, int n_units, int KB) {
+  const int n_full = n_units / gridDim.x * gridDim.x;
+  const int left = n_units - n_full;
+  const int P = min((int)gridDim.x, left * kMaxParts);
+  const long long base = (long long)n_full * KB, Wr = (long long)left * KB;
+  return (int)(((i - base + 1) * P - 1) / Wr);
+}
+
+// Partial-slot element of (slot, gate|up, 16-column chunk, neuron row, column):
+// a warp's 32 rows of one chunk are 2 KB contiguous.
+__device__ __forceinline__ float* part_ptr(const GateUpTcParams& p, int slot, int which,
+                                           int chunk, int row) {
+  const size_t chunks = p.n_max / 16;
+  return p.ws.sk_part + ((((size_t)slot * 2 + which) * chunks + chunk) * kNeuronTile + row) * 16;
+}
+
+// SwiGLU, threshold and compaction of 16 columns (tokens c0 .. c0+15) of one
+// neuron row: masked h to H^T, warp ballots into the union word and counts.
+__device__ __forceinline__ void epi_chunk(const GateUpTcParams& p, const UnitInfo& ui, int word,
+                                          int c0, int m, float tau, const float (&gv)[16],
+                                          const float (&uv)[16], __nv_bfloat16* row,
+                                          uint32_t& uni, unsigned long long& nact, int lane) {
+  const int fw = p.dm.fw;
+  float hv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = c0 + i;
+    const float h = silu_f32(gv[i]) * uv[i];
+    const bool act = p.dense || fabsf(h) > tau;
+    hv[i] = act ? h : 0.f;
+    const uint32_t mask = __ballot_sync(0xffffffffu, act && c < m);
+    uni |= mask;
+    if (lane == 0 && c < m) {
+      nact += __popc(mask);
+      if (p.ws.act_bits) p.ws.act_bits[static_cast<size_t>(ui.gr.slot0 + c) * fw + word] = mask;
+    }
+  }
+  if (c0 + 16 <= m) {
+    uint4 pk[2];
+    uint32_t* w32 = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      __nv_bfloat162 v2 = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
+      w32[i] = *reinterpret_cast<uint32_t*>(&v2);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(row + c0);
+    dst[0] = pk[0];
+    dst[1] = pk[1];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (c0 + i < m) row[c0 + i] = __float2bfloat16_rn(hv[i]);
+  }
+}
+
+// Lane 0 of each epilogue warp: the union word, its row count and the
+// active-neuron counter of a finished unit.
+__device__ __forceinline__ void epi_finish(const GateUpTcParams& p, const UnitInfo& ui, int g,
+                                           int word, uint32_t uni, unsigned long long nact,
+                                           int lane) {
+  if (lane == 0) {
+    p.ws.union_bits[static_cast<size_t>(g) * p.dm.fw + word] = uni;
+    if (uni) atomicAdd(p.ws.union_cnt + g, __popc(uni));
+    atomicAdd(p.ws.counters + (ui.shared ? kCntSharedActive : kCntRoutedActive), nact);
+  }
+}
+
+// Bounded wait for another CTA's release flag (acquire).
+__device__ bool wait_flag(const int* f, volatile int* abort, int* status) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v) return true;
+    if (*abort) return false;
+    __nanosleep(i < 64 ? 20 : 200);
+  }
+  *abort = 1;
+  report_error(status, kErrDeviceTimeout);
+  return false;
+}
+
+// The four epilogue warps only (named barrier 1).
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1)
     gate_up_tc_kernel(const __grid_constant__ GateUpTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -84,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;      // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* fix_ok = abort_flag + 1;  // the parked unit's parts are all published
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -117,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_units = n_rg * tiles_r + (n_g - n_rg) * tiles_s;
   const int KB = p.dm.d / kKBlock;
   const uint32_t buf_cols = 2u * n_max;
+  const int split = p.split;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -132,14 +277,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     uint32_t it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    Segs sg = segs_begin(n_units, KB, split);
+    int u, kb0, kb1;
+    while (ok && segs_next(sg, u, kb0, kb1)) {
       const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
       const int N = (ui.gr.m + 15) & ~15;
       const int nb = N / kBRowBox;
       const CUtensorMap* mg = ui.shared ? &p.tm_wgs : &p.tm_wg;
       const CUtensorMap* mu = ui.shared ? &p.tm_wus : &p.tm_wu;
       const CUtensorMap* mx = ui.shared ? &p.tm_x : &p.tm_xperm;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(empty + s, ph ^ 1u, abort_flag, p.ws.status)) { ok = false; break; }
@@ -168,7 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ MMA issuer
     uint32_t it = 0, uidx = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++uidx) {
+    Segs sg = segs_begin(n_units, KB, split);
+    int u, kb0, kb1;
+    for (; ok && segs_next(sg, u, kb0, kb1); ++uidx) {
       const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
       const int N = (ui.gr.m + 15) & ~15;
       const uint32_t idesc = idesc_bf16_f32(kNeuronTile, N, 0, 0);
@@ -178,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t d_gate = tmem_base + b * buf_cols;
       const uint32_t d_up = d_gate + n_max;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(full + s, ph, abort_flag, p.ws.status)) { ok = false; break; }
@@ -190,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = smem_desc_sw128(sa + 2 * kABytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kKBlock / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
+            const uint32_t acc = (kb != kb0) || (kk != 0);
             // +32 bytes along K per 16-element step (descriptor units of 16 B)
             mma_bf16(d_gate, ag + 2 * kk, bd + 2 * kk, idesc, acc);
             mma_bf16(d_up, au + 2 * kk, bd + 2 * kk, idesc, acc);
@@ -214,72 +363,117 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    const int fw = p.dm.fw;
     const size_t ld = static_cast<size_t>(p.dm.slots_total);
     __nv_bfloat16* ht = static_cast<__nv_bfloat16*>(p.ws.ht);
     uint32_t uidx = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++uidx) {
+    bool ok = true;
+    int park_u = -1;  // split unit whose last K-block is ours: finished at the end
+    Segs sg = segs_begin(n_units, KB, split);
+    int u, kb0, kb1;
+    for (; segs_next(sg, u, kb0, kb1); ++uidx) {
+      // every epilogue warp walks every segment (named barriers below), doing
+      // nothing once a wait has failed
       const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
       const int g = group_of_unit(u, n_rg, tiles_r, tiles_s);
       const int m = ui.gr.m;
       const int N = (m + 15) & ~15;
       const uint32_t b = uidx % p.nbuf;
       const uint32_t tph = (uidx / p.nbuf) & 1u;
-      if (!warp_wait(tfull + b, tph, abort_flag, p.ws.status)) break;
-      tc_fence_after();
-      const float tau = ui.shared ? p.tau_shared : p.tau;
-      const int j = ui.nt * kNeuronTile + 32 * q + lane;  // neuron of this thread
-      const int word = (ui.nt * kNeuronTile + 32 * q) >> 5;
-      __nv_bfloat16* row = ht + static_cast<size_t>(j) * ld + ui.gr.slot0;
-      const uint32_t tg = tmem_base + lane_off + b * buf_cols;
-      const uint32_t tu = tg + n_max;
-      uint32_t uni = 0;
-      unsigned long long nact = 0;
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t gr[16], ur[16];
-        tmem_ld16(tg + c0, gr);
-        tmem_ld16(tu + c0, ur);
-        tmem_ld_wait(gr, ur);
-        float hv[16];
+      if (ok && !warp_wait(tfull + b, tph, abort_flag, p.ws.status)) ok = false;
+      const bool whole = kb0 == 0 && kb1 == KB;
+      const bool last_part = !whole && kb1 == KB;
+      if (ok) {
+        tc_fence_after();
+        const float tau = ui.shared ? p.tau_shared : p.tau;
+        const int row_i = 32 * q + lane;
+        const int j = ui.nt * kNeuronTile + row_i;  // neuron of this thread
+        const int word = (ui.nt * kNeuronTile + 32 * q) >> 5;
+        __nv_bfloat16* row = ht + static_cast<size_t>(j) * ld + ui.gr.slot0;
+        const uint32_t tg = tmem_base + lane_off + b * buf_cols;
+        const uint32_t tu = tg + n_max;
+        uint32_t uni = 0;
+        unsigned long long nact = 0;
+        const int slot = last_part ? gridDim.x + blockIdx.x : blockIdx.x;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          uint32_t gr[16], ur[16];
+          tmem_ld16(tg + c0, gr);
+          tmem_ld16(tu + c0, ur);
+          tmem_ld_wait(gr, ur);
+          float gv[16], uv[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          const float h = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
-          const bool act = p.dense || fabsf(h) > tau;
-          hv[i] = act ? h : 0.f;
-          const uint32_t mask = __ballot_sync(0xffffffffu, act && c < m);
-          uni |= mask;
-          if (lane == 0 && c < m) {
-            nact += __popc(mask);
-            if (p.ws.act_bits)
-              p.ws.act_bits[static_cast<size_t>(ui.gr.slot0 + c) * fw + word] = mask;
+          for (int i = 0; i < 16; ++i) {
+            gv[i] = __uint_as_float(gr[i]);
+            uv[i] = __uint_as_float(ur[i]);
+          }
+          if (whole) {
+            epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane);
+          } else {  // a part of a split unit: park its sums
+            float4* pg = reinterpret_cast<float4*>(part_ptr(p, slot, 0, c0 / 16, row_i));
+            float4* pu = reinterpret_cast<float4*>(part_ptr(p, slot, 1, c0 / 16, row_i));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              pg[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+              pu[i] = make_float4(uv[4 * i], uv[4 * i + 1], uv[4 * i + 2], uv[4 * i + 3]);
+            }
           }
         }
-        if (c0 + 16 <= m) {
-          uint4 pk[2];
-          uint32_t* w32 = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(hv[2 * i], hv[2 * i + 1]);
-            w32[i] = *reinterpret_cast<uint32_t*>(&v2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(row + c0);
-          dst[0] = pk[0];
-          dst[1] = pk[1];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < m) row[c0 + i] = __float2bfloat16_rn(hv[i]);
-        }
+        if (whole) epi_finish(p, ui, g, word, uni, nact, lane);
       }
-      if (lane == 0) {
-        p.ws.union_bits[static_cast<size_t>(g) * fw + word] = uni;
-        if (uni) atomicAdd(p.ws.union_cnt + g, __popc(uni));
-        atomicAdd(p.ws.counters + (ui.shared ? kCntSharedActive : kCntRoutedActive), nact);
-      }
+      if (last_part) park_u = u;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + b);
+      if (!whole && !last_part) {
+        // an earlier part: publish it for the CTA that holds the unit's end
+        __threadfence();
+        epi_sync();
+        if (warp == 2 && lane == 0)
+          asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.ws.sk_flags + blockIdx.x),
+                       "r"(1)
+                       : "memory");
+      }
+    }
+    if (park_u >= 0) {
+      // sum the parts of the parked unit in K order, then its epilogue
+      const int c_first = cta_of_iter((long long)park_u * KB, n_units, KB);
+      if (warp == 2 && lane == 0) {
+        int good = *abort_flag == 0 ? 1 : 0;
+        for (int c2 = c_first; c2 < (int)blockIdx.x && good; ++c2)
+          good = wait_flag(p.ws.sk_flags + c2, abort_flag, p.ws.status) ? 1 : 0;
+        *fix_ok = good;
+      }
+      epi_sync();
+      if (*fix_ok) {
+        const UnitInfo ui = decode_unit(p, park_u, n_rg, tiles_r, tiles_s);
+        const int g = group_of_unit(park_u, n_rg, tiles_r, tiles_s);
+        const int m = ui.gr.m;
+        const int N = (m + 15) & ~15;
+        const float tau = ui.shared ? p.tau_shared : p.tau;
+        const int row_i = 32 * q + lane;
+        const int j = ui.nt * kNeuronTile + row_i;
+        const int word = (ui.nt * kNeuronTile + 32 * q) >> 5;
+        __nv_bfloat16* row = ht + static_cast<size_t>(j) * ld + ui.gr.slot0;
+        uint32_t uni = 0;
+        unsigned long long nact = 0;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+          float gv[16], uv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) gv[i] = uv[i] = 0.f;
+          for (int c2 = c_first; c2 <= (int)blockIdx.x; ++c2) {
+            const int slot = c2 == (int)blockIdx.x ? gridDim.x + blockIdx.x : c2;
+            const float4* pg = reinterpret_cast<const float4*>(part_ptr(p, slot, 0, c0 / 16, row_i));
+            const float4* pu = reinterpret_cast<const float4*>(part_ptr(p, slot, 1, c0 / 16, row_i));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 a = __ldcg(pg + i), c = __ldcg(pu + i);
+              gv[4 * i] += a.x; gv[4 * i + 1] += a.y; gv[4 * i + 2] += a.z; gv[4 * i + 3] += a.w;
+              uv[4 * i] += c.x; uv[4 * i + 1] += c.y; uv[4 * i + 2] += c.z; uv[4 * i + 3] += c.w;
+            }
+          }
+          epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane);
+        }
+        epi_finish(p, ui, g, word, uni, nact, lane);
+      }
     }
   }
 

@@ -83,6 +83,7 @@ struct Dims {
   float gather_density;
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device
+  int sk_ctas;        // capacity of the gate/up split-unit flags (CTAs), 0: no split units
 };
 
 struct Workspace {
@@ -106,6 +107,8 @@ struct Workspace {
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
   int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
   int* y_zero;                  // [E+1] 1: expert's Y rows (last: shared experts') start at zero
+  int* sk_flags;                // [sk_ctas] gate/up: CTA c published its split-unit partial
+  float* sk_part;               // [2 * sk_ctas][2][128][n_max] gate/up split-unit partial sums
 
   uint32_t* act_bits;           // [slots_total][fw] or null (debug off)
   void* xperm;                  // [slots_routed][d] activations gathered by slot
@@ -127,6 +130,7 @@ struct GateUpTcParams {
   int stages;
   int nbuf;                    // TMEM accumulator buffers (1 or 2)
   uint32_t tmem_cols;          // allocated TMEM columns
+  int split;                   // 1: the leftover units after whole rounds are cut along K
 };
 
 // ------------------------------------------------------------ down (tcgen05)

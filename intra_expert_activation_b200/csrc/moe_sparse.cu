@@ -27,6 +27,16 @@ bool pdl_enabled() {
   }();
   return on;
 }
+
+// Gate/up split units (MOE_GATE_UP_SPLIT=0 turns them off; a scheduling
+// choice, the results are the same up to fp32 summation order).
+bool split_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_GATE_UP_SPLIT");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 }  // namespace moe
 
 namespace {
@@ -91,7 +101,7 @@ struct Layout {
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero,
+           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero, bSkFlags, bSkPart,
            bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
@@ -180,6 +190,14 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
   sz[bYZero] = sizeof(int) * (c.E + 1);
+  // gate/up split units (bf16): one flag per CTA and two partial slots per CTA,
+  // for up to 2 x 160 CTAs (2 per SM) when the groups hold <= 32 tokens, else 160
+  {
+    const int nm = std::min(roundup(std::min(c.T, moe::kGroupMax), 16), 64);  // cut only <= 64
+    c.sk_ctas = bf16 ? (nm <= 32 ? 320 : 160) : 0;
+    sz[bSkFlags] = sizeof(int) * (size_t)c.sk_ctas;
+    sz[bSkPart] = sizeof(float) * (size_t)2 * c.sk_ctas * 2 * moe::kNeuronTile * nm;
+  }
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;
   sz[bXperm] = es * (size_t)c.slots_routed * c.d;
   sz[bHt] = es * (size_t)c.F_max * c.slots_total;
@@ -359,6 +377,8 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
   w.y_zero = reinterpret_cast<int*>(b + o[bYZero]);
+  w.sk_flags = reinterpret_cast<int*>(b + o[bSkFlags]);
+  w.sk_part = reinterpret_cast<float*>(b + o[bSkPart]);
   w.act_bits = desc->debug ? reinterpret_cast<uint32_t*>(b + o[bActBits]) : nullptr;
   w.xperm = b + o[bXperm];
   w.ht = b + o[bHt];
@@ -501,6 +521,10 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
                           cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) *
                               (cap.Fs / moe::kNeuronTile);
     const int grid = std::max(1, std::min(units_max, ctas_per_sm * c->n_sms));
+    // leftover units are cut along K only for groups of <= 64 tokens: with
+    // 128-token groups (prefill) the parts' accumulators cost more than the
+    // uneven last round (measured: +24 us at T = 4096, d = 2048)
+    p.split = moe::split_enabled() && n_max <= 64 && grid <= cap.sk_ctas ? 1 : 0;
     e = moe::launch_gate_up_tc(p, grid, smem, st);
   } else {
     e = moe::launch_gate_up_simt(dm, c->ws, static_cast<const float*>(x),
