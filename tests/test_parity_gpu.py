@@ -169,6 +169,41 @@ def test_deterministic(small):
     assert np.array_equal(a, b)
 
 
+def test_graph_replay_parity(small):
+    """One forward captured into a CUDA graph, replayed on new inputs copied
+    into its input buffer: every replay matches the oracle on that input."""
+    T = 24
+    layer = make_layer(SMALL, 64)
+    xbuf = torch.empty((T, SMALL.d_model), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(xbuf)
+    x0 = make_tokens(SMALL.d_model, T, 30, "bf16")
+    tau, _ = _calibrated(small, x0, 0.7)
+
+    def fwd():
+        layer.forward(xbuf, small.W_router, small.W_gate, small.W_up, small.W_down, tau, 2,
+                      router_bias=small.bias, out=out)
+
+    xbuf.copy_(x0.cuda())
+    fwd()  # first call outside capture (one-time kernel attributes)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        fwd()
+    torch.cuda.synchronize()
+    for seed in (31, 32, 33):
+        x = make_tokens(SMALL.d_model, T, seed, "bf16")
+        xbuf.copy_(x.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        gpu = {"out": out.to(torch.float64).cpu().numpy()}
+        gpu.update({k: v.cpu().numpy() for k, v in layer.debug().items()})
+        compare(gpu, oracle_forward(small, x, tau), tau, 0.0, "bf16", dw=small)
+    assert layer.status() == 0
+    del g
+
+
 def test_timing_and_stats(small):
     x = make_tokens(SMALL.d_model, 64, 21, "bf16").cuda()
     layer = make_layer(SMALL, 64)
