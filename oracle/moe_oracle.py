@@ -18,8 +18,14 @@ path reads (bf16/fp32 storage values widened exactly):
    ``SiLU(g) = g / (1 + exp(-g))``.
 3. Threshold mask [gist.science EN, Technical Summary > Methodology >
    System Implementation in vLLM > "Activation Masking": one pass, a
-   threshold test per value, no sort]: neuron j is active iff
-   ``|h_j| > tau``; ``|h_j| <= tau`` is inactive.
+   threshold test per value, no sort]: neuron j is active iff its score
+   exceeds tau, at or below tau is inactive. Two scores:
+   ``score="h"``: the SwiGLU value, active iff ``|h_j| > tau``;
+   ``score="gate"``: the pages' own system, where the dense gate projection
+   alone produces the scores [same list, "Gate Projection"] and only the
+   active neurons' up and down weights are read afterwards ["Fused Up-Down
+   Projection"]: active iff ``|SiLU(g_j)| > tau``. In both modes an active
+   neuron contributes its full ``h_j = SiLU(g_j) u_j``.
 4. Down projection over the active neurons only [same list,
    "Fused Up-Down Projection"]: ``y = sum_{j active} h_j W_down[e][j, :]``,
    written as the product of the masked ``h`` with ``W_down[e]``: the
@@ -69,9 +75,11 @@ class LayerResult:
     out: np.ndarray                  # [T][d] float64
     router: RouterResult
     h: np.ndarray                    # [T][k][F] float64 SwiGLU values of routed pairs
-    active: np.ndarray               # [T][k][F] bool, |h| > tau
+    active: np.ndarray               # [T][k][F] bool, score > tau
     h_shared: Optional[np.ndarray]   # [S][T][Fs] or None
     active_shared: Optional[np.ndarray]
+    gate_abs: Optional[np.ndarray] = None         # [T][k][F] |SiLU(g)| of routed pairs
+    gate_abs_shared: Optional[np.ndarray] = None  # [S][T][Fs]
 
 
 def route(x, W_router, top_k: int, renormalize: bool, bias=None) -> RouterResult:
@@ -98,19 +106,35 @@ def route(x, W_router, top_k: int, renormalize: bool, bias=None) -> RouterResult
     return RouterResult(L, p, idx.astype(np.int64), w, gap)
 
 
-def swiglu(x_rows, W_gate_e, W_up_e) -> np.ndarray:
-    """Step 2: h = SiLU(x W_gate^T) * (x W_up^T) for rows of x, one expert."""
+def swiglu_parts(x_rows, W_gate_e, W_up_e):
+    """Step 2 in its two factors for rows of x, one expert:
+    ``SiLU(x W_gate^T)`` and ``x W_up^T``."""
     xr = _f64(x_rows)
     g = xr @ _f64(W_gate_e).T
     u = xr @ _f64(W_up_e).T
     with np.errstate(over="ignore"):
         silu = g / (1.0 + np.exp(-g))
+    return silu, u
+
+
+def swiglu(x_rows, W_gate_e, W_up_e) -> np.ndarray:
+    """Step 2: h = SiLU(x W_gate^T) * (x W_up^T) for rows of x, one expert."""
+    silu, u = swiglu_parts(x_rows, W_gate_e, W_up_e)
     return silu * u
 
 
-def active_mask(h: np.ndarray, tau: float) -> np.ndarray:
-    """Step 3: active iff |h| > tau (at or below tau is inactive)."""
-    return np.abs(h) > tau
+def active_mask(score: np.ndarray, tau: float) -> np.ndarray:
+    """Step 3: active iff |score| > tau (at or below tau is inactive)."""
+    return np.abs(score) > tau
+
+
+def score_of(silu_g: np.ndarray, h: np.ndarray, score: str) -> np.ndarray:
+    """The value whose magnitude step 3 compares with tau."""
+    if score == "gate":
+        return silu_g
+    if score == "h":
+        return h
+    raise ValueError(f"score must be 'h' or 'gate', not {score!r}")
 
 
 def down_projection(h: np.ndarray, active: np.ndarray, W_down_e) -> np.ndarray:
@@ -120,37 +144,46 @@ def down_projection(h: np.ndarray, active: np.ndarray, W_down_e) -> np.ndarray:
 
 def layer_forward(x, W_router, W_gate, W_up, W_down, tau: float, top_k: int,
                   renormalize: bool, router_bias=None, Ws_gate=None, Ws_up=None,
-                  Ws_down=None, tau_shared: float = 0.0, dense: bool = False) -> LayerResult:
+                  Ws_down=None, tau_shared: float = 0.0, dense: bool = False,
+                  score: str = "h") -> LayerResult:
     """Steps 1-5 for a batch x [T][d]. ``dense=True`` skips the threshold
-    (every neuron active), the layer's dense reference."""
+    (every neuron active), the layer's dense reference; ``score`` picks the
+    value compared with tau (step 3)."""
     x64 = _f64(x)
     T, d = x64.shape
     r = route(x64, W_router, top_k, renormalize, router_bias)
     E = r.logits.shape[1]
     F = W_gate.shape[1]
     h = np.zeros((T, top_k, F))
+    gabs = np.zeros((T, top_k, F))
     act = np.zeros((T, top_k, F), dtype=bool)
     y = np.zeros((T, top_k, d))
     for e in range(E):
         tt, ii = np.nonzero(r.topk_idx == e)
         if tt.size == 0:
             continue
-        he = swiglu(x64[tt], W_gate[e], W_up[e])
-        ae = np.ones_like(he, dtype=bool) if dense else active_mask(he, tau)
+        sg, u = swiglu_parts(x64[tt], W_gate[e], W_up[e])
+        he = sg * u
+        ae = np.ones_like(he, dtype=bool) if dense else active_mask(score_of(sg, he, score), tau)
         h[tt, ii] = he
+        gabs[tt, ii] = np.abs(sg)
         act[tt, ii] = ae
         y[tt, ii] = down_projection(he, ae, W_down[e])
     out = np.einsum("tk,tkd->td", r.topk_w, y)
-    hs = acts = None
+    hs = acts = gs = None
     if Ws_gate is not None and Ws_gate.shape[0] > 0:
         S, Fs = Ws_gate.shape[0], Ws_gate.shape[1]
         hs = np.zeros((S, T, Fs))
+        gs = np.zeros((S, T, Fs))
         acts = np.zeros((S, T, Fs), dtype=bool)
         for s in range(S):
-            hs[s] = swiglu(x64, Ws_gate[s], Ws_up[s])
-            acts[s] = np.ones_like(hs[s], dtype=bool) if dense else active_mask(hs[s], tau_shared)
+            sg, u = swiglu_parts(x64, Ws_gate[s], Ws_up[s])
+            hs[s] = sg * u
+            gs[s] = np.abs(sg)
+            acts[s] = np.ones_like(hs[s], dtype=bool) if dense else \
+                active_mask(score_of(sg, hs[s], score), tau_shared)
             out = out + down_projection(hs[s], acts[s], Ws_down[s])
-    return LayerResult(out, r, h, act, hs, acts)
+    return LayerResult(out, r, h, act, hs, acts, gabs, gs)
 
 
 def calibrate_tau(abs_h, q: float, round_f32: bool = True) -> float:
@@ -182,6 +215,15 @@ def routed_abs_h(layer: LayerResult) -> np.ndarray:
 
 def shared_abs_h(layer: LayerResult) -> np.ndarray:
     return np.abs(layer.h_shared).ravel()
+
+
+def routed_abs_gate(layer: LayerResult) -> np.ndarray:
+    """The calibration pool of the gate score: |SiLU(g)| over routed pairs."""
+    return layer.gate_abs.ravel()
+
+
+def shared_abs_gate(layer: LayerResult) -> np.ndarray:
+    return layer.gate_abs_shared.ravel()
 
 
 def measured_sparsity(abs_h: np.ndarray, tau: float) -> float:

@@ -2,8 +2,10 @@
 
 tau is the nearest-rank quantile of |h| over the calibration batch's routed
 (token, expert) pairs, computed by the CPU oracle in float64 and rounded to
-float32 (shared experts get their own pool and tau). Only the oracle and the
-seeded input generator run here; nothing comes from the CUDA path.
+float32 (shared experts get their own pool and tau). "taus_gate" holds the
+same quantiles of the gate score |SiLU(g)| for the gate-score variant. Only
+the oracle and the seeded input generator run here; nothing comes from the
+CUDA path.
 
     python tests/golden/make_tau_calibration.py [workload ...]
 """
@@ -34,15 +36,18 @@ def calibrate(wl):
              "calib_tokens": wl.calib_tokens, "weight_seed": wl.weight_seed,
              "pool_size": int(pool.size), "min_router_gap": float(res.router.gap.min()),
              "taus": {}}
-    for q in wl.sparsities:
-        tau = om.calibrate_tau(pool, q)
-        e = {"tau": tau, "measured_sparsity": om.measured_sparsity(pool, tau)}
-        if res.h_shared is not None:
-            spool = om.shared_abs_h(res)
-            ts = om.calibrate_tau(spool, q)
-            e["tau_shared"] = ts
-            e["measured_sparsity_shared"] = om.measured_sparsity(spool, ts)
-        entry["taus"][f"{q:.2f}"] = e
+    entry["taus_gate"] = {}
+    for key, rpool, spool_of in (("taus", pool, om.shared_abs_h),
+                                 ("taus_gate", om.routed_abs_gate(res), om.shared_abs_gate)):
+        for q in wl.sparsities:
+            tau = om.calibrate_tau(rpool, q)
+            e = {"tau": tau, "measured_sparsity": om.measured_sparsity(rpool, tau)}
+            if res.h_shared is not None:
+                spool = spool_of(res)
+                ts = om.calibrate_tau(spool, q)
+                e["tau_shared"] = ts
+                e["measured_sparsity_shared"] = om.measured_sparsity(spool, ts)
+            entry[key][f"{q:.2f}"] = e
     return entry
 
 

@@ -197,8 +197,10 @@ def test_masked_dense_equals_einsum_with_mask():
     assert _rel(res.out, ref) <= 1e-12
 
 
-def _scalar_brute_force(x, Wr, Wg, Wu, Wd, k, renorm, tau):
-    """Pure-Python scalar loops: each neuron enumerated, inactive rows skipped."""
+def _scalar_brute_force(x, Wr, Wg, Wu, Wd, k, renorm, tau, score="h"):
+    """Pure-Python scalar loops: each neuron enumerated, inactive rows skipped
+    (score "gate": the neuron's up and down rows are read only when
+    |SiLU(g)| > tau)."""
     T, d = len(x), len(x[0])
     E, F = len(Wg), len(Wg[0])
     out = [[0.0] * d for _ in range(T)]
@@ -214,9 +216,12 @@ def _scalar_brute_force(x, Wr, Wg, Wu, Wd, k, renorm, tau):
             w = p[e] / tot if renorm else p[e]
             for j in range(F):
                 g = sum(x[t][i] * Wg[e][j][i] for i in range(d))
+                silu = g / (1.0 + math.exp(-g))
+                if score == "gate" and abs(silu) <= tau:
+                    continue  # inactive by the gate score: up and down rows never read
                 u = sum(x[t][i] * Wu[e][j][i] for i in range(d))
-                h = g / (1.0 + math.exp(-g)) * u
-                if abs(h) <= tau:
+                h = silu * u
+                if score == "h" and abs(h) <= tau:
                     continue  # inactive neuron: its W_down row is never read
                 for c in range(d):
                     out[t][c] += w * h * Wd[e][j][c]
@@ -327,6 +332,68 @@ def test_threshold_is_strict():
     assert om.active_mask(h, 0.0).tolist() == [[False, True, True, True, True]]
 
 
+# ------------------------------------------------------- gate-score variant
+
+def test_gate_score_closed_form():
+    gs = _load("gate_score_closed_form.json")
+    g = _load("swiglu_closed_form.json")
+    ln3 = math.log(3.0)
+    x = np.array(g["x"])
+    Wr = np.array(g["W_router"])
+    Wg = np.array(g["W_gate_ln3"]) * ln3
+    Wu = np.array(g["W_up"])
+    Wd = np.array(g["W_down"])
+    base = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 1, True, score="gate")
+    np.testing.assert_allclose(base.gate_abs[0, 0], np.array(gs["score_over_ln3"]) * ln3,
+                               rtol=1e-15, atol=1e-15)
+    for case in gs["cases"]:
+        tau = case["tau_over_ln3"] * ln3
+        for mode, key in (("gate", "gate"), ("h", "h")):
+            res = om.layer_forward(x, Wr, Wg, Wu, Wd, tau, 1, True, score=mode)
+            assert res.active[0, 0].tolist() == case[f"active_{key}"], (mode, case)
+            np.testing.assert_allclose(res.out[0], np.array(case[f"out_{key}_over_ln3"]) * ln3,
+                                       rtol=1e-14, atol=1e-14)
+
+
+def test_gate_mode_micro_scalar_brute_force():
+    rng = np.random.default_rng(18)
+    x, Wr, Wg, Wu, Wd, _ = _rand_layer(rng, 3, 4, 3, 6)
+    base = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 2, True, score="gate")
+    for q in (0.0, 0.5, 0.8):
+        tau = om.calibrate_tau(om.routed_abs_gate(base), q)
+        res = om.layer_forward(x, Wr, Wg, Wu, Wd, tau, 2, True, score="gate")
+        ref = _scalar_brute_force(x.tolist(), Wr.tolist(), Wg.tolist(), Wu.tolist(),
+                                  Wd.tolist(), 2, True, tau, score="gate")
+        assert _rel(res.out, ref) <= 1e-12 or np.linalg.norm(ref) == 0.0
+
+
+def test_gate_mode_tau0_equals_dense():
+    rng = np.random.default_rng(19)
+    x, Wr, Wg, Wu, Wd, _ = _rand_layer(rng, 9, 16, 5, 24)
+    res = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 2, True, score="gate")
+    ref = _dense_moe_einsum(x, Wr, Wg, Wu, Wd, 2, True)
+    assert _rel(res.out, ref) <= 1e-12
+
+
+def test_gate_mode_active_sets_nest_and_shared_threshold():
+    rng = np.random.default_rng(20)
+    x, Wr, Wg, Wu, Wd, sh = _rand_layer(rng, 6, 16, 4, 32, S=1, Fs=24)
+    base = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 2, True, score="gate", **sh)
+    pool = om.routed_abs_gate(base)
+    prev = None
+    for q in (0.2, 0.5, 0.8):
+        tau = om.calibrate_tau(pool, q)
+        res = om.layer_forward(x, Wr, Wg, Wu, Wd, tau, 2, True, score="gate", **sh)
+        assert np.array_equal(res.active, res.gate_abs > tau)
+        assert np.array_equal(res.active_shared, res.gate_abs_shared > 0.0)  # tau_shared = 0
+        if prev is not None:
+            assert not np.any(res.active & ~prev)  # a higher tau keeps a subset
+        prev = res.active
+    ts = om.calibrate_tau(om.shared_abs_gate(base), 0.5)
+    res = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 2, True, score="gate", tau_shared=ts, **sh)
+    assert np.array_equal(res.active_shared, res.gate_abs_shared > ts)
+
+
 # ------------------------------------------------ planted mistakes are caught
 
 def _run_pins():
@@ -336,7 +403,8 @@ def _run_pins():
                test_calibration_nearest_rank_hand_values, test_tau0_equals_dense_brute_force,
                test_micro_shape_scalar_brute_force, test_threshold_is_strict,
                test_unrenormalised_weights_are_top_probabilities,
-               test_renormalised_weights_sum_to_one):
+               test_renormalised_weights_sum_to_one, test_gate_score_closed_form,
+               test_gate_mode_micro_scalar_brute_force):
         try:
             fn()
         except AssertionError:
@@ -350,10 +418,22 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     def silu_sign(xr, Wg_e, Wu_e):
         g = F64(xr) @ F64(Wg_e).T
-        return g / (1.0 + np.exp(g)) * (F64(xr) @ F64(Wu_e).T)
+        return g / (1.0 + np.exp(g)), F64(xr) @ F64(Wu_e).T
 
     def gate_up_swapped(xr, Wg_e, Wu_e):
-        return om.__dict__["_orig_swiglu"](xr, Wu_e, Wg_e)
+        return om.__dict__["_orig_parts"](xr, Wu_e, Wg_e)
+
+    def score_always_h(silu_g, h, score):
+        return h
+
+    def score_pre_activation(silu_g, h, score):
+        # the gate's pre-activation instead of SiLU(g): g = SiLU(g) / sigmoid(g)
+        if score != "gate":
+            return h
+        g = np.where(silu_g == 0.0, 0.0, silu_g)
+        for _ in range(60):  # invert SiLU by fixed point g = s (1 + e^-g)
+            g = silu_g * (1.0 + np.exp(-np.clip(g, -30, 30)))
+        return g
 
     def down_transposed(h, act, Wd_e):
         W = F64(Wd_e)
@@ -386,8 +466,9 @@ def test_planted_mistakes_are_caught(monkeypatch):
         r = min(int(math.ceil(q * a.size)), a.size - 1)
         return float(np.float32(a[r])) if round_f32 else float(a[r])
 
-    om.__dict__["_orig_swiglu"] = om.swiglu
-    mutants = [("swiglu", silu_sign), ("swiglu", gate_up_swapped),
+    om.__dict__["_orig_parts"] = om.swiglu_parts
+    mutants = [("swiglu_parts", silu_sign), ("swiglu_parts", gate_up_swapped),
+               ("score_of", score_always_h), ("score_of", score_pre_activation),
                ("down_projection", down_transposed), ("active_mask", mask_ge),
                ("route", no_renorm), ("route", tie_high), ("calibrate_tau", cal_off_by_one)]
     for name, fn in mutants:
