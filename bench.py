@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="mixtral_decode")
     ap.add_argument("--sparsity", type=float, default=0.7)
+    ap.add_argument("--score", choices=("h", "gate"), default="h",
+                    help="h: active iff |SiLU(g) u| > tau; gate: active iff |SiLU(g)| > tau with "
+                         "the sparse up projection (the pages' own system)")
     ap.add_argument("--tokens", type=str, default="", help="comma list overriding the batches")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -65,9 +68,9 @@ def parse():
     return ap.parse_args()
 
 
-def load_tau(workload: str, q: float):
+def load_tau(workload: str, q: float, score: str = "h"):
     with open(os.path.join(ROOT, "tests", "golden", "tau_calibration.json")) as f:
-        e = json.load(f)[workload]["taus"][f"{q:.2f}"]
+        e = json.load(f)[workload]["taus_gate" if score == "gate" else "taus"][f"{q:.2f}"]
     return e["tau"], e.get("tau_shared", 0.0), e["measured_sparsity"]
 
 
@@ -174,7 +177,8 @@ def replica_value(tokens_per_step: int, steps: int, world: int, ms: float) -> fl
 def workload_config(args, wl, tokens, tau, calib_sparsity, world) -> dict:
     """The config block both arms print for a workload."""
     sh = wl.shape
-    return {"workload": args.workload, "batches": tokens, "tokens_per_step": sum(tokens),
+    return {"workload": args.workload, "score": args.score, "batches": tokens,
+            "tokens_per_step": sum(tokens),
             "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
             "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
             "calibrated_sparsity": round(calib_sparsity, 4),
@@ -184,7 +188,7 @@ def workload_config(args, wl, tokens, tau, calib_sparsity, world) -> dict:
 
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_step_time(wl, tokens, tau, tau_s, w_host):
+def oracle_step_time(wl, tokens, tau, tau_s, w_host, score="h"):
     from oracle import moe_oracle as om
     sh = wl.shape
     t0 = time.perf_counter()
@@ -193,7 +197,7 @@ def oracle_step_time(wl, tokens, tau, tau_s, w_host):
         om.layer_forward(x, w_host.W_router, w_host.W_gate, w_host.W_up, w_host.W_down, tau,
                          sh.top_k, sh.renormalize, router_bias=w_host.router_bias,
                          Ws_gate=w_host.Ws_gate, Ws_up=w_host.Ws_up, Ws_down=w_host.Ws_down,
-                         tau_shared=tau_s)
+                         tau_shared=tau_s, score=score)
     return time.perf_counter() - t0
 
 
@@ -205,12 +209,12 @@ def run_reference(args, world, rank):
         return 0
     wl = WORKLOADS[args.workload]
     tokens = [int(t) for t in args.tokens.split(",")] if args.tokens else list(wl.tokens)
-    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity)
+    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity, args.score)
     w = make_weights(wl.shape, wl.weight_seed)
     sample = [8] if 8 in tokens else [min(tokens)]
     for _ in range(args.warmup):
-        oracle_step_time(wl, sample, tau, tau_s, w)
-    t = sum(oracle_step_time(wl, sample, tau, tau_s, w) for _ in range(args.steps))
+        oracle_step_time(wl, sample, tau, tau_s, w, args.score)
+    t = sum(oracle_step_time(wl, sample, tau, tau_s, w, args.score) for _ in range(args.steps))
     toks = sum(sample) * args.steps
     cores = len(os.sched_getaffinity(0))
     value = toks / t
@@ -239,7 +243,7 @@ def run_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     sh = wl.shape
     tokens = [int(t) for t in args.tokens.split(",")] if args.tokens else list(wl.tokens)
-    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity)
+    tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity, args.score)
     w_host = make_weights(sh, wl.weight_seed)
     mv = lambda t: None if t is None else t.to(dev).contiguous()
     W = {k: mv(getattr(w_host, k)) for k in ("W_router", "W_gate", "W_up", "W_down",
@@ -253,7 +257,8 @@ def run_ours(args, world, rank, local):
     def make(path):
         L = MoESparseLayer(sh.d_model, sh.d_ff, sh.n_experts, sh.top_k, tmax,
                            renormalize=sh.renormalize, n_shared=sh.n_shared,
-                           d_ff_shared=sh.d_ff_shared, dtype=sh.dtype, path=path, device=local)
+                           d_ff_shared=sh.d_ff_shared, dtype=sh.dtype, path=path, device=local,
+                           score=args.score if path != "dense" else "h")
         if sh.n_shared:
             L.set_shared(W["Ws_gate"], W["Ws_up"], W["Ws_down"], tau_s)
         return L
@@ -389,15 +394,24 @@ def run_ours(args, world, rank, local):
 
     per_T = []
     gate_bytes_tot = gate_ms_tot = down_bytes_tot = down_ms_tot = 0.0
+    up_bytes_tot = up_ms_tot = 0.0
     for i, T in enumerate(tokens):
         st = stats[i]
         P = T * sh.top_k
         touched = st["n_experts_touched"]
-        g_bytes = touched * 2 * sh.d_ff * sh.d_model * esize + P * sh.d_model * esize \
-            + P * sh.d_ff * esize
-        if sh.n_shared:
-            g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
+        if args.score == "gate":  # W_gate of every unit, W_up only where it ran densely
+            g_bytes = st["gate_up_rows_read"] * sh.d_model * esize + P * sh.d_model * esize \
+                + P * sh.d_ff * esize
+        else:
+            g_bytes = touched * 2 * sh.d_ff * sh.d_model * esize + P * sh.d_model * esize \
+                + P * sh.d_ff * esize
+            if sh.n_shared:
+                g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
         d_bytes = st["down_rows_read"] * sh.d_model * esize
+        u_bytes = st["up_rows_read"] * sh.d_model * esize
+        u_ms = avg_stage(per_fwd, i, "up_gemv")
+        up_bytes_tot += u_bytes * args.steps
+        up_ms_tot += u_ms * args.steps
         g_ms = avg_stage(per_fwd, i, "gate_up")
         d_ms = avg_stage(per_fwd, i, "down_gemv") + avg_stage(per_fwd, i, "down_tc")
         fwd_ms = sum(avg_stage(per_fwd, i, s) for s in per_fwd[0]) if per_fwd else 0.0
@@ -417,6 +431,8 @@ def run_ours(args, world, rank, local):
             round(lat_dense[i] / lat_sparse[i], 3),
             "down_rows_read": st["down_rows_read"],
             "down_rows_dense": touched * sh.d_ff,
+            "up_rows_read": st["up_rows_read"],
+            "gate_up_rows_read": st["gate_up_rows_read"],
             "groups": {"gemv": st["n_groups_gemv"], "tc_gather": st["n_groups_tc_gather"],
                        "tc_allrows": st["n_groups_tc_allrows"]},
             "stage_us": {k: round(1e3 * avg_stage(per_fwd, i, k), 2) for k in
@@ -426,15 +442,17 @@ def run_ours(args, world, rank, local):
             "speedup_vs_dense": None if not fwd_dense else round(fwd_dense / fwd_ms, 3),
             "gate_up_GBps": round(g_bytes / (g_ms * 1e-3) / 1e9, 1) if g_ms else None,
             "down_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1) if d_ms else None,
+            "up_GBps": round(u_bytes / (u_ms * 1e-3) / 1e9, 1) if u_ms else None,
             "dense_down_us": None if d_dense is None else round(1e3 * d_dense, 2),
         })
 
     peak, peak_kind = peaks()
     g_ach = gate_bytes_tot / (gate_ms_tot * 1e-3) / 1e9 if gate_ms_tot else 0.0
     n_gate_launches = args.steps * len(tokens)
-    g_traffic = None if GATE_UP_TRAFFIC_RATIO is None else \
+    g_traffic = None if GATE_UP_TRAFFIC_RATIO is None or args.score != "h" else \
         round(GATE_UP_TRAFFIC_RATIO * gate_bytes_tot / n_gate_launches)
     d_ach = down_bytes_tot / (down_ms_tot * 1e-3) / 1e9 if down_ms_tot else 0.0
+    u_ach = up_bytes_tot / (up_ms_tot * 1e-3) / 1e9 if up_ms_tot else 0.0
     steps_launches = launches
 
     # end to end through the public API with host buffers
@@ -470,7 +488,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t = oracle_step_time(wl, tokens, tau, tau_s, w_host)
+        t = oracle_step_time(wl, tokens, tau, tau_s, w_host, args.score)
         cores = len(os.sched_getaffinity(0))
         cpu = {"value": tok_step / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": f"one step: decode batches T={tokens} of {args.workload} through the "
@@ -491,6 +509,10 @@ def run_ours(args, world, rank, local):
             "roofline_down": {"kernel": "down (GEMV / TC, rows actually read)", "bound": "hbm",
                               "achieved": round(d_ach, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(d_ach / peak, 4), "peak_kind": peak_kind},
+            "roofline_up": None if args.score != "gate" else
+            {"kernel": "up_gemv (gate score: W_up rows actually read)", "bound": "hbm",
+             "achieved": round(u_ach, 1), "peak": peak, "unit": "GB/s",
+             "frac": round(u_ach / peak, 4), "peak_kind": peak_kind},
             "dense": dense_line,
             "speedup_vs_dense": None if not dense_line else
             round(dense_line["ms_per_step"] / (ms_sparse / args.steps), 4),

@@ -32,6 +32,16 @@
  *   Switching"] is made per expert token group on the device from the
  *   group's token count and the size of its active-row union.
  *
+ * Gate score (desc.score = MOE_SCORE_GATE), the pages' own system: step 3
+ * tests the gate projection alone, neuron j is active iff |SiLU(g_j)| > tau
+ * [same list, "Gate Projection" and "Activation Masking"], and for the
+ * small expert token groups (the GEMV path) the up projection of step 2 is
+ * computed only for the group's active-row union, reading only those W_up
+ * rows [same list, "Fused Up-Down Projection": only the active neurons'
+ * up and down weights are fetched]. An active neuron still contributes its
+ * full h_j = SiLU(g_j) u_j. Larger groups compute the up projection densely
+ * and apply the same gate-score mask.
+ *
  * Conventions shared by every entry point
  *   - Tensors are DEVICE pointers on desc.device, contiguous, row-major,
  *     16-byte aligned, in desc.dtype (x, weights, out), except router_bias
@@ -83,6 +93,11 @@ typedef enum {
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
 typedef enum {
+  MOE_SCORE_H = 0,            /* active iff |h| > tau, h = SiLU(g) u */
+  MOE_SCORE_GATE = 1          /* active iff |SiLU(g)| > tau; sparse up projection */
+} moe_score;
+
+typedef enum {
   MOE_PATH_AUTO = 0,          /* threshold on; per group: GEMV, gathered TC or all-rows TC */
   MOE_PATH_DENSE = 1,         /* no threshold: every neuron active (the dense baseline) */
   MOE_PATH_SPARSE_GEMV = 2,   /* threshold on; every group on the CUDA-core row stream */
@@ -105,6 +120,7 @@ typedef struct {
   int32_t device;             /* CUDA device ordinal */
   int32_t gemv_max_tokens;    /* AUTO: groups with <= this many tokens use the GEMV path (0: 4) */
   float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: never) */
+  int32_t score;              /* moe_score (0: MOE_SCORE_H) */
 } moe_sparse_desc;
 
 typedef struct {
@@ -118,6 +134,8 @@ typedef struct {
   int64_t n_groups_tc_gather;
   int64_t n_groups_tc_allrows;
   int64_t n_experts_touched;  /* routed experts with at least one token */
+  int64_t up_rows_read;       /* W_up rows streamed by the sparse up projection (gate score) */
+  int64_t gate_up_rows_read;  /* W_gate + W_up rows loaded by the gate/up projection */
 } moe_stats;
 
 typedef struct moe_sparse_ctx moe_sparse_ctx;

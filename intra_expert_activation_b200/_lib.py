@@ -23,10 +23,13 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID", 2: "MOE_ERR_UNSUPPORTED", 3: 
 
 MOE_F32 = 0
 MOE_BF16 = 1
+MOE_SCORE_H = 0
+MOE_SCORE_GATE = 1
+SCORES = {"h": MOE_SCORE_H, "gate": MOE_SCORE_GATE}
 
 PATHS = {"auto": 0, "dense": 1, "sparse_gemv": 2, "sparse_tc": 3, "sparse_tc_allrows": 4}
 
-STAGES = ("route", "permute", "gate_up", "union_scan", "down_gemv", "down_tc", "combine")
+STAGES = ("route", "permute", "gate_up", "union_scan", "up_gemv", "down_gemv", "down_tc", "combine")
 
 
 class moe_sparse_desc(ctypes.Structure):
@@ -45,6 +48,7 @@ class moe_sparse_desc(ctypes.Structure):
         ("device", ctypes.c_int32),
         ("gemv_max_tokens", ctypes.c_int32),
         ("gather_max_density", ctypes.c_float),
+        ("score", ctypes.c_int32),
     ]
 
 
@@ -52,7 +56,7 @@ class moe_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "n_routed_h", "n_routed_active", "n_shared_h", "n_shared_active", "down_rows_read",
         "n_groups", "n_groups_gemv", "n_groups_tc_gather", "n_groups_tc_allrows",
-        "n_experts_touched")]
+        "n_experts_touched", "up_rows_read", "gate_up_rows_read")]
 
 
 _vp = ctypes.c_void_p

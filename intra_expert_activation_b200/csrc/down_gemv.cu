@@ -32,298 +32,16 @@
 // (zeroed by the router) with vector fp32 atomics: the partials of a unit are
 // summed in arrival order, so results agree to fp32 rounding, not bitwise,
 // between runs on this path.
-#include "common.cuh"
+#include "gemv_common.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kConsumers = 8;
-constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
-constexpr int kBatch = 8;            // rows per stage (the mma's K)
-constexpr int kSliceBytes = 512;     // row bytes per consumer warp
-constexpr int kBlockBytes = kConsumers * kSliceBytes;  // column block: 4 KB of a row
-constexpr int kRowPad = 16;          // row stride = block bytes + 16
 constexpr int kHBytes = 32;          // h bytes per row: 4 x bf16 or 8 x fp32
-constexpr int kMaxStages = 6;
-constexpr int kSmemBudget = 190 * 1024;  // stages; the result staging comes on top
-constexpr int kListRows = 256;       // producer's row list (uint16 neuron indices)
-constexpr int kTight = 4096;         // barrier probes before sleeping: stages arrive every few us
 constexpr int kYStride = 260;        // floats per staged result row of a consumer warp
 constexpr int kYBytes = kGemvTokens * kYStride * 4;  // a consumer warp's result staging
-
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
-// Packed pair of fp32 values and d = a * b + d on both halves.
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-__device__ __forceinline__ void fma2(uint64_t& d, uint64_t a, uint64_t b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
-}
-
-// Four 8x8 bf16 matrices from shared memory, transposed (lane i supplies the
-// address of row i % 8 of matrix i / 8).
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-// d += A (16 x 8, bf16) * B (8 x 8, bf16), fp32 accumulation.
-__device__ __forceinline__ void mma_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-// Arrive on bar once this thread's earlier cp.async copies have landed (the
-// barrier's expected count includes this arrival).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16) from global to shared memory,
-// completion counted on bar as transaction bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-// Stage geometry for a row of row_bytes: the column block (<= 4 KB), the
-// stage size and the number of stages that fit the budget.
-struct Geometry {
-  int block, stride, stage, n_stages;
-};
-__host__ __device__ inline Geometry geometry(int row_bytes) {
-  Geometry g;
-  g.block = row_bytes < kBlockBytes ? row_bytes : kBlockBytes;
-  g.stride = g.block + kRowPad;
-  g.stage = kBatch * g.stride + kBatch * kHBytes + 16;  // rows | h | meta
-  g.n_stages = kSmemBudget / g.stage;
-  if (g.n_stages > kMaxStages) g.n_stages = kMaxStages;
-  return g;
-}
-
-// Where a CTA's share of the row sequence starts.
-struct Start {
-  int i;        // GEMV list index of the first group
-  int p;        // pass within it
-  int w;        // bitmap word of the first row
-  uint32_t m;   // mask of the rows of word w that are still to come
-  int rows;     // rows of this CTA
-  int g, row;   // the first group and the row within its pass (prologue scratch)
-};
-
-// The producer's walk over its CTA's rows: group list index, pass, next word
-// and the mask for it, rows still to produce, and the unit being produced.
-struct Walk {
-  int i, p, w;
-  uint32_t m;
-  int left;
-  int n_gv;  // GEMV groups
-  int g, words, passes, slot0, m_tok, expert;  // unit data of group i
-  int serial;  // increments whenever the unit (group, pass) changes
-};
-
-// Loads group i's unit data; false past the end of the GEMV list.
-__device__ __forceinline__ bool walk_load_group(const Dims& dm, const Workspace& ws, Walk& k,
-                                                int MT) {
-  if (k.i >= k.n_gv) return false;
-  k.g = __ldcg(ws.gemv_list + k.i);
-  const Group gr = ws.groups[k.g];
-  k.expert = gr.expert;
-  k.slot0 = gr.slot0;
-  k.m_tok = gr.m;
-  k.passes = (gr.m + MT - 1) / MT;
-  k.words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
-  return true;
-}
-
-// Next run of rows of one unit into the list: the set bits of up to 32
-// bitmap words (one per lane), at most kListRows and at most k.left rows.
-// Returns the number of rows (0 once the walk is over). Whole warp.
-__device__ int walk_next(const Dims& dm, const Workspace& ws, Walk& k, uint16_t* list, int MT,
-                         int lane) {
-  int n = 0;
-  while (k.left > 0) {
-    if (k.w >= k.words) {  // unit finished: next pass, or the next group with rows
-      k.w = 0;
-      k.m = ~0u;
-      ++k.serial;
-      if (++k.p >= k.passes) {
-        k.p = 0;
-        bool ok;
-        do {
-          ++k.i;
-          ok = walk_load_group(dm, ws, k, MT);
-        } while (ok && __ldcg(ws.union_cnt + k.g) == 0);
-        if (!ok) {  // the union counts and the bitmaps disagree
-          if (lane == 0) report_error(ws.status, kErrDeviceInvalid);
-          k.left = 0;
-          break;
-        }
-      }
-      continue;
-    }
-    const int word = k.w + lane;
-    uint32_t bits = word < k.words ? __ldcg(ws.union_bits + (size_t)k.g * dm.fw + word) : 0u;
-    if (lane == 0) bits &= k.m;
-    const int c = __popc(bits);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    const int excl = incl - c;
-    const int cap = min(kListRows, k.left);
-    const int take = min(max(cap - excl, 0), c);  // this lane's rows: its lowest `take` bits
-    uint32_t bb = bits;
-    int pos = excl;
-    for (int t = 0; t < take; ++t) {
-      list[pos++] = static_cast<uint16_t>(32 * word + __ffs(bb) - 1);
-      bb &= bb - 1;
-    }
-    // the first lane that did not take all of its word holds the cursor
-    const unsigned short_lanes = __ballot_sync(0xffffffffu, take < c);
-    n = min(cap, __shfl_sync(0xffffffffu, incl, 31));
-    if (short_lanes) {
-      const int l = __ffs(short_lanes) - 1;
-      k.m = __shfl_sync(0xffffffffu, bb, l);  // the rows of that word not taken yet
-      k.w += l;
-    } else {
-      k.w += 32;
-      k.m = ~0u;
-    }
-    k.left -= n;
-    if (n > 0) break;
-  }
-  __syncwarp();  // list entries are read by every lane
-  return n;
-}
-
-// The CTA's share of rows and where it starts. Every thread calls it.
-__device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* st,
-                           long long* sm_warp) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nw = blockDim.x / 32;
-  // the first list entries are read while the list length is still in
-  // flight (they are inside the list's capacity either way)
-  const int g_spec = tid < dm.groups_max ? __ldcg(ws.gemv_list + tid) : 0;
-  const int n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
-  // rows of each GEMV group (all passes); one sweep when the groups fit the
-  // CTA, else a first sweep for the total
-  const bool one = n_gv <= (int)blockDim.x;
-  long long lo = 0;
-  if (tid == 0) {
-    st->i = -1;
-    st->rows = 0;
-  }
-  for (int sweep = one ? 1 : 0; sweep < 2; ++sweep) {
-    long long carry = 0;
-    for (int base = 0; base < n_gv; base += blockDim.x) {
-      const int i = base + tid;
-      long long v = 0;
-      int g = 0, cnt = 0, words = 0;
-      if (i < n_gv) {
-        g = base == 0 ? g_spec : __ldcg(ws.gemv_list + i);
-        cnt = __ldcg(ws.union_cnt + g);
-        const Group gr = ws.groups[g];
-        v = (long long)((gr.m + MT - 1) / MT) * cnt;
-        words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
-      }
-      long long incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const long long u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (lane == 31) sm_warp[warp] = incl;
-      __syncthreads();
-      long long before = 0, chunk = 0;
-      for (int w = 0; w < nw; ++w) {
-        const long long x = sm_warp[w];
-        if (w < warp) before += x;
-        chunk += x;
-      }
-      const long long excl = carry + before + incl - v;
-      if (sweep == 1) {
-        if (one) {  // the total is known now
-          lo = chunk * blockIdx.x / gridDim.x;
-          if (tid == 0) st->rows = (int)(chunk * (blockIdx.x + 1) / gridDim.x - lo);
-        }
-        if (v > 0 && excl <= lo && lo < excl + v) {
-          const long long off = lo - excl;
-          st->i = i;
-          st->p = (int)(off / cnt);
-          st->g = g;
-          st->row = (int)(off % cnt);
-          st->w = words;  // the group's word count, until warp 0 positions the cursor
-        }
-      }
-      carry += chunk;
-      __syncthreads();
-    }
-    if (sweep == 0) {
-      lo = carry * blockIdx.x / gridDim.x;
-      if (tid == 0) st->rows = (int)(carry * (blockIdx.x + 1) / gridDim.x - lo);
-    }
-  }
-  __syncthreads();
-  if (st->rows <= 0 || st->i < 0) return;  // uniform
-  // warp 0: the bitmap word holding row st->row of group st->g
-  if (warp == 0) {
-    const int g = st->g, words = st->w;
-    int skip = st->row;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-      const uint32_t bits =
-          w0 + lane < words ? __ldcg(ws.union_bits + (size_t)g * dm.fw + w0 + lane) : 0u;
-      const int c = __popc(bits);
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      const int excl = incl - c;
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-      __syncwarp();  // every lane has read st->w before the owner lane rewrites it
-      if (excl <= skip && skip < incl) {  // this lane's word holds the first row
-        uint32_t m = bits;
-        for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
-        st->w = w0 + lane;
-        st->m = m;
-      }
-      if (skip < total) break;
-      skip -= total;
-    }
-  }
-  __syncthreads();
-}
+constexpr int kStageExtra = kBatch * kHBytes + 16;   // per stage after the rows: h | meta
 
 template <typename TW>
 struct Rows;
@@ -452,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int row_bytes = d * ES;
-  const Geometry geo = geometry(row_bytes);
+  const Geometry geo = geometry(row_bytes, kStageExtra);
   const int NS = geo.n_stages;
   const int n_blocks = (row_bytes + kBlockBytes - 1) / kBlockBytes;
 
@@ -589,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t down_gemv_smem_bytes(int d, bool bf16) {
-  const Geometry g = geometry(d * (bf16 ? 2 : 4));
+  const Geometry g = geometry(d * (bf16 ? 2 : 4), kStageExtra);
   return static_cast<size_t>(g.n_stages) * g.stage + (bf16 ? kConsumers * kYBytes : 0);
 }
 

@@ -2,7 +2,9 @@
 // cores, for layers stored in fp32 (the tensor cores' tf32 mode would not
 // keep the fp32 accuracy). Same outputs as the tensor-core kernel: masked h
 // transposed into H^T[neuron][slot] (fp32 here), the group's active-row
-// union bitmap and, with debugging on, per-slot active bitmaps.
+// union bitmap and, with debugging on, per-slot active bitmaps. With the
+// gate score only the gate projection runs here and H^T receives the masked
+// SiLU(g) (the sparse up kernel completes h).
 // [gist.science EN "Uncovering Intra-expert Activation Sparsity for Efficient
 // Mixture-of-Expert Model Execution", Technical Summary > Methodology >
 // System Implementation in vLLM > "Gate Projection" and "Activation Masking"]
@@ -55,6 +57,7 @@ __global__ void __launch_bounds__(kThreads)
                               : Wu + static_cast<size_t>(gr.expert) * F_e * d;
     const float* X = shared ? x : xperm;
     const float th = shared ? tau_shared : tau;
+    const bool gate_only = dm.score_gate != 0;
 
     for (int t = threadIdx.x; t < gr.m; t += kThreads) tok_bits[t] = 0u;
     if (threadIdx.x == 0) uni = 0u;
@@ -70,15 +73,18 @@ __global__ void __launch_bounds__(kThreads)
         for (int i = lane; i < d; i += 32) {
           const float xv = xr[i];
           gs = fmaf(xv, wg[i], gs);
-          us = fmaf(xv, wu[i], us);
+          if (!gate_only) us = fmaf(xv, wu[i], us);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           gs += __shfl_xor_sync(0xffffffffu, gs, o);
           us += __shfl_xor_sync(0xffffffffu, us, o);
         }
-        const float h = silu_f32(gs) * us;
-        const bool act = dense || fabsf(h) > th;
+        // gate score: active iff |SiLU(g)| > tau, and the masked SiLU(g) is
+        // stored for the sparse up kernel (every fp32 group is on the GEMV path)
+        const float sg = silu_f32(gs);
+        const float h = gate_only ? sg : sg * us;
+        const bool act = dense || fabsf(gate_only ? sg : h) > th;
         if (lane == 0) {
           ht[static_cast<size_t>(j) * ld + gr.slot0 + t] = act ? h : 0.f;
           if (act) atomicOr(&tok_bits[t], 1u << (j & 31));
@@ -98,6 +104,7 @@ __global__ void __launch_bounds__(kThreads)
     if (threadIdx.x == 0) {
       ws.union_bits[static_cast<size_t>(g) * dm.fw + blk] = uni;
       if (uni) atomicAdd(ws.union_cnt + g, __popc(uni));
+      atomicAdd(ws.counters + kCntGateUpRows, (gate_only ? 1ull : 2ull) * 32ull);
     }
     __syncthreads();
   }

@@ -10,6 +10,11 @@
 // h = SiLU(g) * u. The threshold test |h| > tau is one pass over the
 // accumulators with no sort [same list, "Activation Masking"].
 //
+// With the gate score (dm.score_gate) a neuron is active iff |SiLU(g)| > tau
+// [same list, "Gate Projection" and "Activation Masking"]; units of groups
+// on the GEMV path then load and multiply W_gate only and store the masked
+// SiLU(g) in H^T, and the sparse up kernel forms h for the active rows.
+//
 // Work unit: (expert token group, 128-neuron tile), full K = d_model.
 //   D_gate[128 neurons][N tokens] = W_gate[e][tile rows] . X_group^T
 //   D_up  [128 neurons][N tokens] = W_up  [e][tile rows] . X_group^T
@@ -54,6 +59,7 @@ struct UnitInfo {
   int shared;     // 0 routed, 1 shared
   int F_e;
   int wrow;       // first weight row in the 2-D [experts*F][d] view
+  int gate_only;  // gate score and a GEMV group: the up projection is left to the sparse kernel
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, int n_rg,
@@ -71,6 +77,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, 
     ui.shared = 1;
   }
   ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
+  ui.gate_only = p.dm.score_gate && __ldcg(p.ws.group_path + g) == kPathGemv;
   ui.F_e = ui.shared ? p.dm.Fs : p.dm.F;
   const int e_local = ui.shared ? ui.gr.expert - p.dm.E : ui.gr.expert;
   ui.wrow = e_local * ui.F_e + ui.nt * kNeuronTile;
@@ -146,6 +153,8 @@ __device__ __forceinline__ float* part_ptr(const GateUpTcParams& p, int slot, in
 
 // SwiGLU, threshold and compaction of 16 columns (tokens c0 .. c0+15) of one
 // neuron row: masked h to H^T, warp ballots into the union word and counts.
+// The score is |h| or, with the gate score, |SiLU(g)|; a gate-only unit
+// (sparse up projection to follow) stores the masked SiLU(g) in place of h.
 __device__ __forceinline__ void epi_chunk(const GateUpTcParams& p, const UnitInfo& ui, int word,
                                           int c0, int m, float tau, const float (&gv)[16],
                                           const float (&uv)[16], __nv_bfloat16* row,
@@ -155,8 +164,9 @@ __device__ __forceinline__ void epi_chunk(const GateUpTcParams& p, const UnitInf
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int c = c0 + i;
-    const float h = silu_f32(gv[i]) * uv[i];
-    const bool act = p.dense || fabsf(h) > tau;
+    const float sg = silu_f32(gv[i]);
+    const float h = ui.gate_only ? sg : sg * uv[i];
+    const bool act = p.dense || fabsf(p.dm.score_gate ? sg : h) > tau;
     hv[i] = act ? h : 0.f;
     const uint32_t mask = __ballot_sync(0xffffffffu, act && c < m);
     uni |= mask;
@@ -291,11 +301,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(empty + s, ph ^ 1u, abort_flag, p.ws.status)) { ok = false; break; }
         uint8_t* sa = smem + s * stage_bytes;
-        if (lane == 0) mbar_arrive_expect_tx(full + s, 2 * kABytes + nb * kBRowBox * 128);
+        if (lane == 0)
+          mbar_arrive_expect_tx(full + s, (ui.gate_only ? 1 : 2) * kABytes + nb * kBRowBox * 128);
         __syncwarp();
         if (lane == 0) {
           tma_load_2d(sa, mg, full + s, kb * kKBlock, ui.wrow);
-          tma_load_2d(sa + kABytes, mu, full + s, kb * kKBlock, ui.wrow);
+          if (!ui.gate_only) tma_load_2d(sa + kABytes, mu, full + s, kb * kKBlock, ui.wrow);
         }
         if (lane < nb)
           tma_load_2d(sa + 2 * kABytes + lane * kBRowBox * 128, mx, full + s, kb * kKBlock,
@@ -342,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t acc = (kb != kb0) || (kk != 0);
             // +32 bytes along K per 16-element step (descriptor units of 16 B)
             mma_bf16(d_gate, ag + 2 * kk, bd + 2 * kk, idesc, acc);
-            mma_bf16(d_up, au + 2 * kk, bd + 2 * kk, idesc, acc);
+            if (!ui.gate_only) mma_bf16(d_up, au + 2 * kk, bd + 2 * kk, idesc, acc);
           }
           mma_commit(empty + s);
         }
@@ -397,8 +408,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 0; c0 < N; c0 += 16) {
           uint32_t gr[16], ur[16];
           tmem_ld16(tg + c0, gr);
-          tmem_ld16(tu + c0, ur);
-          tmem_ld_wait(gr, ur);
+          if (ui.gate_only) {
+            tmem_ld_wait(gr);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ur[i] = 0u;
+          } else {
+            tmem_ld16(tu + c0, ur);
+            tmem_ld_wait(gr, ur);
+          }
           float gv[16], uv[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -417,7 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (whole) epi_finish(p, ui, g, word, uni, nact, lane);
+        if (whole) {
+          epi_finish(p, ui, g, word, uni, nact, lane);
+          if (q == 0 && lane == 0)  // weight rows this unit loaded
+            atomicAdd(p.ws.counters + kCntGateUpRows, (ui.gate_only ? 1ull : 2ull) * kNeuronTile);
+        }
       }
       if (last_part) park_u = u;
       tc_fence_before();
@@ -473,6 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane);
         }
         epi_finish(p, ui, g, word, uni, nact, lane);
+        if (q == 0 && lane == 0)
+          atomicAdd(p.ws.counters + kCntGateUpRows, (ui.gate_only ? 1ull : 2ull) * kNeuronTile);
       }
     }
   }

@@ -55,7 +55,7 @@ enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUse
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
                kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
-               kCntWords = 8 };
+               kCntUpRows = 8, kCntGateUpRows = 9, kCntWords = 10 };
 
 enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3 };
 
@@ -84,6 +84,7 @@ struct Dims {
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device
   int sk_ctas;        // capacity of the gate/up split-unit flags (CTAs), 0: no split units
+  int score_gate;     // 1: active iff |SiLU(g)| > tau, sparse up projection for GEMV groups
 };
 
 struct Workspace {
@@ -154,6 +155,8 @@ cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, b
                            cudaStream_t st);
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);
 size_t gate_up_tc_smem_bytes(int n_max, int stages);
+cudaError_t launch_up_gemv(const Dims& dm, const Workspace& ws, const void* Wu, const void* Wus,
+                           const void* x, bool bf16, int n_sms, cudaStream_t st);
 cudaError_t launch_gate_up_simt(const Dims& dm, const Workspace& ws, const float* x,
                                 const float* Wg, const float* Wu, const float* Wgs,
                                 const float* Wus, float tau, float tau_shared, int dense,

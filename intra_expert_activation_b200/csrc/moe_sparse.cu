@@ -41,9 +41,9 @@ bool split_enabled() {
 
 namespace {
 
-constexpr int kStages = 7;
-const char* kStageNames[kStages] = {"route",      "permute", "gate_up", "union_scan",
-                                    "down_gemv", "down_tc", "combine"};
+constexpr int kStages = 8;
+const char* kStageNames[kStages] = {"route",   "permute",   "gate_up", "union_scan",
+                                    "up_gemv", "down_gemv", "down_tc", "combine"};
 
 thread_local std::string g_init_error;
 
@@ -127,6 +127,7 @@ moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
     }
   }
   if (d->path < MOE_PATH_AUTO || d->path > MOE_PATH_SPARSE_TC_ALLROWS) { err = "unknown path"; return MOE_ERR_INVALID; }
+  if (d->score != MOE_SCORE_H && d->score != MOE_SCORE_GATE) { err = "unknown score"; return MOE_ERR_INVALID; }
   if (!bf16 && (d->path == MOE_PATH_SPARSE_TC || d->path == MOE_PATH_SPARSE_TC_ALLROWS)) {
     err = "tensor-core down paths need bf16";
     return MOE_ERR_UNSUPPORTED;
@@ -168,6 +169,7 @@ Layout make_layout(const moe_sparse_desc* d) {
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
   c.gather_density = d->gather_max_density;
   c.no_tc = bf16 ? 0 : 1;
+  c.score_gate = d->score == MOE_SCORE_GATE ? 1 : 0;
 
   const size_t es = bf16 ? 2 : 4;
   size_t sz[bCount];
@@ -547,12 +549,18 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
                          std::min(T, moe::kGroupMax) <= cap.gemv_max);
-  if (need_gemv) {
-    e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, st);
-    if (e != cudaSuccess) return cuda_fail(c, e, "down_gemv launch");
+  if (need_gemv && dm.score_gate) {  // h of the GEMV groups' active rows
+    e = moe::launch_up_gemv(dm, c->ws, W_up, c->Wus, x, c->bf16, c->n_sms, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "up_gemv launch");
     stage_ran[4] = true;
   }
   mark(5);
+  if (need_gemv) {
+    e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "down_gemv launch");
+    stage_ran[5] = true;
+  }
+  mark(6);
   if (need_tc) {
     moe::DownTcParams p;
     p.tm_wd_row = c->tm_wd_row;
@@ -577,13 +585,13 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     const int grid = std::max(1, std::min(units_max, ctas_per_sm * c->n_sms));
     e = moe::launch_down_tc(p, grid, smem, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_tc launch");
-    stage_ran[5] = true;
+    stage_ran[6] = true;
   }
-  mark(6);
+  mark(7);
   e = moe::launch_combine(dm, c->ws, out, c->bf16, st);
   if (e != cudaSuccess) return cuda_fail(c, e, "combine launch");
-  stage_ran[6] = true;
-  mark(7);
+  stage_ran[7] = true;
+  mark(8);
   int nl = 0;
   for (int i = 0; i < kStages; ++i) nl += stage_ran[i];
   c->launches += nl;
@@ -634,6 +642,8 @@ moe_status moe_sparse_get_stats(moe_sparse_ctx* c, moe_stats* s, void* stream) {
   s->n_groups_tc_gather = (int64_t)cnt[moe::kCntTcGather];
   s->n_groups_tc_allrows = (int64_t)(cnt[moe::kCntTc] - cnt[moe::kCntTcGather]);
   s->n_experts_touched = meta[moe::kMetaExpertsTouched];
+  s->up_rows_read = (int64_t)cnt[moe::kCntUpRows];
+  s->gate_up_rows_read = (int64_t)cnt[moe::kCntGateUpRows];
   return MOE_OK;
 }
 

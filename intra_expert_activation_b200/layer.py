@@ -34,7 +34,7 @@ class MoESparseLayer:
                  max_tokens: int, renormalize: bool = True, n_shared: int = 0,
                  d_ff_shared: int = 0, dtype: str = "bf16", path: str = "auto",
                  debug: bool = False, device: int = 0, gemv_max_tokens: int = 0,
-                 gather_max_density: float = 0.0):
+                 gather_max_density: float = 0.0, score: str = "h"):
         self.lib = _lib.load()
         self.torch_dtype, code = _DT[dtype]
         self.dtype = dtype
@@ -44,7 +44,8 @@ class MoESparseLayer:
         self.desc = _lib.moe_sparse_desc(
             d_model, d_ff, n_experts, top_k_max, max_tokens, int(renormalize), n_shared,
             d_ff_shared, code, _lib.PATHS[path], int(debug), device, gemv_max_tokens,
-            gather_max_density)
+            gather_max_density, _lib.SCORES[score])
+        self.score = score
         self.ctx = ctypes.c_void_p()
         _lib.check(self.lib.moe_sparse_init(ctypes.byref(self.desc), ctypes.byref(self.ctx)),
                    "moe_sparse_init")

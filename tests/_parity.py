@@ -32,8 +32,8 @@ with open(os.path.join(GOLDEN, "tau_calibration.json")) as _f:
     TAUS = json.load(_f)
 
 
-def tau_of(workload: str, q: float):
-    e = TAUS[workload]["taus"][f"{q:.2f}"]
+def tau_of(workload: str, q: float, score: str = "h"):
+    e = TAUS[workload]["taus_gate" if score == "gate" else "taus"][f"{q:.2f}"]
     return e["tau"], e.get("tau_shared", 0.0)
 
 
@@ -83,13 +83,13 @@ def unpack_bits(words: np.ndarray, F: int) -> np.ndarray:
 
 
 def oracle_forward(dw: DeviceWeights, x: torch.Tensor, tau: float, tau_shared: float = 0.0,
-                   dense: bool = False, top_k: Optional[int] = None):
+                   dense: bool = False, top_k: Optional[int] = None, score: str = "h"):
     w = dw.host
     sh = dw.shape
     return om.layer_forward(x, w.W_router, w.W_gate, w.W_up, w.W_down, tau, top_k or sh.top_k,
                             sh.renormalize, router_bias=w.router_bias, Ws_gate=w.Ws_gate,
                             Ws_up=w.Ws_up, Ws_down=w.Ws_down, tau_shared=tau_shared,
-                            dense=dense)
+                            dense=dense, score=score)
 
 
 def _band_corrected(ref, dw, gpu_act, gpu_act_shared, tau, tau_shared, ok_tok):
@@ -119,8 +119,9 @@ def _band_corrected(ref, dw, gpu_act, gpu_act_shared, tau, tau_shared, ok_tok):
 
 
 def compare(gpu: dict, ref, tau: float, tau_shared: float, dtype: str, dw=None,
-            check_active=True, dense=False) -> dict:
-    """Assert the parity criteria; return the measured errors."""
+            check_active=True, dense=False, score: str = "h") -> dict:
+    """Assert the parity criteria; return the measured errors. The band is
+    taken on the score the mask used: |h|, or |SiLU(g)| for the gate score."""
     r = ref.router
     T, k = r.topk_idx.shape
     Lmax = np.abs(r.logits).max(axis=1)
@@ -140,7 +141,8 @@ def compare(gpu: dict, ref, tau: float, tau_shared: float, dtype: str, dw=None,
         if dense:
             assert ga[ok_tok].all(), "dense path must keep every neuron"
         else:
-            band = np.abs(np.abs(ref.h[ok_tok]) - tau) <= BAND_REL * tau
+            sc = ref.gate_abs if score == "gate" else np.abs(ref.h)
+            band = np.abs(sc[ok_tok] - tau) <= BAND_REL * tau
             bad = diff & ~band
             assert not bad.any(), f"{int(bad.sum())} active-set mismatches outside the band"
         info["active_mismatch_in_band"] = int(diff.sum())
@@ -151,7 +153,8 @@ def compare(gpu: dict, ref, tau: float, tau_shared: float, dtype: str, dw=None,
             if dense:
                 assert gs.all(), "dense path must keep every shared neuron"
             else:
-                bs = np.abs(np.abs(ref.h_shared) - tau_shared) <= BAND_REL * tau_shared
+                scs = ref.gate_abs_shared if score == "gate" else np.abs(ref.h_shared)
+                bs = np.abs(scs - tau_shared) <= BAND_REL * tau_shared
                 assert not (ds & ~bs).any(), "shared active-set mismatch outside the band"
             info["shared_mismatch_in_band"] = int(ds.sum())
 

@@ -52,8 +52,8 @@ def test_only_the_abi_is_exported():
 
 
 def test_struct_sizes_match_header():
-    assert ctypes.sizeof(_lib.moe_sparse_desc) == 14 * 4
-    assert ctypes.sizeof(_lib.moe_stats) == 10 * 8
+    assert ctypes.sizeof(_lib.moe_sparse_desc) == 15 * 4
+    assert ctypes.sizeof(_lib.moe_stats) == 12 * 8
 
 
 def test_valid_desc_accepted(lib):
@@ -62,6 +62,8 @@ def test_valid_desc_accepted(lib):
     assert lib.moe_sparse_validate_desc(ctypes.byref(f32)) == _lib.MOE_OK
     shared = good_desc(n_shared=2, d_ff_shared=256)
     assert lib.moe_sparse_validate_desc(ctypes.byref(shared)) == _lib.MOE_OK
+    gate = good_desc(score=_lib.MOE_SCORE_GATE)
+    assert lib.moe_sparse_validate_desc(ctypes.byref(gate)) == _lib.MOE_OK
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -74,6 +76,7 @@ def test_valid_desc_accepted(lib):
     (dict(max_tokens=70000), _lib.MOE_ERR_UNSUPPORTED),
     (dict(dtype=7), _lib.MOE_ERR_INVALID),
     (dict(path=9), _lib.MOE_ERR_INVALID),
+    (dict(score=2), _lib.MOE_ERR_INVALID),
     (dict(n_shared=1, d_ff_shared=0), _lib.MOE_ERR_UNSUPPORTED),
     (dict(n_shared=9, d_ff_shared=128), _lib.MOE_ERR_INVALID),
     (dict(dtype=_lib.MOE_F32, d_model=256, d_ff=512, path=3), _lib.MOE_ERR_UNSUPPORTED),

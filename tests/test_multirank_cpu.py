@@ -43,7 +43,7 @@ def _rank_main(rank: int, world: int, port: int, out_dir: str):
     res["value"] = bench.replica_value(105, 20, w, res["max"])
     # the oracle arm: rank 0 alone runs it and prints one line
     args = bench.argparse.Namespace(workload="tiny_f32", sparsity=0.7, steps=1, warmup=0,
-                                    tokens="", gpus=w)
+                                    tokens="", gpus=w, score="h")
     buf = io.StringIO()
     with redirect_stdout(buf):
         rc = bench.run_reference(args, w, r)
