@@ -409,15 +409,18 @@ def run_ours(args, world, rank, local):
                 g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
         d_bytes = st["down_rows_read"] * sh.d_model * esize
         u_bytes = st["up_rows_read"] * sh.d_model * esize
-        u_ms = avg_stage(per_fwd, i, "up_gemv")
+        u_ms = avg_stage(per_fwd, i, "updown_gemv")  # gate score: fused sparse up + down
         up_bytes_tot += u_bytes * args.steps
         up_ms_tot += u_ms * args.steps
         g_ms = avg_stage(per_fwd, i, "gate_up")
-        d_ms = avg_stage(per_fwd, i, "down_gemv") + avg_stage(per_fwd, i, "down_tc")
+        d_ms = avg_stage(per_fwd, i, "down_gemv") + avg_stage(per_fwd, i, "down_tc") \
+            + avg_stage(per_fwd, i, "updown_gemv")
         fwd_ms = sum(avg_stage(per_fwd, i, s) for s in per_fwd[0]) if per_fwd else 0.0
         fwd_dense = sum(avg_stage(per_dense, i, s) for s in per_dense[0]) if per_dense else None
         d_dense = (avg_stage(per_dense, i, "down_gemv") + avg_stage(per_dense, i, "down_tc")) \
             if per_dense else None
+        if args.score == "gate":  # the fused kernel streams W_up and W_down rows
+            d_bytes += u_bytes
         gate_bytes_tot += g_bytes * args.steps
         gate_ms_tot += g_ms * args.steps
         down_bytes_tot += d_bytes * args.steps
@@ -442,7 +445,8 @@ def run_ours(args, world, rank, local):
             "speedup_vs_dense": None if not fwd_dense else round(fwd_dense / fwd_ms, 3),
             "gate_up_GBps": round(g_bytes / (g_ms * 1e-3) / 1e9, 1) if g_ms else None,
             "down_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1) if d_ms else None,
-            "up_GBps": round(u_bytes / (u_ms * 1e-3) / 1e9, 1) if u_ms else None,
+            # the fused kernel reads each active row of W_up and of W_down once
+            "updown_GBps": round(2 * u_bytes / (u_ms * 1e-3) / 1e9, 1) if u_ms else None,
             "dense_down_us": None if d_dense is None else round(1e3 * d_dense, 2),
         })
 
@@ -506,13 +510,14 @@ def run_ours(args, world, rank, local):
                          "traffic": g_traffic,
                          "algorithmic_bytes": round(gate_bytes_tot / n_gate_launches),
                          "peak_kind": peak_kind},
-            "roofline_down": {"kernel": "down (GEMV / TC, rows actually read)", "bound": "hbm",
+            "roofline_down": {"kernel": "down (GEMV / TC / fused up+down, rows actually read)",
+                              "bound": "hbm",
                               "achieved": round(d_ach, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(d_ach / peak, 4), "peak_kind": peak_kind},
-            "roofline_up": None if args.score != "gate" else
-            {"kernel": "up_gemv (gate score: W_up rows actually read)", "bound": "hbm",
-             "achieved": round(u_ach, 1), "peak": peak, "unit": "GB/s",
-             "frac": round(u_ach / peak, 4), "peak_kind": peak_kind},
+            "roofline_updown": None if args.score != "gate" else
+            {"kernel": "updown_gemv (gate score: W_up + W_down rows actually read)",
+             "bound": "hbm", "achieved": round(2 * u_ach, 1), "peak": peak, "unit": "GB/s",
+             "frac": round(2 * u_ach / peak, 4), "peak_kind": peak_kind},
             "dense": dense_line,
             "speedup_vs_dense": None if not dense_line else
             round(dense_line["ms_per_step"] / (ms_sparse / args.steps), 4),

@@ -29,7 +29,8 @@ SCORES = {"h": MOE_SCORE_H, "gate": MOE_SCORE_GATE}
 
 PATHS = {"auto": 0, "dense": 1, "sparse_gemv": 2, "sparse_tc": 3, "sparse_tc_allrows": 4}
 
-STAGES = ("route", "permute", "gate_up", "union_scan", "up_gemv", "down_gemv", "down_tc", "combine")
+STAGES = ("route", "permute", "gate_up", "union_scan", "updown_gemv", "down_gemv", "down_tc",
+          "combine")
 
 
 class moe_sparse_desc(ctypes.Structure):

@@ -32,123 +32,13 @@
 // (zeroed by the router) with vector fp32 atomics: the partials of a unit are
 // summed in arrival order, so results agree to fp32 rounding, not bitwise,
 // between runs on this path.
-#include "gemv_common.cuh"
+#include "gemv_consumers.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kHBytes = 32;          // h bytes per row: 4 x bf16 or 8 x fp32
-constexpr int kYStride = 260;        // floats per staged result row of a consumer warp
-constexpr int kYBytes = kGemvTokens * kYStride * 4;  // a consumer warp's result staging
 constexpr int kStageExtra = kBatch * kHBytes + 16;   // per stage after the rows: h | meta
-
-template <typename TW>
-struct Rows;
-
-// bf16: tensor-core multiply of the landed rows.
-template <>
-struct Rows<__nv_bfloat16> {
-  static constexpr int MT = kGemvTokens;  // tokens per pass
-  static constexpr int kTiles = 16;       // 16-column tiles of the warp's 256 columns
-  float acc[kTiles][4];
-
-  __device__ void zero() {
-#pragma unroll
-    for (int i = 0; i < kTiles; ++i)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[i][v] = 0.f;
-  }
-  // D[16 columns][8 tokens] += W^T[16 columns][8 rows] * H[8 rows][8 tokens];
-  // tokens >= mt and rows >= cnt enter as zero h.
-  __device__ void consume(uint32_t rows_s, const uint8_t*, int stride, const uint8_t* hs, int cnt,
-                          int mt, int lane) {
-    const int g = lane >> 2, c2 = 2 * (lane & 3);
-    uint32_t hb2 = 0u;  // H[rows c2, c2 + 1][token g]
-    if (g < mt) {
-      const uint32_t lo = c2 < cnt ? reinterpret_cast<const uint16_t*>(hs + c2 * kHBytes)[g] : 0u;
-      const uint32_t hi =
-          c2 + 1 < cnt ? reinterpret_cast<const uint16_t*>(hs + (c2 + 1) * kHBytes)[g] : 0u;
-      hb2 = lo | (hi << 16);
-    }
-    const uint32_t row_s = rows_s + (lane & 7) * stride + (lane >> 3) * 16;
-#pragma unroll
-    for (int p = 0; p < kTiles / 2; ++p) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(row_s + p * 64, a0, a1, a2, a3);
-      mma_16x8x8(acc[2 * p], a0, a1, hb2);
-      mma_16x8x8(acc[2 * p + 1], a2, a3, hb2);
-    }
-  }
-  // acc[i] = D[column 16i + g (+8)][tokens c2, c2 + 1]; lanes g and g ^ 1
-  // swap halves so that each holds two adjacent columns of one token.
-  // acc[i] = D[column 16i + g (+8)][tokens c2, c2 + 1] goes through the
-  // warp's staging rows ys[token][kYStride] (row stride 260 floats: the four
-  // token rows a store touches fall in different banks), then leaves as
-  // 16-byte vector adds.
-  __device__ void flush(float* y, int d, int mt, float* ys, int lane) {
-    const int g = lane >> 2, c2 = 2 * (lane & 3);
-#pragma unroll
-    for (int i = 0; i < kTiles; ++i) {
-      if (c2 < mt) {
-        ys[c2 * kYStride + 16 * i + g] = acc[i][0];
-        ys[c2 * kYStride + 16 * i + g + 8] = acc[i][2];
-      }
-      if (c2 + 1 < mt) {
-        ys[(c2 + 1) * kYStride + 16 * i + g] = acc[i][1];
-        ys[(c2 + 1) * kYStride + 16 * i + g + 8] = acc[i][3];
-      }
-    }
-    __syncwarp();
-    for (int t = 0; t < mt; ++t) {
-#pragma unroll
-      for (int h = 0; h < kTiles / 8; ++h) {
-        const int col = 128 * h + 4 * lane;
-        const float4 v = *reinterpret_cast<const float4*>(ys + t * kYStride + col);
-        red_add_v4(y + (size_t)t * d + col, v.x, v.y, v.z, v.w);
-      }
-    }
-    __syncwarp();
-  }
-};
-
-// fp32: packed fp32x2 FMAs, 4 columns per lane, up to 8 tokens.
-template <>
-struct Rows<float> {
-  static constexpr int MT = 8;
-  uint64_t acc[MT][2];
-
-  __device__ void zero() {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = 0ull;
-  }
-  __device__ void consume(uint32_t, const uint8_t* rows, int stride, const uint8_t* hs, int cnt,
-                          int mt, int lane) {
-    for (int r = 0; r < cnt; ++r) {
-      const float* hr = reinterpret_cast<const float*>(hs + r * kHBytes);
-      const uint4 u = *reinterpret_cast<const uint4*>(rows + r * stride + lane * 16);
-      const uint64_t w0 = pack2(__uint_as_float(u.x), __uint_as_float(u.y));
-      const uint64_t w1 = pack2(__uint_as_float(u.z), __uint_as_float(u.w));
-#pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        if (t < mt) {
-          const uint64_t h2 = pack2(hr[t], hr[t]);
-          fma2(acc[t][0], h2, w0);
-          fma2(acc[t][1], h2, w1);
-        }
-      }
-    }
-  }
-  __device__ void flush(float* y, int d, int mt, float*, int lane) {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      if (t < mt) {
-        const float2 a = unpack2(acc[t][0]), b = unpack2(acc[t][1]);
-        red_add_v4(y + (size_t)t * d + lane * 4, a.x, a.y, b.x, b.y);
-      }
-    }
-  }
-};
 
 template <typename TW>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -155,8 +155,9 @@ cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, b
                            cudaStream_t st);
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);
 size_t gate_up_tc_smem_bytes(int n_max, int stages);
-cudaError_t launch_up_gemv(const Dims& dm, const Workspace& ws, const void* Wu, const void* Wus,
-                           const void* x, bool bf16, int n_sms, cudaStream_t st);
+cudaError_t launch_updown_gemv(const Dims& dm, const Workspace& ws, const void* Wu,
+                               const void* Wus, const void* Wd, const void* Wds, const void* x,
+                               bool bf16, int n_sms, cudaStream_t st);
 cudaError_t launch_gate_up_simt(const Dims& dm, const Workspace& ws, const float* x,
                                 const float* Wg, const float* Wu, const float* Wgs,
                                 const float* Wus, float tau, float tau_shared, int dense,

@@ -42,8 +42,8 @@ bool split_enabled() {
 namespace {
 
 constexpr int kStages = 8;
-const char* kStageNames[kStages] = {"route",   "permute",   "gate_up", "union_scan",
-                                    "up_gemv", "down_gemv", "down_tc", "combine"};
+const char* kStageNames[kStages] = {"route",       "permute",   "gate_up", "union_scan",
+                                    "updown_gemv", "down_gemv", "down_tc", "combine"};
 
 thread_local std::string g_init_error;
 
@@ -549,13 +549,14 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
                          std::min(T, moe::kGroupMax) <= cap.gemv_max);
-  if (need_gemv && dm.score_gate) {  // h of the GEMV groups' active rows
-    e = moe::launch_up_gemv(dm, c->ws, W_up, c->Wus, x, c->bf16, c->n_sms, st);
-    if (e != cudaSuccess) return cuda_fail(c, e, "up_gemv launch");
+  if (need_gemv && dm.score_gate) {  // GEMV groups: fused sparse up + down over the active rows
+    e = moe::launch_updown_gemv(dm, c->ws, W_up, c->Wus, W_down, c->Wds, x, c->bf16, c->n_sms,
+                                st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "updown_gemv launch");
     stage_ran[4] = true;
   }
   mark(5);
-  if (need_gemv) {
+  if (need_gemv && !dm.score_gate) {
     e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_gemv launch");
     stage_ran[5] = true;
