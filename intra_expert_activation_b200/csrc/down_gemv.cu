@@ -158,7 +158,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ consumers
     R rows;
-    float* ystage = reinterpret_cast<float*>(smem + NS * geo.stage) + warp * (kYBytes / 4);
     rows.zero();
     int cur_tag = -1, cur_slot = 0, cur_mt = 0, cur_col0 = 0;
     for (int s = 0;; ++s) {
@@ -176,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mine = phase < n_phase && (s % n_phase) == phase;
       if (meta.x != cur_tag && (mine || meta.x < 0)) {
         if (cur_tag >= 0) {
-          rows.flush(ws.y + (size_t)cur_slot * d + cur_col0, d, cur_mt, ystage, lane);
+          rows.flush(ws.y + (size_t)cur_slot * d + cur_col0, d, cur_mt, lane);
           rows.zero();
         }
         cur_tag = meta.x;
@@ -198,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t down_gemv_smem_bytes(int d, bool bf16) {
   const Geometry g = geometry(d * (bf16 ? 2 : 4), kStageExtra);
-  return static_cast<size_t>(g.n_stages) * g.stage + (bf16 ? kConsumers * kYBytes : 0);
+  return static_cast<size_t>(g.n_stages) * g.stage;
 }
 
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
@@ -207,11 +206,11 @@ cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(down_gemv_kernel<__nv_bfloat16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBudget + kConsumers * kYBytes);
+                                         kSmemBudget);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(down_gemv_kernel<float>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSmemBudget + kConsumers * kYBytes);
+                               kSmemBudget);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }

@@ -21,10 +21,13 @@ constexpr int kSliceBytes = 512;     // row bytes per consumer warp
 constexpr int kBlockBytes = kConsumers * kSliceBytes;  // column block: 4 KB of a row
 constexpr int kRowPad = 16;          // row stride = block bytes + 16
 constexpr int kMaxStages = 6;
-constexpr int kSmemBudget = 190 * 1024;  // stages; the result staging comes on top
+constexpr int kSmemBudget = 200 * 1024;  // ring of stages (6 stages of 4 KB blocks)
 constexpr int kListRows = 256;       // producer's row list (uint16 neuron indices)
 constexpr int kTight = 4096;         // barrier probes before sleeping: stages arrive every few us
 
+__device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
                "f"(d)

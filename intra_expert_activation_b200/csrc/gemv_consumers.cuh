@@ -12,8 +12,6 @@ namespace {
 constexpr int kTok = 8;         // token columns of the mma (passes hold up to 8)
 constexpr int kTokStride = kTok;  // floats per row of an fp32 h array [row][token]
 constexpr int kHBytes = 32;          // h bytes per row: 4 x bf16 or 8 x fp32
-constexpr int kYStride = 260;        // floats per staged result row of a consumer warp
-constexpr int kYBytes = kGemvTokens * kYStride * 4;  // a consumer warp's result staging
 
 template <typename TW>
 struct Rows;
@@ -69,35 +67,28 @@ struct Rows<__nv_bfloat16> {
       mma_16x8x8(acc[2 * p + 1], a2, a3, hb2);
     }
   }
-  // acc[i] = D[column 16i + g (+8)][tokens c2, c2 + 1]; lanes g and g ^ 1
-  // swap halves so that each holds two adjacent columns of one token.
-  // acc[i] = D[column 16i + g (+8)][tokens c2, c2 + 1] goes through the
-  // warp's staging rows ys[token][kYStride] (row stride 260 floats: the four
-  // token rows a store touches fall in different banks), then leaves as
-  // 16-byte vector adds.
-  __device__ void flush(float* y, int d, int mt, float* ys, int lane) {
+  // acc[i] = D[column 16i + g (+8)][tokens c2, c2 + 1]: lanes g and g ^ 1
+  // swap halves so that each holds two adjacent columns of one token, added
+  // into Y with 8-byte vector atomics (no shared-memory staging, so the ring
+  // of stages gets that space).
+  __device__ void flush(float* y, int d, int mt, int lane) {
     const int g = lane >> 2, c2 = 2 * (lane & 3);
+    const bool odd = g & 1;
+    const int tok = c2 + odd;
+    float* yt = y + (size_t)tok * d + (g & ~1);
 #pragma unroll
     for (int i = 0; i < kTiles; ++i) {
-      if (c2 < mt) {
-        ys[c2 * kYStride + 16 * i + g] = acc[i][0];
-        ys[c2 * kYStride + 16 * i + g + 8] = acc[i][2];
-      }
-      if (c2 + 1 < mt) {
-        ys[(c2 + 1) * kYStride + 16 * i + g] = acc[i][1];
-        ys[(c2 + 1) * kYStride + 16 * i + g + 8] = acc[i][3];
-      }
-    }
-    __syncwarp();
-    for (int t = 0; t < mt; ++t) {
-#pragma unroll
-      for (int h = 0; h < kTiles / 8; ++h) {
-        const int col = 128 * h + 4 * lane;
-        const float4 v = *reinterpret_cast<const float4*>(ys + t * kYStride + col);
-        red_add_v4(y + (size_t)t * d + col, v.x, v.y, v.z, v.w);
+      const float s0 = odd ? acc[i][0] : acc[i][1];
+      const float s1 = odd ? acc[i][2] : acc[i][3];
+      const float r0 = __shfl_xor_sync(0xffffffffu, s0, 4);
+      const float r1 = __shfl_xor_sync(0xffffffffu, s1, 4);
+      if (tok < mt) {
+        const float2 a = odd ? make_float2(r0, acc[i][1]) : make_float2(acc[i][0], r0);
+        const float2 b = odd ? make_float2(r1, acc[i][3]) : make_float2(acc[i][2], r1);
+        red_add_v2(yt + 16 * i, a.x, a.y);
+        red_add_v2(yt + 16 * i + 8, b.x, b.y);
       }
     }
-    __syncwarp();
   }
 };
 
@@ -145,7 +136,7 @@ struct Rows<float> {
       }
     }
   }
-  __device__ void flush(float* y, int d, int mt, float*, int lane) {
+  __device__ void flush(float* y, int d, int mt, int lane) {
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       if (t < mt) {

@@ -151,7 +151,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     U up;
     R down;
     down.zero();
-    float* ystage = reinterpret_cast<float*>(smem + NS * geo.stage) + warp * (kYBytes / 4);
     const size_t ld = static_cast<size_t>(dm.slots_total);
     const TW* ht = static_cast<const TW*>(ws.ht);
     int up_tag = -2;  // unit and block whose x values the warp holds
@@ -196,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (dn_tag >= 0 && (tag < 0 || (is_down && active && tag != dn_tag))) {
-        down.flush(ws.y + (size_t)dn_slot * d + dn_col0, d, dn_mt, ystage, lane);
+        down.flush(ws.y + (size_t)dn_slot * d + dn_col0, d, dn_mt, lane);
         down.zero();
         dn_tag = -1;
       }
@@ -245,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t updown_gemv_smem_bytes(int d, bool bf16) {
   const Geometry g = geometry(d * (bf16 ? 2 : 4), kMetaBytes);
-  return static_cast<size_t>(g.n_stages) * g.stage + (bf16 ? kConsumers * kYBytes : 0);
+  return static_cast<size_t>(g.n_stages) * g.stage;
 }
 
 cudaError_t launch_updown_gemv(const Dims& dm, const Workspace& ws, const void* Wu,
