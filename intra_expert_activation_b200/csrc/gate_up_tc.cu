@@ -229,7 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = p.stages;
   const int n_max = p.n_max;
-  const uint32_t stage_bytes = 2 * kABytes + n_max * 128;
+  // stage: two 16 KB weight boxes, then b_blocks activation regions of n_max
+  // rows (with the gate score a gate-only unit puts two K-blocks of W_gate and
+  // of x in one stage, so that a stage still carries two weight boxes)
+  const uint32_t b_half = n_max * 128;
+  const uint32_t stage_bytes = 2 * kABytes + p.b_blocks * b_half;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
   uint64_t* empty = full + stages;
   uint64_t* tfull = empty + stages;  // [2]
@@ -296,21 +300,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* mg = ui.shared ? &p.tm_wgs : &p.tm_wg;
       const CUtensorMap* mu = ui.shared ? &p.tm_wus : &p.tm_wu;
       const CUtensorMap* mx = ui.shared ? &p.tm_x : &p.tm_xperm;
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      const int kstep = ui.gate_only && p.b_blocks == 2 ? 2 : 1;  // K-blocks per stage
+      for (int kb = kb0; kb < kb1; kb += kstep, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(empty + s, ph ^ 1u, abort_flag, p.ws.status)) { ok = false; break; }
         uint8_t* sa = smem + s * stage_bytes;
+        const int nk = min(kstep, kb1 - kb);
+        const uint32_t xbytes = nb * kBRowBox * 128;
         if (lane == 0)
-          mbar_arrive_expect_tx(full + s, (ui.gate_only ? 1 : 2) * kABytes + nb * kBRowBox * 128);
+          mbar_arrive_expect_tx(full + s, ui.gate_only ? nk * (kABytes + xbytes)
+                                                       : 2 * kABytes + xbytes);
         __syncwarp();
-        if (lane == 0) {
-          tma_load_2d(sa, mg, full + s, kb * kKBlock, ui.wrow);
-          if (!ui.gate_only) tma_load_2d(sa + kABytes, mu, full + s, kb * kKBlock, ui.wrow);
+        if (ui.gate_only) {  // W_gate and x of K-blocks kb (, kb + 1)
+          for (int j = 0; j < nk; ++j) {
+            if (lane == 0) tma_load_2d(sa + j * kABytes, mg, full + s, (kb + j) * kKBlock, ui.wrow);
+            if (lane < nb)
+              tma_load_2d(sa + 2 * kABytes + j * b_half + lane * kBRowBox * 128, mx, full + s,
+                          (kb + j) * kKBlock, ui.gr.xrow0 + lane * (int)kBRowBox);
+          }
+        } else {
+          if (lane == 0) {
+            tma_load_2d(sa, mg, full + s, kb * kKBlock, ui.wrow);
+            tma_load_2d(sa + kABytes, mu, full + s, kb * kKBlock, ui.wrow);
+          }
+          if (lane < nb)
+            tma_load_2d(sa + 2 * kABytes + lane * kBRowBox * 128, mx, full + s, kb * kKBlock,
+                        ui.gr.xrow0 + lane * (int)kBRowBox);
         }
-        if (lane < nb)
-          tma_load_2d(sa + 2 * kABytes + lane * kBRowBox * 128, mx, full + s, kb * kKBlock,
-                      ui.gr.xrow0 + lane * (int)kBRowBox);
         __syncwarp();
       }
     }
@@ -338,22 +355,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t d_gate = tmem_base + b * buf_cols;
       const uint32_t d_up = d_gate + n_max;
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      const int kstep = ui.gate_only && p.b_blocks == 2 ? 2 : 1;  // K-blocks per stage
+      for (int kb = kb0; kb < kb1; kb += kstep, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(full + s, ph, abort_flag, p.ws.status)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint64_t ag = smem_desc_sw128(sa, 16, 1024);
-          const uint64_t au = smem_desc_sw128(sa + kABytes, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sa + 2 * kABytes, 16, 1024);
+          if (ui.gate_only) {
+            const int nk = min(kstep, kb1 - kb);
+            for (int j = 0; j < nk; ++j) {
+              const uint64_t ag = smem_desc_sw128(sa + j * kABytes, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(sa + 2 * kABytes + j * b_half, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kKBlock / 16; ++kk) {
-            const uint32_t acc = (kb != kb0) || (kk != 0);
-            // +32 bytes along K per 16-element step (descriptor units of 16 B)
-            mma_bf16(d_gate, ag + 2 * kk, bd + 2 * kk, idesc, acc);
-            if (!ui.gate_only) mma_bf16(d_up, au + 2 * kk, bd + 2 * kk, idesc, acc);
+              for (int kk = 0; kk < kKBlock / 16; ++kk)
+                mma_bf16(d_gate, ag + 2 * kk, bd + 2 * kk, idesc, (kb + j != kb0) || (kk != 0));
+            }
+          } else {
+            const uint64_t ag = smem_desc_sw128(sa, 16, 1024);
+            const uint64_t au = smem_desc_sw128(sa + kABytes, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sa + 2 * kABytes, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kKBlock / 16; ++kk) {
+              const uint32_t acc = (kb != kb0) || (kk != 0);
+              // +32 bytes along K per 16-element step (descriptor units of 16 B)
+              mma_bf16(d_gate, ag + 2 * kk, bd + 2 * kk, idesc, acc);
+              mma_bf16(d_up, au + 2 * kk, bd + 2 * kk, idesc, acc);
+            }
           }
           mma_commit(empty + s);
         }
@@ -510,8 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t gate_up_tc_smem_bytes(int n_max, int stages) {
-  const size_t stage_bytes = 2 * kABytes + static_cast<size_t>(n_max) * 128;
+size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks) {
+  const size_t stage_bytes = 2 * kABytes + static_cast<size_t>(b_blocks) * n_max * 128;
   return 1024 + stages * stage_bytes + (2 * stages + 5) * sizeof(uint64_t) + 16;
 }
 

@@ -132,6 +132,7 @@ struct GateUpTcParams {
   int nbuf;                    // TMEM accumulator buffers (1 or 2)
   uint32_t tmem_cols;          // allocated TMEM columns
   int split;                   // 1: the leftover units after whole rounds are cut along K
+  int b_blocks;                // activation regions per stage: 2 with the gate score, else 1
 };
 
 // ------------------------------------------------------------ down (tcgen05)
@@ -154,7 +155,7 @@ bool route_is_small(const Dims& dm);
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st);
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);
-size_t gate_up_tc_smem_bytes(int n_max, int stages);
+size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks);
 cudaError_t launch_updown_gemv(const Dims& dm, const Workspace& ws, const void* Wu,
                                const void* Wus, const void* Wd, const void* Wds, const void* x,
                                bool bf16, int n_sms, cudaStream_t st);

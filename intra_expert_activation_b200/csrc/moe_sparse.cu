@@ -516,9 +516,13 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     p.tmem_cols = pow2_at_least(p.nbuf * buf);
     const int ctas_per_sm = n_max <= 32 ? 2 : 1;
     const size_t budget = ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
-    const size_t stage_bytes = 32768 + (size_t)n_max * 128;
+    // gate score: gate-only units take two K-blocks per stage; the second
+    // activation region costs a stage of the pipeline when groups are larger
+    // than 16 tokens (measured at T = 32: 303 -> 358 us), so only below that
+    p.b_blocks = dm.score_gate && n_max <= 16 ? 2 : 1;
+    const size_t stage_bytes = 32768 + (size_t)p.b_blocks * n_max * 128;
     p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
-    const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages);
+    const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages, p.b_blocks);
     const int units_max = (P / moe::kGroupMax + std::min(cap.E, P)) * (cap.F / moe::kNeuronTile) +
                           cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) *
                               (cap.Fs / moe::kNeuronTile);
