@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # launch of the same kernel (decode batch T=8, 7 experts touched): traffic grows with the
 # touched experts, so a launch's traffic is this ratio times its algorithmic bytes
 # (profiles/gate_up_tc.mixtral_decode_T8.md). None once the kernel has changed since.
-GATE_UP_TRAFFIC_RATIO = 1.0047
+GATE_UP_TRAFFIC_RATIO = 1.0106
 
 
 def parse():
