@@ -90,36 +90,39 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 }
 
 template <typename TX>
-__global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX* out) {
+__global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX* out, int nb) {
   grid_dep_wait();
-  const int t = blockIdx.x;
+  // CTA = (token, block of blockDim x 4 columns): every column of a token is
+  // in flight at once, and each thread's k + S row loads are issued together
+  const int t = blockIdx.x / nb;
+  const int c = ((blockIdx.x % nb) * blockDim.x + threadIdx.x) * 4;
   const int d = dm.d, k = dm.k;
   __shared__ int slot[16];
   __shared__ float w[16];
   if (threadIdx.x < k) {
-    slot[threadIdx.x] = ws.slot_of[t * k + threadIdx.x];
-    w[threadIdx.x] = ws.topk_w[t * k + threadIdx.x];
+    slot[threadIdx.x] = __ldcg(ws.slot_of + t * k + threadIdx.x);
+    w[threadIdx.x] = __ldcg(ws.topk_w + t * k + threadIdx.x);
   }
   __syncthreads();
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < k; ++i) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + static_cast<size_t>(slot[i]) * d + c));
-      acc.x = fmaf(w[i], v.x, acc.x);
-      acc.y = fmaf(w[i], v.y, acc.y);
-      acc.z = fmaf(w[i], v.z, acc.z);
-      acc.w = fmaf(w[i], v.w, acc.w);
-    }
-    for (int s = 0; s < dm.S; ++s) {
-      const size_t srow = static_cast<size_t>(dm.slots_routed + s * dm.T_pad + t);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + srow * d + c));
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    store4<TX>(out + static_cast<size_t>(t) * d + c, acc);
+  if (c >= d) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int i = 0; i < k; ++i) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + static_cast<size_t>(slot[i]) * d + c));
+    acc.x = fmaf(w[i], v.x, acc.x);
+    acc.y = fmaf(w[i], v.y, acc.y);
+    acc.z = fmaf(w[i], v.z, acc.z);
+    acc.w = fmaf(w[i], v.w, acc.w);
   }
+  for (int s = 0; s < dm.S; ++s) {
+    const size_t srow = static_cast<size_t>(dm.slots_routed + s * dm.T_pad + t);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(ws.y + srow * d + c));
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  store4<TX>(out + static_cast<size_t>(t) * d + c, acc);
 }
 
 __global__ void debug_gather_kernel(Dims dm, Workspace ws, int32_t* topk_idx, float* topk_w,
@@ -159,10 +162,13 @@ cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t 
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
                            cudaStream_t st) {
   const int threads = dm.d / 4 >= 256 ? 256 : ((dm.d / 4 + 31) / 32) * 32;
+  const int nb = (dm.d / 4 + threads - 1) / threads;  // column blocks per token
+  const int grid = dm.T * nb;
   if (bf16)
-    return launch_k(combine_kernel<__nv_bfloat16>, dm.T, threads, 0, st, dm, ws,
-                    static_cast<__nv_bfloat16*>(out));
-  return launch_k(combine_kernel<float>, dm.T, threads, 0, st, dm, ws, static_cast<float*>(out));
+    return launch_k(combine_kernel<__nv_bfloat16>, grid, threads, 0, st, dm, ws,
+                    static_cast<__nv_bfloat16*>(out), nb);
+  return launch_k(combine_kernel<float>, grid, threads, 0, st, dm, ws, static_cast<float*>(out),
+                  nb);
 }
 
 cudaError_t launch_debug_gather(const Dims& dm, const Workspace& ws, int32_t* topk_idx,

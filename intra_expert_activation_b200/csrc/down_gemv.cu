@@ -83,14 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t ld = static_cast<size_t>(dm.slots_total);
     const char* ht = static_cast<const char*>(ws.ht);
     Walk k;
-    k.i = start.i;
-    k.p = start.p;
-    k.w = start.w;
-    k.m = start.m;
-    k.left = start.rows;
-    k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
-    k.serial = 0;
-    walk_load_group(dm, ws, k, MT);
+    walk_begin(dm, ws, start, k, MT);
     int s = 0;  // stages filled
     bool ok = true;
     for (bool last = false; ok && !last;) {
@@ -135,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t hdst = stg_s + kBatch * geo.stride + lane * kHBytes;
               const char* hsrc = ht + ((size_t)j * ld + slot) * ES;
               if constexpr (ES == 2) {
-                cp_async8(hdst, hsrc);
+                cp_async16(hdst, hsrc);  // 8 bf16 h values (slots of a pass are 16-B aligned)
               } else {
                 cp_async16(hdst, hsrc);
                 cp_async16(hdst + 16, hsrc + 16);

@@ -39,6 +39,8 @@ struct DownUnit {
   int cnt;        // union rows (gathered)
   int row_base;   // first row of this expert in the 2-D [experts*F][d] view
   int shared;
+  int cand;       // candidate group, decided from its union
+  int skip;       // candidate taken by the GEMV kernel: no work, no Y writes here
 };
 
 __device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_slices) {
@@ -50,9 +52,12 @@ __device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_s
   const int F_e = du.shared ? p.dm.Fs : p.dm.F;
   const int e_local = du.shared ? du.gr.expert - p.dm.E : du.gr.expert;
   du.row_base = e_local * F_e;
-  du.gather = __ldcg(p.ws.group_path + du.g) == kPathTcGather;
+  const int path = __ldcg(p.ws.group_path + du.g);
+  du.gather = path == kPathTcGather;
   du.cnt = __ldcg(p.ws.union_cnt + du.g);
-  du.nk = du.gather ? (du.cnt + kKBlock - 1) / kKBlock : F_e / kKBlock;
+  du.cand = path == kPathCand;
+  du.skip = du.cand && cand_takes_gemv(du.cnt, (du.gr.m + kGemvTokens - 1) / kGemvTokens, F_e);
+  du.nk = du.skip ? 0 : du.gather ? (du.cnt + kKBlock - 1) / kKBlock : F_e / kKBlock;
   return du;
 }
 
@@ -90,14 +95,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMEM is taken only once the previous kernel has completed, so a CTA of
   // this kernel never holds TMEM while waiting on another kernel
   grid_dep_wait();
+  const int n_slices = p.dm.d / kDownSlice;
+  const int n_units = __ldcg(p.ws.meta + kMetaTcCount) * n_slices;
+  if (static_cast<int>(blockIdx.x) >= n_units) return;  // no unit for this CTA: leave before TMEM
   if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  const int n_slices = p.dm.d / kDownSlice;
-  const int n_units = __ldcg(p.ws.meta + kMetaTcCount) * n_slices;
   const uint32_t buf_cols = p.n_max;
   const int ht_oob = p.dm.F_max;  // H^T row past the end: zero fill
 
@@ -113,6 +118,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const DownUnit du = decode(p, u, n_slices);
+      if (du.cand && !du.skip && du.slice == 0 && lane == 0) {  // a candidate taken here
+        atomicAdd(p.ws.counters + kCntDownRows,
+                  static_cast<unsigned long long>(du.shared ? p.dm.Fs : p.dm.F));
+        atomicAdd(p.ws.counters + kCntTc, 1ull);
+      }
       const int N = (du.gr.m + 15) & ~15;
       const int x0 = du.slice * kDownSlice;
       const int* rows = p.ws.union_rows + static_cast<size_t>(du.g) * p.dm.F_max;
@@ -217,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m = du.gr.m;
       const int col = du.slice * kDownSlice + 32 * q + lane;
       float* yc = p.ws.y + static_cast<size_t>(du.gr.slot0) * d + col;
+      if (du.skip) continue;  // the GEMV kernel has added this group's rows into Y
       if (du.nk == 0) {
         for (int c = 0; c < m; ++c) yc[static_cast<size_t>(c) * d] = 0.f;
         continue;

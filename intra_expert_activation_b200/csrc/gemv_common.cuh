@@ -66,9 +66,6 @@ __device__ __forceinline__ void mma_16x8x8(float (&d)[4], uint32_t a0, uint32_t 
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -127,7 +124,8 @@ struct Start {
   int w;        // bitmap word of the first row
   uint32_t m;   // mask of the rows of word w that are still to come
   int rows;     // rows of this CTA
-  int g, row;   // the first group and the row within its pass (prologue scratch)
+  int g, row;   // the first group and the row within its pass
+  Group gr;     // the first group's record
 };
 
 // The producer's walk over its CTA's rows: group list index, pass, next word
@@ -140,6 +138,31 @@ struct Walk {
   int g, words, passes, slot0, m_tok, expert, xrow0;  // unit data of group i
   int serial;  // increments whenever the unit (group, pass) changes
 };
+
+// Unit data of group g (record gr).
+__device__ __forceinline__ void walk_set_group(const Dims& dm, Walk& k, int g, const Group& gr,
+                                               int MT) {
+  k.g = g;
+  k.expert = gr.expert;
+  k.slot0 = gr.slot0;
+  k.m_tok = gr.m;
+  k.xrow0 = gr.xrow0;
+  k.passes = (gr.m + MT - 1) / MT;
+  k.words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
+}
+
+// The producer's walk from the CTA's start (no global loads).
+__device__ __forceinline__ void walk_begin(const Dims& dm, const Workspace& ws, const Start& st,
+                                           Walk& k, int MT) {
+  k.i = st.i;
+  k.p = st.p;
+  k.w = st.w;
+  k.m = st.m;
+  k.left = st.rows;
+  k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
+  k.serial = 0;
+  walk_set_group(dm, k, st.g, st.gr, MT);
+}
 
 // Loads group i's unit data; false past the end of the GEMV list.
 __device__ __forceinline__ bool walk_load_group(const Dims& dm, const Workspace& ws, Walk& k,
@@ -154,6 +177,15 @@ __device__ __forceinline__ bool walk_load_group(const Dims& dm, const Workspace&
   k.passes = (gr.m + MT - 1) / MT;
   k.words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
   return true;
+}
+
+// Rows per pass of group k.g on this kernel: its union count, or 0 for a
+// candidate group that the tensor-core path takes.
+__device__ __forceinline__ int walk_unit_rows(const Workspace& ws, const Walk& k) {
+  const int cnt = __ldcg(ws.union_cnt + k.g);
+  if (__ldcg(ws.group_path + k.g) == kPathCand && !cand_takes_gemv(cnt, k.passes, 32 * k.words))
+    return 0;
+  return cnt;
 }
 
 // Next run of rows of one unit into the list: the set bits of up to 32
@@ -173,7 +205,7 @@ __device__ int walk_next(const Dims& dm, const Workspace& ws, Walk& k, uint16_t*
         do {
           ++k.i;
           ok = walk_load_group(dm, ws, k, MT);
-        } while (ok && __ldcg(ws.union_cnt + k.g) == 0);
+        } while (ok && walk_unit_rows(ws, k) == 0);
         if (!ok) {  // the union counts and the bitmaps disagree
           if (lane == 0) report_error(ws.status, kErrDeviceInvalid);
           k.left = 0;
@@ -242,12 +274,21 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
       const int i = base + tid;
       long long v = 0;
       int g = 0, cnt = 0, words = 0;
+      Group gr{};
       if (i < n_gv) {
         g = base == 0 ? g_spec : __ldcg(ws.gemv_list + i);
         cnt = __ldcg(ws.union_cnt + g);
-        const Group gr = ws.groups[g];
-        v = (long long)((gr.m + MT - 1) / MT) * cnt;
+        const int path = __ldcg(ws.group_path + g);
+        gr = ws.groups[g];
+        const int passes = (gr.m + MT - 1) / MT;
         words = (gr.expert >= dm.E ? dm.Fs : dm.F) / 32;
+        if (path == kPathCand) {  // decided now, from its union (the TC kernel agrees)
+          const bool take = cand_takes_gemv(cnt, passes, 32 * words);
+          if (!take) cnt = 0;
+          if (take && sweep == 1 && blockIdx.x == 0)
+            atomicAdd(ws.counters + kCntGemv, 1ull);
+        }
+        v = (long long)passes * cnt;
       }
       long long incl = v;
 #pragma unroll
@@ -274,8 +315,9 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
           st->i = i;
           st->p = (int)(off / cnt);
           st->g = g;
+          st->gr = gr;
           st->row = (int)(off % cnt);
-          st->w = words;  // the group's word count, until warp 0 positions the cursor
+          st->w = words;  // the group's word count, until the cursor is placed
         }
       }
       carry += chunk;
@@ -288,32 +330,40 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* s
   }
   __syncthreads();
   if (st->rows <= 0 || st->i < 0) return;  // uniform
-  // warp 0: the bitmap word holding row st->row of group st->g
-  if (warp == 0) {
-    const int g = st->g, words = st->w;
-    int skip = st->row;
-    for (int w0 = 0; w0 < words; w0 += 32) {
-      const uint32_t bits =
-          w0 + lane < words ? __ldcg(ws.union_bits + (size_t)g * dm.fw + w0 + lane) : 0u;
-      const int c = __popc(bits);
-      int incl = c;
+  // the bitmap word holding row st->row of group st->g: every thread loads
+  // one word of a window of blockDim words (all loads in flight together),
+  // a CTA-wide prefix sum of their row counts finds the word
+  const int g = st->g, words = st->w;
+  int skip = st->row;
+  int* cnt_w = reinterpret_cast<int*>(sm_warp);
+  for (int w0 = 0; w0 < words; w0 += blockDim.x) {
+    const int word = w0 + tid;
+    const uint32_t bits = word < words ? __ldcg(ws.union_bits + (size_t)g * dm.fw + word) : 0u;
+    const int c = __popc(bits);
+    int incl = c;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      const int excl = incl - c;
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-      __syncwarp();  // every lane has read st->w before the owner lane rewrites it
-      if (excl <= skip && skip < incl) {  // this lane's word holds the first row
-        uint32_t m = bits;
-        for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
-        st->w = w0 + lane;
-        st->m = m;
-      }
-      if (skip < total) break;
-      skip -= total;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
     }
+    if (lane == 31) cnt_w[warp] = incl;
+    __syncthreads();  // also: every thread has read st->w before its owner rewrites it
+    int before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int x = cnt_w[w];
+      if (w < warp) before += x;
+      total += x;
+    }
+    const int excl = before + incl - c;
+    if (excl <= skip && skip < excl + c) {  // this thread's word holds the first row
+      uint32_t m = bits;
+      for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
+      st->w = word;
+      st->m = m;
+    }
+    __syncthreads();  // cnt_w is rewritten by the next window
+    if (skip < total) break;  // uniform
+    skip -= total;
   }
   __syncthreads();
 }

@@ -11,7 +11,7 @@ namespace {
 
 constexpr int kTok = 8;         // token columns of the mma (passes hold up to 8)
 constexpr int kTokStride = kTok;  // floats per row of an fp32 h array [row][token]
-constexpr int kHBytes = 32;          // h bytes per row: 4 x bf16 or 8 x fp32
+constexpr int kHBytes = 32;          // h bytes per row slot: 8 x bf16 (16 B used) or 8 x fp32
 
 template <typename TW>
 struct Rows;

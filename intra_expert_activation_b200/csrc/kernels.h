@@ -46,7 +46,15 @@ constexpr int kDownSlice = 128;     // d_model columns per down TC tile (M)
 constexpr int kKBlock = 64;         // K elements per pipeline stage (128 B of bf16)
 constexpr int kRouteTokens = 16;    // tokens per router CTA
 constexpr int kListMax = 2048;      // expert token groups per forward at most
-constexpr int kGemvTokens = 4;      // tokens per GEMV unit (bf16); fp32 uses 8
+constexpr int kGemvTokens = 8;      // tokens per GEMV pass (the row-stream mma's N)
+// AUTO with the |h| score: groups of gemv_max < m <= kGemvCandMax tokens
+// (one GEMV pass) choose their down path after gate/up from the size of
+// their active-row union: the row stream if passes x union rows <=
+// kCandNum / kCandDen x d_ff, else all rows on the tensor cores. The ratio is
+// the measured bandwidth of the row stream over that of the all-rows
+// tensor-core path on the Mixtral-shaped layer.
+constexpr int kGemvCandMax = 8;
+constexpr int kCandNum = 9, kCandDen = 10;
 
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
@@ -57,7 +65,8 @@ enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCn
                kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
                kCntUpRows = 8, kCntGateUpRows = 9, kCntWords = 10 };
 
-enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3 };
+// kPathCand: GEMV or all-rows TC, chosen after gate/up (cand_takes_gemv)
+enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3, kPathCand = 4 };
 
 // Requested path (mirrors moe_path in the public header).
 enum Mode { kModeAuto = 0, kModeDense = 1, kModeGemv = 2, kModeTc = 3, kModeTcAll = 4 };
@@ -80,6 +89,7 @@ struct Dims {
   int groups_max;
   int mode;           // Mode
   int gemv_max;       // AUTO: GEMV for groups with m <= gemv_max
+  int gemv_cand;      // AUTO: groups with gemv_max < m <= gemv_cand are candidates
   float gather_density;
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device

@@ -167,6 +167,11 @@ Layout make_layout(const moe_sparse_desc* d) {
                  c.S * ((c.T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
   c.mode = d->path;
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
+  // automatic threshold: groups of 5..kGemvCandMax tokens choose after gate/up
+  c.gemv_cand = d->gemv_max_tokens == 0 && bf16 && d->path == MOE_PATH_AUTO &&
+                        d->score != MOE_SCORE_GATE
+                    ? moe::kGemvCandMax
+                    : c.gemv_max;
   c.gather_density = d->gather_max_density;
   c.no_tc = bf16 ? 0 : 1;
   c.score_gate = d->score == MOE_SCORE_GATE ? 1 : 0;

@@ -83,7 +83,8 @@ __device__ __forceinline__ int group_path_of(const Dims& dm, int m) {
   if (dm.no_tc || dm.mode == kModeGemv) return kPathGemv;
   if (dm.mode == kModeTc) return kPathTcAll;  // gathered or not: decided by the union scan
   if (dm.mode == kModeTcAll) return kPathTcAll;
-  return m <= dm.gemv_max ? kPathGemv : kPathTcAll;  // auto and dense
+  if (m <= dm.gemv_max) return kPathGemv;  // auto and dense
+  return m <= dm.gemv_cand ? kPathCand : kPathTcAll;
 }
 
 // Last CTA: histograms -> base offsets, expert slot ranges, token groups and
@@ -192,6 +193,11 @@ __device__ __forceinline__ void block_exclusive_scan(int (&v)[N], int (&total)[N
 
 // How one entry's tokens are cut into groups. An entry is a routed expert
 // (q < E, its me = cnt[q] pairs) or a shared expert (q >= E, all T tokens):
+__device__ __forceinline__ int on_gemv_list(int path) {
+  return path == kPathGemv || path == kPathCand;
+}
+__device__ __forceinline__ int on_tc_list(int path) { return path != kPathGemv; }
+
 // ng groups of gsz tokens (a multiple of kSlotAlign; the last one has
 // m_last), each at most kGroupMax.
 struct EntryCut {
@@ -236,7 +242,9 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
   if (tid == 0) zero_shared = 0;
 
   // ---- pass 1: slots, groups, GEMV / TC list positions
-  enum { kSlots, kGroups, kGemv, kTc, kRoutedGroups, kTcShared, kTouched, kN };
+  // kGemv / kTc: list lengths (a candidate group is in both lists); kCand:
+  // candidates; kTcSharedDef: shared groups whose all-rows TC path is fixed now
+  enum { kSlots, kGroups, kGemv, kTc, kCand, kRoutedGroups, kTcSharedDef, kTouched, kN };
   int v[kN] = {}, tot[kN];
   EntryCut cut[kPer];
 #pragma unroll
@@ -246,17 +254,20 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     const EntryCut c = entry_cut(dm, cnt, q);
     cut[i] = c;
     if (c.ng == 0) continue;
-    const int n_gemv = (c.ng - 1) * (c.path_full == kPathGemv) + (c.path_last == kPathGemv);
+    const int n_gemv = (c.ng - 1) * on_gemv_list(c.path_full) + on_gemv_list(c.path_last);
+    const int n_tc = (c.ng - 1) * on_tc_list(c.path_full) + on_tc_list(c.path_last);
+    const int n_cand = (c.ng - 1) * (c.path_full == kPathCand) + (c.path_last == kPathCand);
     if (q < E) {
       v[kSlots] += (c.me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
       v[kRoutedGroups] += c.ng;
       v[kTouched] += 1;
     } else {
-      v[kTcShared] += c.ng - n_gemv;
+      v[kTcSharedDef] += n_tc - n_cand;
     }
     v[kGroups] += c.ng;
     v[kGemv] += n_gemv;
-    v[kTc] += c.ng - n_gemv;
+    v[kTc] += n_tc;
+    v[kCand] += n_cand;
   }
   block_exclusive_scan<kN>(v, tot, scan_sm);
 
@@ -283,12 +294,11 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
           ws.groups[g] = gr;
           ws.group_path[g] = path;
           ws.union_cnt[g] = 0;
-          if (path == kPathGemv) {
+          if (on_gemv_list(path)) {
             any_gemv = 1;
             ws.gemv_list[gv++] = g;
-          } else {
-            ws.tc_list[tc++] = g;
           }
+          if (on_tc_list(path)) ws.tc_list[tc++] = g;
         }
       }
       if (routed) {
@@ -309,12 +319,13 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     ws.meta[kMetaExpertsTouched] = tot[kTouched];
     ws.meta[kMetaGemvCount] = tot[kGemv];
     ws.meta[kMetaTcCount] = tot[kTc];
-    ws.counters[kCntGemv] = tot[kGemv];
-    ws.counters[kCntTc] = tot[kTc];
+    // candidates are counted by the down kernel that takes them
+    ws.counters[kCntGemv] = tot[kGemv] - tot[kCand];
+    ws.counters[kCntTc] = tot[kTc] - tot[kCand];
     if (dm.mode != kModeTc)  // the GEMV kernel adds its rows
       ws.counters[kCntDownRows] =
-          (unsigned long long)(tot[kTc] - tot[kTcShared]) * dm.F +
-          (unsigned long long)tot[kTcShared] * dm.Fs;
+          (unsigned long long)(tot[kTc] - tot[kCand] - tot[kTcSharedDef]) * dm.F +
+          (unsigned long long)tot[kTcSharedDef] * dm.Fs;
     ws.counters[kCntRoutedH] = (unsigned long long)T * k * (unsigned long long)dm.F;
     ws.counters[kCntSharedH] =
         (unsigned long long)S * (unsigned long long)T * (unsigned long long)dm.Fs;

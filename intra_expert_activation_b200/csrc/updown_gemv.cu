@@ -82,14 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
     Walk k;
-    k.i = start.i;
-    k.p = start.p;
-    k.w = start.w;
-    k.m = start.m;
-    k.left = start.rows;
-    k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
-    k.serial = 0;
-    walk_load_group(dm, ws, k, MT);
+    walk_begin(dm, ws, start, k, MT);
     int s = 0;
     bool ok = true;
     for (bool last_run = false; ok && !last_run;) {

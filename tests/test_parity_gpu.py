@@ -11,7 +11,7 @@ import torch
 from moe_inputs import LayerShape, make_tokens, make_weights
 from oracle import moe_oracle as om
 from _parity import (DeviceWeights, compare, make_layer, oracle_forward, run_gpu, tau_of,
-                     workload_tokens, workload_weights)
+                     unpack_bits, workload_tokens, workload_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -267,3 +267,46 @@ def test_mixtral_sweep(sweep, T, q):
     tau, _ = tau_of("mixtral_sweep", q)
     layer = make_layer(wl.shape, 512)
     _check(layer, dw, workload_tokens(wl, T), tau, 0.0, "bf16")
+
+
+def _expected_down_rows(gpu, F):
+    """Rows the automatic per-group switch reads, from the GPU's own active
+    sets: groups of <= 4 tokens stream their union; groups of 5..8 tokens
+    stream it iff 10 x union <= 9 x d_ff (one pass of 8 tokens), else all
+    d_ff rows on the tensor cores, as do larger groups."""
+    act = unpack_bits(gpu["active_bits"], F)
+    idx = gpu["topk_idx"].ravel()
+    rows = n_gemv = n_tc = cand_gemv = cand_tc = 0
+    for e in np.unique(idx):
+        m = int((idx == e).sum())
+        u = int(act[idx == e].any(axis=0).sum())
+        if m <= 4 or (m <= 8 and 10 * u <= 9 * F):
+            rows += u
+            n_gemv += 1
+            cand_gemv += m > 4
+        else:
+            rows += F
+            n_tc += 1
+            cand_tc += m <= 8
+    return rows, n_gemv, n_tc, cand_gemv, cand_tc
+
+
+def test_candidate_groups_choose_by_union(sweep):
+    """Groups of 5..8 tokens pick the row stream or all rows on the tensor
+    cores after gate/up from their union size: both choices occur (high
+    sparsity: row stream; tau = 0: tensor cores), the rows read and the group
+    counts follow the rule, and the output matches the oracle."""
+    wl, dw = sweep
+    F = wl.shape.d_ff
+    seen_gemv = seen_tc = 0
+    for q in (0.0, 0.9):
+        tau, _ = tau_of("mixtral_sweep", q)
+        layer = make_layer(wl.shape, 512)
+        gpu, _, _ = _check(layer, dw, workload_tokens(wl, 24), tau, 0.0, "bf16")
+        rows, n_gemv, n_tc, cand_gemv, cand_tc = _expected_down_rows(gpu, F)
+        st = gpu["stats"]
+        assert st["down_rows_read"] == rows
+        assert st["n_groups_gemv"] == n_gemv and st["n_groups_tc_allrows"] == n_tc
+        seen_gemv += cand_gemv
+        seen_tc += cand_tc
+    assert seen_gemv > 0 and seen_tc > 0
