@@ -156,8 +156,14 @@ MOE_API moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx**
 
 /* Always-on shared experts (desc.n_shared > 0): W*_s are device pointers
  * [n_shared][d_ff_shared][d_model] in desc.dtype, kept by pointer (the caller
- * keeps them alive); tau_shared is their own threshold. Must be called
- * before the first forward of a context with shared experts. */
+ * keeps them alive); tau_shared is their own threshold. A negative tau_shared
+ * keeps every shared neuron active, so the shared experts run dense while the
+ * routed experts stay sparse (the configuration of the paper's system, which
+ * leaves shared-expert execution unchanged [gist.science EN "Uncovering
+ * Intra-expert Activation Sparsity for Efficient Mixture-of-Expert Model
+ * Execution", Technical Summary > Methodology > System Implementation in
+ * vLLM]). Must be called before the first forward of a context with shared
+ * experts. */
 MOE_API moe_status moe_sparse_set_shared(moe_sparse_ctx* ctx, const void* Wg_s, const void* Wu_s,
                                  const void* Wd_s, float tau_shared);
 

@@ -27,6 +27,20 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 192;
+
+// The four epilogue warps (warps 2..5) only: named barrier 1, plain and as
+// an AND vote (every thread gets the same answer).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool epi_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
 constexpr uint32_t kAAtom = 64 * 128;  // one 64-row x 128-byte swizzled atom column
 constexpr uint32_t kABytes = 2 * kAAtom;
 
@@ -34,6 +48,9 @@ struct DownUnit {
   Group gr;
   int g;
   int slice;
+  int k0;         // first K-block of this unit's part
+  int part;       // K part of the unit (0 .. ks-1)
+  int ub;         // (list index, slice) of the unit: its ticket
   int gather;     // 1: gathered rows, 0: all rows
   int nk;         // K-blocks
   int cnt;        // union rows (gathered)
@@ -43,10 +60,19 @@ struct DownUnit {
   int skip;       // candidate taken by the GEMV kernel: no work, no Y writes here
 };
 
-__device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_slices) {
+// Unit u = ((list index, part), slice): the slices of one part of a group
+// are consecutive units, so the CTAs that run at the same time read whole
+// W_down rows between them (as without parts), not narrow strips of
+// different rows.
+__device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_slices, int ks) {
   DownUnit du;
-  du.g = __ldcg(p.ws.tc_list + u / n_slices);
   du.slice = u % n_slices;
+  u /= n_slices;
+  const int part = u % ks;
+  const int li = u / ks;
+  du.part = part;
+  du.ub = li * n_slices + du.slice;
+  du.g = __ldcg(p.ws.tc_list + li);
   du.gr = p.ws.groups[du.g];
   du.shared = du.gr.expert >= p.dm.E;
   const int F_e = du.shared ? p.dm.Fs : p.dm.F;
@@ -57,7 +83,9 @@ __device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_s
   du.cnt = __ldcg(p.ws.union_cnt + du.g);
   du.cand = path == kPathCand;
   du.skip = du.cand && cand_takes_gemv(du.cnt, (du.gr.m + kGemvTokens - 1) / kGemvTokens, F_e);
-  du.nk = du.skip ? 0 : du.gather ? (du.cnt + kKBlock - 1) / kKBlock : F_e / kKBlock;
+  const int nk = du.skip ? 0 : du.gather ? (du.cnt + kKBlock - 1) / kKBlock : F_e / kKBlock;
+  du.k0 = nk * part / ks;
+  du.nk = nk * (part + 1) / ks - du.k0;
   return du;
 }
 
@@ -75,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_part = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -96,7 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // this kernel never holds TMEM while waiting on another kernel
   grid_dep_wait();
   const int n_slices = p.dm.d / kDownSlice;
-  const int n_units = __ldcg(p.ws.meta + kMetaTcCount) * n_slices;
+  const int n_tc = __ldcg(p.ws.meta + kMetaTcCount);
+  const int ks = tc_ksplit(p.dm, n_tc);  // > 1: parts add into Y (zeroed by the router's layout)
+  const int n_units = n_tc * n_slices * ks;
   if (static_cast<int>(blockIdx.x) >= n_units) return;  // no unit for this CTA: leave before TMEM
   if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);
   tc_fence_before();
@@ -117,8 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const DownUnit du = decode(p, u, n_slices);
-      if (du.cand && !du.skip && du.slice == 0 && lane == 0) {  // a candidate taken here
+      const DownUnit du = decode(p, u, n_slices, ks);
+      if (du.cand && !du.skip && du.slice == 0 && du.k0 == 0 && lane == 0) {  // a candidate taken here
         atomicAdd(p.ws.counters + kCntDownRows,
                   static_cast<unsigned long long>(du.shared ? p.dm.Fs : p.dm.F));
         atomicAdd(p.ws.counters + kCntTc, 1ull);
@@ -129,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* wrow = du.shared ? &p.tm_wds_row : &p.tm_wd_row;
       const CUtensorMap* wblk = du.shared ? &p.tm_wds_blk : &p.tm_wd_blk;
       const int w_oob = du.shared ? p.dm.S * p.dm.Fs : p.dm.E * p.dm.F;
-      for (int kc = 0; kc < du.nk; ++kc, ++it) {
+      for (int kc = du.k0; kc < du.k0 + du.nk; ++kc, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
         if (!warp_wait(empty + s, ph ^ 1u, abort_flag, p.ws.status)) { ok = false; break; }
@@ -178,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0, uidx = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const DownUnit du = decode(p, u, n_slices);
+      const DownUnit du = decode(p, u, n_slices, ks);
       if (du.nk == 0) continue;  // empty union: the epilogue writes zeros
       const int N = (du.gr.m + 15) & ~15;
       const uint32_t idesc = idesc_bf16_f32(kDownSlice, N, 1, 1);
@@ -223,33 +254,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = p.dm.d;
     uint32_t uidx = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const DownUnit du = decode(p, u, n_slices);
+      const DownUnit du = decode(p, u, n_slices, ks);
       const int m = du.gr.m;
       const int col = du.slice * kDownSlice + 32 * q + lane;
       float* yc = p.ws.y + static_cast<size_t>(du.gr.slot0) * d + col;
       if (du.skip) continue;  // the GEMV kernel has added this group's rows into Y
-      if (du.nk == 0) {
+      if (du.nk == 0) {  // empty union (gathered mode, never cut into parts)
         for (int c = 0; c < m; ++c) yc[static_cast<size_t>(c) * d] = 0.f;
         continue;
       }
       const int N = (m + 15) & ~15;
       const uint32_t b = uidx % 2;
       const uint32_t tph = (uidx / 2) & 1u;
-      if (!warp_wait(tfull + b, tph, abort_flag, p.ws.status)) break;
+      bool ok = warp_wait(tfull + b, tph, abort_flag, p.ws.status);
+      if (ks > 1) ok = epi_all(ok);  // the part path's barriers below need all four warps
+      if (!ok) break;
       tc_fence_after();
+      // parts: this part's sums go to its block of the part buffer, [token][128 columns]
+      float* pc = p.ws.tc_part +
+                  (static_cast<size_t>(du.ub) * ks + du.part) * kTcPartTokens * kDownSlice + 32 * q +
+                  lane;
       const uint32_t ta = tmem_base + lane_off + b * buf_cols;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(ta + c0, r);
         tmem_ld_wait(r);
+        if (ks == 1) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = __uint_as_float(r[i]);
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = __uint_as_float(r[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < m) pc[(c0 + i) * kDownSlice] = __uint_as_float(r[i]);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + b);
       ++uidx;
+      if (ks > 1) {
+        // the last part of this (group, slice) to finish adds the ks parts
+        // in part order and stores Y
+        const int ub = du.ub;
+        __threadfence();
+        epi_bar();  // the four warps' columns of this part are written
+        if (warp == 2 && lane == 0) *last_part = atomicAdd(p.ws.tc_ticket + ub, 1) == ks - 1;
+        epi_bar();
+        if (*last_part) {
+          __threadfence();
+          const float* pb = p.ws.tc_part + static_cast<size_t>(ub) * ks * kTcPartTokens * kDownSlice +
+                            32 * q + lane;
+          // 8 tokens x all parts per batch: their loads are in flight together
+          // (one L2 round trip per batch, not one per value)
+          constexpr int kC = 8;
+          for (int c0 = 0; c0 < m; c0 += kC) {
+            float v[kC][kTcMaxParts];
+#pragma unroll
+            for (int i = 0; i < kC; ++i)
+#pragma unroll
+              for (int pp = 0; pp < kTcMaxParts; ++pp)
+                v[i][pp] = c0 + i < m && pp < ks
+                               ? __ldcg(pb + (static_cast<size_t>(pp) * kTcPartTokens + c0 + i) *
+                                                 kDownSlice)
+                               : 0.f;
+#pragma unroll
+            for (int i = 0; i < kC; ++i) {
+              float acc = 0.f;
+#pragma unroll
+              for (int pp = 0; pp < kTcMaxParts; ++pp) acc += v[i][pp];  // part order
+              if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = acc;
+            }
+          }
+        }
+      }
     }
   }
 

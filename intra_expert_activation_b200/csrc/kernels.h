@@ -95,7 +95,38 @@ struct Dims {
   int n_sms;          // streaming multiprocessors of the device
   int sk_ctas;        // capacity of the gate/up split-unit flags (CTAs), 0: no split units
   int score_gate;     // 1: active iff |SiLU(g)| > tau, sparse up projection for GEMV groups
+  int tc_grid;        // CTAs of this forward's tensor-core down launch
+  int tc_part_units;  // capacity of the tensor-core down part buffers (units), 0: none
 };
+
+// K parts per tensor-core down unit (group, 128-column slice). A unit reads
+// all of its group's rows for its columns, and one CTA streams at most about
+// 35 GB/s (one 117 MB group of the Mixtral-shaped layer = 32 units took
+// 108 us), while HBM shared by the whole grid gives each CTA about 22 GB/s.
+// So the path is HBM-bound only with at least ~0.6 of the grid busy; with
+// fewer units each unit's rows are cut into ks parts: the smallest ks giving
+// that many units, at most kTcMaxParts and at most the K-blocks of the
+// smallest expert. Parts write fp32 partial sums to the workspace and the
+// last part of a unit to finish (a ticket) adds them in part order into Y,
+// so results do not depend on timing. Only groups of <= kTcPartTokens tokens
+// are cut (decode batches; larger batches have units enough), and at most
+// dm.tc_part_units part units exist. The router (to clear the tickets) and
+// the kernel evaluate it on the same inputs.
+constexpr int kTcMaxParts = 8;
+constexpr int kTcPartTokens = 64;
+__host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
+  if (dm.mode == kModeTc || n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
+  const int tmax = dm.T < kGroupMax ? dm.T : kGroupMax;
+  if ((tmax + 15) / 16 * 16 > kTcPartTokens) return 1;
+  const int f_min = dm.S > 0 && dm.Fs < dm.F ? dm.Fs : dm.F;
+  const int cap = f_min / kKBlock < kTcMaxParts ? f_min / kKBlock : kTcMaxParts;
+  const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);
+  const long long want = (3LL * dm.tc_grid + 4) / 5;
+  long long ks = (want + base - 1) / base;
+  if (ks > cap) ks = cap;
+  while (ks > 1 && base * ks > dm.tc_part_units) --ks;
+  return ks < 1 ? 1 : static_cast<int>(ks);
+}
 
 struct Workspace {
   int* status;                  // [1] device error word
@@ -120,6 +151,8 @@ struct Workspace {
   int* y_zero;                  // [E+1] 1: expert's Y rows (last: shared experts') start at zero
   int* sk_flags;                // [sk_ctas] gate/up: CTA c published its split-unit partial
   float* sk_part;               // [2 * sk_ctas][2][128][n_max] gate/up split-unit partial sums
+  int* tc_ticket;               // [tc_part_units] parts of a TC down unit done (cleared by the router)
+  float* tc_part;               // [tc_part_units][kTcPartTokens][128] TC down part sums
 
   uint32_t* act_bits;           // [slots_total][fw] or null (debug off)
   void* xperm;                  // [slots_routed][d] activations gathered by slot

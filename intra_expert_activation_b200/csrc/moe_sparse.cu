@@ -102,7 +102,7 @@ struct Layout {
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
            bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero, bSkFlags, bSkPart,
-           bActBits, bXperm, bHt, bY, bCount };
+           bTcTicket, bTcPart, bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   if (!d) { err = "desc is NULL"; return MOE_ERR_INVALID; }
@@ -205,6 +205,11 @@ Layout make_layout(const moe_sparse_desc* d) {
     sz[bSkFlags] = sizeof(int) * (size_t)c.sk_ctas;
     sz[bSkPart] = sizeof(float) * (size_t)2 * c.sk_ctas * 2 * moe::kNeuronTile * nm;
   }
+  // tensor-core down units cut along K (bf16, groups of <= 64 tokens): a
+  // ticket per unit and a partial-sum block per part unit
+  c.tc_part_units = bf16 ? 384 : 0;
+  sz[bTcTicket] = sizeof(int) * (size_t)c.tc_part_units;
+  sz[bTcPart] = sizeof(float) * (size_t)c.tc_part_units * moe::kTcPartTokens * moe::kDownSlice;
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;
   sz[bXperm] = es * (size_t)c.slots_routed * c.d;
   sz[bHt] = es * (size_t)c.F_max * c.slots_total;
@@ -386,6 +391,8 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.y_zero = reinterpret_cast<int*>(b + o[bYZero]);
   w.sk_flags = reinterpret_cast<int*>(b + o[bSkFlags]);
   w.sk_part = reinterpret_cast<float*>(b + o[bSkPart]);
+  w.tc_ticket = reinterpret_cast<int*>(b + o[bTcTicket]);
+  w.tc_part = reinterpret_cast<float*>(b + o[bTcPart]);
   w.act_bits = desc->debug ? reinterpret_cast<uint32_t*>(b + o[bActBits]) : nullptr;
   w.xperm = b + o[bXperm];
   w.ht = b + o[bHt];
@@ -469,6 +476,22 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   dm.groups_max = P / moe::kGroupMax + std::min(cap.E, P) +
                   cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
   const bool dense = c->desc.path == MOE_PATH_DENSE;
+  const int mode = c->desc.path;
+  const bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
+  const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
+                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
+                         std::min(T, moe::kGroupMax) <= cap.gemv_max);
+  const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
+  // the tensor-core down launch's grid is fixed here: the router's layout
+  // and the kernel both derive the units' K parts from it
+  const int tc_ctas_per_sm = n_max <= 64 ? 2 : 1;
+  {
+    const long long units_max =
+        (long long)dm.groups_max * (cap.d / moe::kDownSlice) * moe::kTcMaxParts;
+    dm.tc_grid = need_tc ? (int)std::max<long long>(
+                               1, std::min<long long>(units_max, tc_ctas_per_sm * c->n_sms))
+                         : 0;
+  }
 
   if (c->bf16) {
     if (!build_weight_maps(c, W_gate, W_up, W_down)) return MOE_ERR_CUDA;
@@ -501,7 +524,6 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   }
   mark(2);
 
-  const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
   if (c->bf16) {
     moe::GateUpTcParams p;
     p.tm_wg = c->tm_wg;
@@ -553,11 +575,6 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   }
   mark(4);
 
-  const int mode = c->desc.path;
-  const bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
-  const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
-                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
-                         std::min(T, moe::kGroupMax) <= cap.gemv_max);
   if (need_gemv && dm.score_gate) {  // GEMV groups: fused sparse up + down over the active rows
     e = moe::launch_updown_gemv(dm, c->ws, W_up, c->Wus, W_down, c->Wds, x, c->bf16, c->n_sms,
                                 st);
@@ -586,14 +603,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     p.tmem_cols = pow2_at_least(2u * n_max);
     // small groups (decode): two CTAs per SM so that a unit's epilogue and
     // the next unit's loads overlap across CTAs; large groups: one CTA
-    const int ctas_per_sm = n_max <= 64 ? 2 : 1;
-    const size_t budget = ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
+    const size_t budget = tc_ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
     const size_t stage_bytes = 16384 + (size_t)p.b_bytes;
     p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
     const size_t smem = moe::down_tc_smem_bytes(p.b_bytes, p.stages);
-    const int units_max = dm.groups_max * (cap.d / moe::kDownSlice);
-    const int grid = std::max(1, std::min(units_max, ctas_per_sm * c->n_sms));
-    e = moe::launch_down_tc(p, grid, smem, st);
+    e = moe::launch_down_tc(p, dm.tc_grid, smem, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_tc launch");
     stage_ran[6] = true;
   }

@@ -335,6 +335,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
   for (int x = tid; x <= E; x += blockDim.x) ws.expert_off[x] = poff[x];
   for (int x = tid; x < E; x += blockDim.x) ws.expert_cnt[x] = cnt[x];
   for (int x = tid; x < dm.sk_ctas; x += blockDim.x) ws.sk_flags[x] = 0;  // gate/up split units
+  for (int x = tid; x < dm.tc_part_units; x += blockDim.x) ws.tc_ticket[x] = 0;  // TC down parts
 }
 
 // Dot product of one token row with one router row, lanes over d in chunks

@@ -284,6 +284,24 @@ def test_shared_threshold_is_separate():
     assert _rel(r0.out - r1.out, delta) <= 1e-10
 
 
+def test_negative_shared_threshold_runs_shared_experts_dense():
+    # the pages' system keeps shared experts dense and sparsifies only the
+    # routed ones: with tau_shared < 0 every shared neuron is active, and the
+    # output is the sparse routed part plus the textbook shared SwiGLU FFNs
+    rng = np.random.default_rng(41)
+    x, Wr, Wg, Wu, Wd, sh = _rand_layer(rng, 7, 8, 4, 10, S=2, Fs=12)
+    base = om.layer_forward(x, Wr, Wg, Wu, Wd, 0.0, 2, True)
+    tau = float(np.quantile(np.abs(base.h), 0.7))
+    res = om.layer_forward(x, Wr, Wg, Wu, Wd, tau, 2, True, tau_shared=-1.0, **sh)
+    assert res.active_shared.all()
+    routed = om.layer_forward(x, Wr, Wg, Wu, Wd, tau, 2, True)
+    G = np.einsum("td,sfd->stf", x, sh["Ws_gate"])
+    H = G / (1 + np.exp(-G)) * np.einsum("td,sfd->stf", x, sh["Ws_up"])
+    shared = np.einsum("stf,sfd->td", H, sh["Ws_down"])
+    assert np.array_equal(res.active, routed.active)
+    assert _rel(res.out, routed.out + shared) <= 1e-13
+
+
 # ------------------------------------------------------------- invariances
 
 def test_token_permutation():

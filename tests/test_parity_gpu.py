@@ -118,6 +118,19 @@ def test_small_bf16_shared(small_shared, T, path):
     _check(layer, small_shared, x, tau, ts, "bf16", dense=(path == "dense"))
 
 
+@pytest.mark.parametrize("T", [2, 45])
+def test_small_bf16_shared_dense(small_shared, T):
+    """tau_shared < 0: the shared experts run dense (every shared neuron
+    active) while the routed experts stay sparse."""
+    x = make_tokens(SMALL_SHARED.d_model, T, 22, "bf16")
+    tau, _ = _calibrated(small_shared, x, 0.7, 0.5)
+    layer = make_layer(SMALL_SHARED, 512)
+    gpu, ref, _ = _check(layer, small_shared, x, tau, -1.0, "bf16")
+    st = gpu["stats"]
+    assert st["n_shared_active"] == st["n_shared_h"] > 0
+    assert st["n_routed_active"] < st["n_routed_h"]
+
+
 def test_sparse_tau0_equals_dense(small):
     x = make_tokens(SMALL.d_model, 37, 21, "bf16")
     a = run_gpu(make_layer(SMALL, 64, path="auto"), small, x, 0.0)
@@ -167,6 +180,21 @@ def test_deterministic(small):
     a = run_gpu(layer, small, x, 0.2)["out"]
     b = run_gpu(layer, small, x, 0.2)["out"]
     assert np.array_equal(a, b)
+
+
+def test_deterministic_k_parts(small):
+    """Few tensor-core groups (T = 20: four groups of ~10 tokens): each
+    (group, column slice) unit is cut into K parts whose sums are added in
+    part order by the last part to finish, so repeated runs agree bitwise."""
+    x = make_tokens(SMALL.d_model, 20, 21, "bf16")
+    layer = make_layer(SMALL, 64)
+    tau = 0.2
+    a = run_gpu(layer, small, x, tau)
+    b = run_gpu(layer, small, x, tau)
+    assert np.array_equal(a["out"], b["out"])
+    assert a["stats"]["n_groups_tc_allrows"] >= 2
+    compare(a, oracle_forward(small, x, tau), tau, 0.0, "bf16", dw=small)
+    assert layer.status() == 0
 
 
 def test_graph_replay_parity(small):
