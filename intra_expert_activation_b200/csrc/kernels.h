@@ -100,32 +100,40 @@ struct Dims {
 };
 
 // K parts per tensor-core down unit (group, 128-column slice). A unit reads
-// all of its group's rows for its columns, and one CTA streams at most about
-// 35 GB/s (one 117 MB group of the Mixtral-shaped layer = 32 units took
-// 108 us), while HBM shared by the whole grid gives each CTA about 22 GB/s.
-// So the path is HBM-bound only with at least ~0.6 of the grid busy; with
-// fewer units each unit's rows are cut into ks parts: the smallest ks giving
-// that many units, at most kTcMaxParts and at most the K-blocks of the
-// smallest expert. Parts write fp32 partial sums to the workspace and the
-// last part of a unit to finish (a ticket) adds them in part order into Y,
-// so results do not depend on timing. Only groups of <= kTcPartTokens tokens
-// are cut (decode batches; larger batches have units enough), and at most
-// dm.tc_part_units part units exist. The router (to clear the tickets) and
-// the kernel evaluate it on the same inputs.
-constexpr int kTcMaxParts = 8;
+// all of its group's rows for its columns, and an SM streams at most about
+// 35-40 GB/s, so HBM is only saturated when every SM has work: with few
+// groups most SMs idled (one 117 MB group of the Mixtral-shaped layer = 32
+// units took 108 us). When the units fill less than 3/4 of the grid, each
+// unit's rows are cut into ks parts, ks in 1..kTcMaxParts minimising the
+// rounds per unit of work, ceil(units x ks / grid) / ks (the smaller ks on
+// ties), with at most dm.tc_part_units part units and at least one K-block
+// per part. Parts write fp32 partial sums to the workspace and the last part
+// of a unit to finish (a ticket) adds them in part order into Y, so results
+// do not depend on timing. Only groups of <= kTcPartTokens tokens are cut
+// (decode batches). The router (to clear the tickets) and the kernel
+// evaluate it on the same inputs.
+constexpr int kTcMaxParts = 12;
 constexpr int kTcPartTokens = 64;
 __host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
   if (dm.mode == kModeTc || n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
   const int tmax = dm.T < kGroupMax ? dm.T : kGroupMax;
   if ((tmax + 15) / 16 * 16 > kTcPartTokens) return 1;
+  const long long grid = dm.tc_grid;
+  const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);
+  if (4 * base >= 3 * grid) return 1;
   const int f_min = dm.S > 0 && dm.Fs < dm.F ? dm.Fs : dm.F;
   const int cap = f_min / kKBlock < kTcMaxParts ? f_min / kKBlock : kTcMaxParts;
-  const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);
-  const long long want = (3LL * dm.tc_grid + 4) / 5;
-  long long ks = (want + base - 1) / base;
-  if (ks > cap) ks = cap;
-  while (ks > 1 && base * ks > dm.tc_part_units) --ks;
-  return ks < 1 ? 1 : static_cast<int>(ks);
+  int best = 1;
+  long long bn = (base + grid - 1) / grid, bd = 1;  // rounds per unit of work: bn / bd
+  for (int ks = 2; ks <= cap && base * ks <= dm.tc_part_units; ++ks) {
+    const long long r = (base * ks + grid - 1) / grid;
+    if (r * bd < bn * ks) {
+      best = ks;
+      bn = r;
+      bd = ks;
+    }
+  }
+  return best;
 }
 
 struct Workspace {
