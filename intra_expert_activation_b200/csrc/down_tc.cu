@@ -20,6 +20,11 @@
 //     inactive neurons is an exact zero, so the sum is the same.
 // Warp roles as in the gate/up kernel: warp 0 TMA, warp 1 MMA + TMEM owner,
 // warps 2-5 drain TMEM into Y[slot][col] (fp32), coalesced across lanes.
+// With few units for the grid (decode batches with one to a few groups on
+// this path), a unit's K-blocks are cut into parts (tc_ksplit): each part
+// drains its sums into a workspace block, and the part that finishes last
+// (an atomic ticket per unit) adds the parts in part order and stores Y.
+// A candidate group that the row stream takes (cand_takes_gemv) is skipped.
 #include "common.cuh"
 
 namespace moe {
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_dep_wait();
   const int n_slices = p.dm.d / kDownSlice;
   const int n_tc = __ldcg(p.ws.meta + kMetaTcCount);
-  const int ks = tc_ksplit(p.dm, n_tc);  // > 1: parts add into Y (zeroed by the router's layout)
+  const int ks = tc_ksplit(p.dm, n_tc);  // > 1: units cut into K parts (ticketed sum)
   const int n_units = n_tc * n_slices * ks;
   if (static_cast<int>(blockIdx.x) >= n_units) return;  // no unit for this CTA: leave before TMEM
   if (warp == 1) tmem_alloc(tmem_slot, p.tmem_cols);

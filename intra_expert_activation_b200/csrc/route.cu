@@ -520,7 +520,21 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(Dims dm, Workspace w
     TX* xs = reinterpret_cast<TX*>(xs_raw);  // [tb][d]
     const int nvec = tb * d * (int)sizeof(TX) / 16;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok0 * d);
-    for (int i = tid; i < nvec; i += kThreads) reinterpret_cast<uint4*>(xs)[i] = __ldg(src + i);
+    uint4* xs4 = reinterpret_cast<uint4*>(xs);
+    constexpr int kV = 8;  // vectors per thread in flight together
+    for (int base = 0; base < nvec; base += kThreads * kV) {
+      uint4 r[kV];
+#pragma unroll
+      for (int i = 0; i < kV; ++i) {
+        const int j = base + tid + kThreads * i;
+        if (j < nvec) r[i] = __ldg(src + j);
+      }
+#pragma unroll
+      for (int i = 0; i < kV; ++i) {
+        const int j = base + tid + kThreads * i;
+        if (j < nvec) xs4[j] = r[i];
+      }
+    }
     __syncthreads();
     // the split-d partial sums (slices x E <= 32, so at most 32 x TPC
     // floats) reuse wcnt, which is cleared only after the top-k
@@ -574,6 +588,26 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(Dims dm, Workspace w
   route_finish(dm, ws, gridDim.x);
 }
 
+// One warp copies a row of nv 16-byte vectors with each lane's loads in
+// flight together (a row of d = 4096 bf16 is one batch of 16 vectors per
+// lane), instead of one load-store round trip per vector.
+__device__ __forceinline__ void copy_row(uint4* dst, const uint4* src, int nv, int lane) {
+  constexpr int kV = 16;
+  for (int base = 0; base < nv; base += 32 * kV) {
+    uint4 r[kV];
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+      const int j = base + lane + 32 * i;
+      if (j < nv) r[i] = __ldg(src + j);
+    }
+#pragma unroll
+    for (int i = 0; i < kV; ++i) {
+      const int j = base + lane + 32 * i;
+      if (j < nv) dst[j] = r[i];
+    }
+  }
+}
+
 template <typename TX>
 __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, const TX* x,
                                                       int tpc) {
@@ -597,7 +631,7 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
     }
     uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * dm.d);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * dm.d);
-    for (int i = lane; i < nv; i += 32) dst[i] = __ldg(src + i);
+    copy_row(dst, src, nv, lane);
     if (__ldcg(ws.y_zero + e)) {  // the GEMV path adds split partials into Y
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)slot * dm.d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -632,6 +666,7 @@ template <typename TX>
 __global__ void __launch_bounds__(kSmallThreads, 1)
     route_small_kernel(Dims dm, Workspace ws, const TX* x, const TX* Wr, const float* bias) {
   __shared__ float lg[kSmallTokens][kMaxExperts + 1];
+  __shared__ float lpart[4][kSmallTokens][kMaxExperts];  // split-d partial logits
   __shared__ int sel[kSmallTokens * 16];
   __shared__ int slot_s[kSmallTokens * 16];
   __shared__ int cnt[kMaxExperts];
@@ -642,13 +677,27 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   const int E = dm.E, d = dm.d, T = dm.T, k = dm.k;
   const int P = T * k;
 
-  for (int task = warp; task < T * E; task += kSmallWarps) {
-    const int t = task / E, e = task % E;
-    const float a = row_dot<TX>(x + (size_t)t * d, Wr + (size_t)e * d, d, lane);
-    if (lane == 0) lg[t][e] = a + (bias ? bias[e] : 0.f);
+  // (token, expert) dots; with fewer dots than warps each is split into ns
+  // slices of d (slices added in order), so every warp has one
+  const int TE = T * E;
+  const int ns = TE * 4 <= kSmallWarps ? 4 : TE * 2 <= kSmallWarps ? 2 : 1;
+  const int dsl = d / ns;  // d is a multiple of 256: slices stay whole vectors
+  for (int task = warp; task < TE * ns; task += kSmallWarps) {
+    const int sl = task / TE, te = task % TE;
+    const int t = te / E, e = te % E;
+    const float a = row_dot<TX>(x + (size_t)t * d + (size_t)sl * dsl,
+                                Wr + (size_t)e * d + (size_t)sl * dsl, dsl, lane);
+    if (lane == 0) lpart[sl][t][e] = a;
   }
   for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
   if (tid < kCntWords) ws.counters[tid] = 0ull;
+  __syncthreads();
+  for (int i = tid; i < TE; i += kSmallThreads) {
+    const int t = i / E, e = i % E;
+    float a = 0.f;
+    for (int sl = 0; sl < ns; ++sl) a += lpart[sl][t][e];
+    lg[t][e] = a + (bias ? bias[e] : 0.f);
+  }
   __syncthreads();
   for (int t = warp; t < T; t += kSmallWarps)
     topk_token(dm, ws, lg[t], t, lane, sel + t * k);
@@ -678,7 +727,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     const int slot = slot_s[p];
     uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * d);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(p / k) * d);
-    for (int i = lane; i < nv; i += 32) dst[i] = __ldg(src + i);
+    copy_row(dst, src, nv, lane);
     if (ws.y_zero[sel[p]]) {
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)slot * d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
