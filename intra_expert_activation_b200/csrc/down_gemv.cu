@@ -195,18 +195,9 @@ size_t down_gemv_smem_bytes(int d, bool bf16) {
 
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
                              const void* Wds, bool bf16, int n_sms, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(down_gemv_kernel<__nv_bfloat16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBudget);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(down_gemv_kernel<float>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kSmemBudget);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = bf16 ? smem_limit(down_gemv_kernel<__nv_bfloat16>, kSmemBudget)
+                             : smem_limit(down_gemv_kernel<float>, kSmemBudget);
+  if (e != cudaSuccess) return e;
   const int grid = n_sms;  // one CTA per SM
   const size_t smem = down_gemv_smem_bytes(dm.d, bf16);
   if (bf16)

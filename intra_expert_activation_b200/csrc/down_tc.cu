@@ -352,13 +352,8 @@ size_t down_tc_smem_bytes(int b_bytes, int stages) {
 }
 
 cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(down_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = smem_limit(down_tc_kernel, 227 * 1024);
+  if (e != cudaSuccess) return e;
   return launch_k(down_tc_kernel, grid, kThreads, smem, st, p);
 }
 

@@ -545,13 +545,8 @@ size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks) {
 }
 
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gate_up_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = smem_limit(gate_up_tc_kernel, 227 * 1024);
+  if (e != cudaSuccess) return e;
   return launch_k(gate_up_tc_kernel, grid, kThreads, smem, st, p);
 }
 

@@ -34,6 +34,16 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is per device, so it is set once per
+// (kernel, device) and remembered under a lock: contexts on several devices
+// of one process, or on several threads, each get it.
+cudaError_t smem_limit_at_least(const void* kernel, int bytes);
+template <typename... KArgs>
+cudaError_t smem_limit(void (*kernel)(KArgs...), int bytes) {
+  return smem_limit_at_least(reinterpret_cast<const void*>(kernel), bytes);
+}
+
 constexpr uint32_t kSpinLimit = 4u << 20;  // ~1 s of polling with backoff
 constexpr int kErrDeviceInvalid = 1;       // == MOE_ERR_INVALID: an internal consistency check failed
 constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT

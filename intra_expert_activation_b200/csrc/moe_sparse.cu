@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -20,6 +21,29 @@ using moe::Workspace;
 
 namespace moe {
 void set_last_error(const std::string& msg);
+cudaError_t smem_limit_at_least(const void* kernel, int bytes) {
+  struct Set {
+    const void* kernel;
+    int device, bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Set> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Set& s : done)
+    if (s.kernel == kernel && s.device == dev) {
+      if (s.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e == cudaSuccess) s.bytes = bytes;
+      return e;
+    }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({kernel, dev, bytes});
+  return e;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("MOE_PDL");

@@ -773,13 +773,8 @@ cudaError_t launch_route_t(const Dims& dm, const Workspace& ws, const TX* x, con
   const int grid = (dm.T + tpc - 1) / tpc;
   const size_t xbytes = (size_t)tpc * dm.d * sizeof(TX);
   const int stage_x = xbytes <= kStageBytes;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        route_kernel<TX, TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStageBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = smem_limit(route_kernel<TX, TPC>, (int)kStageBytes);
+  if (e != cudaSuccess) return e;
   return launch_k(route_kernel<TX, TPC>, grid, kThreads, stage_x ? xbytes : 0, st, dm, ws, x,
                   Wr, bias, tpc, stage_x);
 }

@@ -245,17 +245,10 @@ cudaError_t launch_updown_gemv(const Dims& dm, const Workspace& ws, const void* 
                                bool bf16, int n_sms, cudaStream_t st) {
   // dynamic shared memory as this launch needs it (the kernel's static
   // arrays come on top, so the attribute is raised to what is used only)
-  static size_t attr_bytes[2] = {0, 0};
   const size_t smem = updown_gemv_smem_bytes(dm.d, bf16);
-  if (smem > attr_bytes[bf16]) {
-    const cudaError_t e =
-        bf16 ? cudaFuncSetAttribute(updown_gemv_kernel<__nv_bfloat16>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-             : cudaFuncSetAttribute(updown_gemv_kernel<float>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_bytes[bf16] = smem;
-  }
+  const cudaError_t e = bf16 ? smem_limit(updown_gemv_kernel<__nv_bfloat16>, (int)smem)
+                             : smem_limit(updown_gemv_kernel<float>, (int)smem);
+  if (e != cudaSuccess) return e;
   if (bf16)
     return launch_k(updown_gemv_kernel<__nv_bfloat16>, n_sms, kThreads, smem, st, dm, ws,
                     static_cast<const __nv_bfloat16*>(Wu), static_cast<const __nv_bfloat16*>(Wus),
