@@ -263,14 +263,6 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
 
-// A candidate group (kPathCand) takes the row stream when its passes over
-// the union rows cost less than all F_e rows on the tensor cores; both down
-// kernels evaluate it on the union count the gate/up epilogue left.
-__device__ __forceinline__ bool cand_takes_gemv(int union_rows, int passes, int F_e) {
-  return static_cast<long long>(union_rows) * passes * kCandDen <=
-         static_cast<long long>(F_e) * kCandNum;
-}
-
 template <typename T>
 __device__ __forceinline__ T from_f32(float v);
 template <>

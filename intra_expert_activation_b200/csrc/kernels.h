@@ -66,6 +66,14 @@ constexpr int kGemvTokens = 8;      // tokens per GEMV pass (the row-stream mma'
 constexpr int kGemvCandMax = 8;
 constexpr int kCandNum = 9, kCandDen = 10;
 
+// A candidate group (kPathCand) takes the row stream when its passes over
+// the union rows cost less than all F_e rows on the tensor cores; both down
+// kernels evaluate it on the union count the gate/up epilogue left.
+__host__ __device__ inline bool cand_takes_gemv(int union_rows, int passes, int F_e) {
+  return static_cast<long long>(union_rows) * passes * kCandDen <=
+         static_cast<long long>(F_e) * kCandNum;
+}
+
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
             kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6, kMetaWords = 16 };

@@ -1,0 +1,125 @@
+// Host-side check of the scheduling rules that the router and the kernels
+// share (compiled with nvcc and run on the CPU, no GPU call): the K parts of
+// the tensor-core down units stay inside the workspace's part buffers and
+// tickets and give every part at least one K-block; the candidate-group rule
+// is the stated threshold; the row-stream stage geometry fits its budget.
+// Exits non-zero with the first violated case.
+#include <cstdio>
+#include <cstdlib>
+
+#include "gemv_common.cuh"
+#include "kernels.h"
+
+using namespace moe;
+
+static int fails = 0;
+static long long checked = 0;
+
+#define CHECK(cond, ...)                       \
+  do {                                         \
+    ++checked;                                 \
+    if (!(cond)) {                             \
+      if (fails++ < 10) {                      \
+        std::printf("FAIL %s: ", #cond);       \
+        std::printf(__VA_ARGS__);              \
+        std::printf("\n");                     \
+      }                                        \
+    }                                          \
+  } while (0)
+
+static void check_ksplit() {
+  const int modes[] = {kModeAuto, kModeDense, kModeGemv, kModeTc, kModeTcAll};
+  const int ds[] = {256, 512, 2048, 4096, 7168, 8192};
+  const int Fs_[] = {128, 384, 768, 1408, 14336, 65536};
+  const int Ts[] = {1, 2, 4, 8, 16, 17, 32, 48, 64, 65, 100, 128, 4096};
+  const int grids[] = {0, 1, 16, 148, 160, 296, 320, 512};
+  const int units_caps[] = {0, 640};
+  for (int mode : modes)
+    for (int d : ds)
+      for (int F : Fs_)
+        for (int S = 0; S <= 2; ++S)
+          for (int Fsh : {128, 1408})
+            for (int T : Ts)
+              for (int grid : grids)
+                for (int cap_units : units_caps) {
+                  Dims dm = {};
+                  dm.mode = mode;
+                  dm.d = d;
+                  dm.F = F;
+                  dm.S = S;
+                  dm.Fs = S > 0 ? Fsh : 0;
+                  dm.T = T;
+                  dm.tc_grid = grid;
+                  dm.tc_part_units = cap_units;
+                  const int nslices = d / kDownSlice;
+                  const int tmax = T < kGroupMax ? T : kGroupMax;
+                  const int n_max = (tmax + 15) / 16 * 16;
+                  for (int n_tc = 0; n_tc <= 700; n_tc += (n_tc < 40 ? 1 : 37)) {
+                    const int ks = tc_ksplit(dm, n_tc);
+                    const long long base = (long long)n_tc * nslices;
+                    CHECK(ks >= 1 && ks <= kTcMaxParts, "ks %d", ks);
+                    if (mode == kModeTc || n_max > kTcPartTokens || cap_units == 0 || grid == 0)
+                      CHECK(ks == 1, "mode %d n_max %d cap %d grid %d ks %d", mode, n_max,
+                            cap_units, grid, ks);
+                    if (ks > 1) {
+                      CHECK(base * ks <= cap_units, "base %lld ks %d cap %d", base, ks, cap_units);
+                      CHECK(4 * base < 3LL * grid, "base %lld grid %d", base, grid);
+                      // every part of every expert kind has at least one K-block
+                      for (int kind = 0; kind < (S > 0 ? 2 : 1); ++kind) {
+                        const int nk = (kind ? dm.Fs : F) / kKBlock;
+                        for (int p = 0; p < ks; ++p) {
+                          const int k0 = nk * p / ks, k1 = nk * (p + 1) / ks;
+                          CHECK(k1 - k0 >= 1, "F %d Fs %d ks %d part %d", F, dm.Fs, ks, p);
+                        }
+                      }
+                      // the largest part-buffer element a unit touches
+                      const long long last =
+                          ((base - 1) * ks + (ks - 1)) * kTcPartTokens * kDownSlice +
+                          (long long)(n_max - 1) * kDownSlice + (kDownSlice - 1);
+                      CHECK(last < (long long)cap_units * kTcPartTokens * kDownSlice,
+                            "part buffer index %lld", last);
+                      CHECK(base <= cap_units, "tickets %lld > %d", base, cap_units);
+                    }
+                  }
+                }
+}
+
+static void check_candidates() {
+  for (int F : {128, 768, 1408, 14336}) {
+    for (int passes = 1; passes <= 2; ++passes) {
+      bool prev = true;
+      for (int u = 0; u <= F; ++u) {
+        const bool take = cand_takes_gemv(u, passes, F);
+        CHECK(take == ((long long)u * passes * 10 <= 9LL * F), "F %d u %d", F, u);
+        CHECK(!take || prev, "not monotone at F %d u %d", F, u);  // once false, stays false
+        prev = take;
+      }
+      CHECK(cand_takes_gemv(0, passes, F), "empty union");
+      CHECK(!cand_takes_gemv(F, passes, F), "full union");
+    }
+  }
+}
+
+static void check_geometry() {
+  for (int es : {2, 4})
+    for (int d = 128; d <= 16384; d += 128) {
+      if (es == 2 && d % 256) continue;  // bf16 layers: d_model a multiple of 256
+      const int row_bytes = d * es;
+      for (int extra : {0, 16, 272, 512}) {
+        const Geometry g = geometry(row_bytes, extra);
+        CHECK(g.n_stages >= 2 && g.n_stages <= kMaxStages, "d %d es %d stages %d", d, es,
+              g.n_stages);
+        CHECK((long long)g.n_stages * g.stage <= kSmemBudget, "d %d smem", d);
+        CHECK(g.block <= kBlockBytes && g.block % kSliceBytes == 0, "block %d", g.block);
+        CHECK(g.stride % 16 == 0 && g.stage % 16 == 0, "alignment d %d", d);
+      }
+    }
+}
+
+int main() {
+  check_ksplit();
+  check_candidates();
+  check_geometry();
+  std::printf("%s %lld checks, %d failed\n", fails ? "FAIL" : "OK", checked, fails);
+  return fails ? 1 : 0;
+}
