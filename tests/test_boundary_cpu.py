@@ -136,3 +136,24 @@ def test_binding_refuses_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_LIB", None)
     with pytest.raises(RuntimeError, match="missing"):
         _lib.load()
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C11 program compiled against include/moe_sparse.h with warnings as
+    errors links against the library and gets the host-only answers
+    (descriptor checks, workspace size, stage names, clean init failure)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if not cc:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "c_abi_check")
+    pkg = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", exe,
+                        "-L", pkg, "-lmoe_sparse", f"-Wl,-rpath,{pkg}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
