@@ -8,3 +8,4 @@ Python binding.
 
 from ._lib import LIB_PATH, PATHS, STAGES, MoEError, load  # noqa: F401
 from .layer import MoESparseLayer  # noqa: F401
+from .sharded import DffShardedLayer, shard_rows  # noqa: F401
