@@ -3,6 +3,7 @@
 //   route -> permute -> gate_up -> union_scan -> down (GEMV and/or TC) -> combine
 // all on the caller's stream, with no allocation and no host synchronisation.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -68,6 +69,30 @@ namespace {
 constexpr int kStages = 8;
 const char* kStageNames[kStages] = {"route",       "permute",   "gate_up", "union_scan",
                                     "updown_gemv", "down_gemv", "down_tc", "combine"};
+// NVTX ranges (no-ops unless a profiler is attached): one per forward, one
+// per stage, so that a profiler can select the layer's launches by name
+const char* kNvtxNames[kStages] = {"moe.route",       "moe.permute",   "moe.gate_up",
+                                   "moe.union_scan",  "moe.updown_gemv", "moe.down_gemv",
+                                   "moe.down_tc",     "moe.combine"};
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+// The stage range that is open: mark(i) closes the previous stage's range
+// and opens stage i's; whatever is still open closes with the forward.
+struct NvtxStages {
+  bool open = false;
+  void next(int i) {
+    if (open) nvtxRangePop();
+    open = i < kStages;
+    if (open) nvtxRangePushA(kNvtxNames[i]);
+  }
+  ~NvtxStages() {
+    if (open) nvtxRangePop();
+  }
+};
 
 thread_local std::string g_init_error;
 
@@ -532,7 +557,10 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   cudaEvent_t* evs = timing ? &c->ev[static_cast<size_t>(set) * (kStages + 1)] : nullptr;
   uint8_t* ran = timing ? &c->ran[static_cast<size_t>(set) * kStages] : nullptr;
   bool stage_ran[kStages] = {};
+  NvtxRange forward_range("moe.forward");
+  NvtxStages stage_range;
   auto mark = [&](int i) {
+    stage_range.next(i);
     if (timing) cudaEventRecord(evs[i], st);
   };
   cudaError_t e;
