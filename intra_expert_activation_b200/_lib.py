@@ -10,7 +10,10 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_sparse.so")
+# MOE_SPARSE_LIB=check selects the bounds-checked build (build.py --check)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libmoe_sparse_check.so" if os.environ.get("MOE_SPARSE_LIB") == "check"
+                        else "libmoe_sparse.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID = 1

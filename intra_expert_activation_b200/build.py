@@ -1,6 +1,11 @@
 """Build libmoe_sparse.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m intra_expert_activation_b200.build [--force] [-v]
+    python -m intra_expert_activation_b200.build [--force] [-v] [--check]
+
+--check builds libmoe_sparse_check.so instead: the same library with the
+kernels' bounds checks on the data-derived indices compiled in
+(-DMOE_CHECK=1; a failed check sets MOE_ERR_INVALID in the status word). The
+binding loads it when MOE_SPARSE_LIB=check is set in the environment.
 
 Objects go to _build/ at the repository root; the shared library is written
 next to this file so that the Python binding loads it from the package.
@@ -20,6 +25,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_sparse.so")
+LIB_CHECK = os.path.join(PKG, "libmoe_sparse_check.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
@@ -45,15 +51,19 @@ def _mtime(p):
     return os.path.getmtime(p) if os.path.exists(p) else -1.0
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          check: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "check") if check else BUILD
+    lib = LIB_CHECK if check else LIB
+    flags = FLAGS + (["-DMOE_CHECK=1"] if check else [])
+    os.makedirs(out_dir, exist_ok=True)
     hdr_t = max(_mtime(h) for h in headers())
     objs, jobs = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _mtime(obj) < max(_mtime(src), hdr_t):
-            cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [nvcc(), *ARCH, *flags, "-c", src, "-o", obj]
             if ptxas_info:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
@@ -69,8 +79,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
 
     with ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as pool:
         list(pool.map(run, jobs))
-    if jobs or not os.path.exists(LIB) or _mtime(LIB) < max(_mtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcudart_static", "-lrt", "-ldl",
+    if jobs or not os.path.exists(lib) or _mtime(lib) < max(_mtime(o) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", lib, *objs, "-lcudart_static", "-lrt", "-ldl",
                "-lpthread"]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -78,7 +88,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
@@ -86,5 +96,6 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
+    ap.add_argument("--check", action="store_true", help="bounds-checked build (MOE_CHECK=1)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_info))
+    print(build(a.force, a.verbose, a.ptxas_info, a.check))

@@ -100,7 +100,9 @@ __global__ void __launch_bounds__(256) combine_kernel(Dims dm, Workspace ws, TX*
   __shared__ int slot[16];
   __shared__ float w[16];
   if (threadIdx.x < k) {
-    slot[threadIdx.x] = __ldcg(ws.slot_of + t * k + threadIdx.x);
+    int s = __ldcg(ws.slot_of + t * k + threadIdx.x);
+    if (!moe_in_bounds(ws.status, s >= 0 && s < dm.slots_routed)) s = 0;
+    slot[threadIdx.x] = s;
     w[threadIdx.x] = __ldcg(ws.topk_w + t * k + threadIdx.x);
   }
   __syncthreads();

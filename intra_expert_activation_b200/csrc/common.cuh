@@ -19,6 +19,21 @@ __device__ __forceinline__ void report_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Checked builds (-DMOE_CHECK=1, `build.py --check`): bounds checks on the
+// indices the kernels compute from data (slots, union rows). A failed check
+// records MOE_ERR_INVALID in the status word and the caller skips or clamps
+// the access; in the normal build the checks compile away.
+#ifndef MOE_CHECK
+#define MOE_CHECK 0
+#endif
+__device__ __forceinline__ bool moe_in_bounds(int* status, bool ok) {
+  if (MOE_CHECK && !ok) {
+    report_error(status, kErrDeviceInvalid);
+    return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

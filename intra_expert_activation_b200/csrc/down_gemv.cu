@@ -124,7 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane < kBatch) {
             if (lane < cnt) {
-              const int j = list[pos + lane];
+              int j = list[pos + lane];
+              if (!moe_in_bounds(ws.status, j < 32 * k.words && slot + MT <= dm.slots_total))
+                j = 0;  // checked build: a bad row or slot is recorded and clamped
               const uint32_t hdst = stg_s + kBatch * geo.stride + lane * kHBytes;
               const char* hsrc = ht + ((size_t)j * ld + slot) * ES;
               if constexpr (ES == 2) {

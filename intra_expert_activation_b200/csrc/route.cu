@@ -623,8 +623,10 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
     const int t = item / k;
     const int e = __ldcg(ws.topk_idx + item);
     const int cta = t / tpc;
+    if (!moe_in_bounds(ws.status, e >= 0 && e < E)) return;
     const int slot = __ldcg(ws.expert_off + e) + __ldcg(ws.hist + (size_t)e * n_cta + cta) +
                      __ldcg(ws.rank_cta + item);
+    if (!moe_in_bounds(ws.status, slot >= 0 && slot < dm.slots_routed)) return;
     if (lane == 0) {
       ws.perm[slot] = t;
       ws.slot_of[item] = slot;
@@ -714,7 +716,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   build_layout(dm, ws, cnt, poff);
   __syncthreads();
   for (int p = tid; p < P; p += kSmallThreads) {
-    const int slot = poff[sel[p]] + slot_s[p];
+    int slot = poff[sel[p]] + slot_s[p];
+    if (!moe_in_bounds(ws.status, slot >= 0 && slot < dm.slots_routed)) slot = 0;
     slot_s[p] = slot;
     ws.perm[slot] = p / k;
     ws.slot_of[p] = slot;

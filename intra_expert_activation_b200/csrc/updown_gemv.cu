@@ -122,14 +122,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   mt | (cb << 8) | (last_up << 16) | (phase ? kKindDown : 0));
               meta[1] = make_int4(pos, k.xrow0 + k.p * MT, shared, n_list);
               uint16_t* rj = reinterpret_cast<uint16_t*>(meta + 2);
-              for (int r = 0; r < kBatch; ++r) rj[r] = r < cnt ? list[pos + r] : 0;
+              for (int r = 0; r < kBatch; ++r) {
+                const int j = r < cnt ? list[pos + r] : 0;
+                rj[r] = moe_in_bounds(ws.status, j < 32 * k.words) ? j : 0;  // checked build: clamp
+              }
               mbar_arrive_expect_tx(full + b, static_cast<uint32_t>(cnt * cbytes));
             }
             __syncwarp();
-            if (lane < cnt)
-              bulk_load(stg_s + lane * geo.stride,
-                        wexp + (size_t)list[pos + lane] * d + cb * (kBlockBytes / ES), cbytes,
-                        smem_u32(full + b));
+            if (lane < cnt) {
+              int j = list[pos + lane];
+              if (!moe_in_bounds(ws.status, j < 32 * k.words)) j = 0;  // checked build: clamp
+              bulk_load(stg_s + lane * geo.stride, wexp + (size_t)j * d + cb * (kBlockBytes / ES),
+                        cbytes, smem_u32(full + b));
+            }
             ++s;
           }
         }

@@ -157,3 +157,23 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
+
+
+@pytest.mark.timeout(600)
+def test_checked_build_exports_the_same_abi():
+    """build.py --check compiles the kernels' bounds checks in (MOE_CHECK=1)
+    into a separate library with the same exported entry points, which the
+    binding loads under MOE_SPARSE_LIB=check."""
+    import subprocess
+    import sys
+    from intra_expert_activation_b200 import build
+    path = build.build(check=True)
+    assert path.endswith("libmoe_sparse_check.so") and os.path.exists(path)
+    out = os.popen(f"nm -D --defined-only {path}").read()
+    syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert {s for s in syms if s.startswith("moe_")} == set(declared_functions())
+    r = subprocess.run([sys.executable, "-c",
+                        "from intra_expert_activation_b200 import _lib; print(_lib.LIB_PATH)"],
+                       capture_output=True, text=True, cwd=ROOT,
+                       env={**os.environ, "MOE_SPARSE_LIB": "check"})
+    assert r.returncode == 0 and r.stdout.strip() == path, r.stdout + r.stderr
