@@ -49,20 +49,25 @@ GATE_UP_TRAFFIC_RATIO = 1.0106
 
 
 def parse():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="mixtral_decode")
-    ap.add_argument("--sparsity", type=float, default=0.7)
+    ap = argparse.ArgumentParser(description="MoE-layer tokens/s of the sparse layer on B200")
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks (one per GPU, launched by torchrun for N > 1): replicas")
+    ap.add_argument("--steps", type=int, default=20, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours",
+                    help="reference: time the CPU oracle on the host cores instead")
+    ap.add_argument("--workload", default="mixtral_decode", choices=sorted(WORKLOADS),
+                    help="synthetic workload (moe_inputs/workloads.py)")
+    ap.add_argument("--sparsity", type=float, default=0.7,
+                    help="target sparsity; tau comes from tests/golden/tau_calibration.json")
     ap.add_argument("--score", choices=("h", "gate"), default="h",
                     help="h: active iff |SiLU(g) u| > tau; gate: active iff |SiLU(g)| > tau with "
                          "the sparse up projection (the pages' own system)")
     ap.add_argument("--tokens", type=str, default="", help="comma list overriding the batches")
-    ap.add_argument("--no-dense", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-path comparison")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end run with host buffers")
     ap.add_argument("--eager", action="store_true",
                     help="time eager API calls instead of replaying a captured CUDA graph")
     return ap.parse_args()
