@@ -43,9 +43,21 @@ METRIC = "MoE-layer tokens/s and effective HBM GB/s vs own dense path, 0-90% spa
 FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic / algorithmic bytes of gate_up_tc_kernel from one ncu capture of a smaller
 # launch of the same kernel (decode batch T=8, 7 experts touched): traffic grows with the
-# touched experts, so a launch's traffic is this ratio times its algorithmic bytes
-# (profiles/gate_up_tc.mixtral_decode_T8.md). None once the kernel has changed since.
-GATE_UP_TRAFFIC_RATIO = 1.0106
+# touched experts, so a launch's traffic is this ratio times its algorithmic bytes. The
+# ratio holds only for the kernel source it was captured on: SOURCE_SHA16 is the hash of
+# those files (kernel_source_hash); when the sources differ the line reports traffic null.
+GATE_UP_TRAFFIC = {"ratio": 1.0106, "source_sha16": "",
+                   "files": ("gate_up_tc.cu", "common.cuh", "kernels.h")}
+
+
+def kernel_source_hash(files) -> str:
+    """First 16 hex digits of the sha256 over the named kernel sources, in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "intra_expert_activation_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def parse():
@@ -220,15 +232,15 @@ def oracle_step_time(wl, tokens, tau, tau_s, w_host, score="h"):
 
 def run_reference(args, world, rank):
     """The oracle arm: the fp64 CPU oracle timed on the host cores, on rank 0
-    only; each step is a bounded sample of the workload's step (its T = 8
-    batch, or its smallest one)."""
+    only; each step is the same step the GPU arm times (every batch of the
+    workload), the same sample as the GPU arm's cpu_baseline."""
     if rank != 0:
         return 0
     wl = WORKLOADS[args.workload]
     tokens = [int(t) for t in args.tokens.split(",")] if args.tokens else list(wl.tokens)
     tau, tau_s, calib_sparsity = load_tau(args.workload, args.sparsity, args.score)
     w = make_weights(wl.shape, wl.weight_seed)
-    sample = [8] if 8 in tokens else [min(tokens)]
+    sample = list(tokens)
     for _ in range(args.warmup):
         oracle_step_time(wl, sample, tau, tau_s, w, args.score)
     t = sum(oracle_step_time(wl, sample, tau, tau_s, w, args.score) for _ in range(args.steps))
@@ -242,8 +254,9 @@ def run_reference(args, world, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args, wl, tokens, tau, calib_sparsity, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: the decode batch T={sample} of {args.workload} "
-                                   f"(fp64 numpy oracle on {cores} host threads)"},
+                         "sample": f"each step: the decode batches T={sample} of "
+                                   f"{args.workload}, as in the GPU arm's step (fp64 numpy "
+                                   f"oracle on {cores} host threads)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -476,8 +489,9 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = peaks()
     g_ach = gate_bytes_tot / (gate_ms_tot * 1e-3) / 1e9 if gate_ms_tot else 0.0
     n_gate_launches = args.steps * len(tokens)
-    g_traffic = None if GATE_UP_TRAFFIC_RATIO is None or args.score != "h" else \
-        round(GATE_UP_TRAFFIC_RATIO * gate_bytes_tot / n_gate_launches)
+    traffic_ok = kernel_source_hash(GATE_UP_TRAFFIC["files"]) == GATE_UP_TRAFFIC["source_sha16"]
+    g_traffic = None if not traffic_ok or args.score != "h" else \
+        round(GATE_UP_TRAFFIC["ratio"] * gate_bytes_tot / n_gate_launches)
     d_ach = down_bytes_tot / (down_ms_tot * 1e-3) / 1e9 if down_ms_tot else 0.0
     # the gate/up kernel is HBM-bound below the ridge (decode, few tokens per
     # expert) and tensor-bound above it (prefill): grade it on its own bound

@@ -45,7 +45,7 @@
  * Conventions shared by every entry point
  *   - Tensors are DEVICE pointers on desc.device, contiguous, row-major,
  *     16-byte aligned, in desc.dtype (x, weights, out), except router_bias
- *     (float32). The caller owns them; the library never frees them.
+ *     (float32) and out when desc.out_f32 is set (float32). The caller owns them; the library never frees them.
  *       x         [T][d_model]
  *       W_router  [n_experts][d_model]            logits = x W_router^T
  *       W_gate    [n_experts][d_ff][d_model]      row j: neuron j's input weights
@@ -125,6 +125,9 @@ typedef struct {
                                  else all rows on the tensor cores */
   float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: never) */
   int32_t score;              /* moe_score (0: MOE_SCORE_H) */
+  int32_t out_f32;            /* 1: out is float32 [T][d_model] for either dtype (the combine's
+                                 fp32 sums, not rounded; for partial outputs that are summed
+                                 afterwards, e.g. over d_ff shards); 0: out is in dtype */
 } moe_sparse_desc;
 
 typedef struct {
@@ -218,11 +221,13 @@ MOE_API const char* moe_sparse_stage_name(int32_t i);
 /* Last error message of ctx (or of the last failed init if ctx is NULL). */
 MOE_API const char* moe_sparse_last_error(const moe_sparse_ctx* ctx);
 
-/* Routing only, for callers that must not allocate device memory (code that
- * runs while a CUDA graph is being captured, plug-ins living inside another
- * framework's fixed memory plan, serving loops that reserve all memory up
- * front). The paper has no counterpart: it is an allocation-free variant of
- * the forward's router kernel, not a step of the method.
+/* Routing only, for callers that must not allocate device memory: plug-ins
+ * living inside another framework's fixed memory plan (where a private
+ * cudaMalloc breaks the host's accounting or fragments its pool), and serving
+ * loops that reserve all device memory up front and treat any later
+ * allocation as a failure. The paper has no counterpart: it is an
+ * allocation-free variant of the forward's router kernel, not a step of the
+ * method.
  * It computes what moe_sparse_forward's router computes for x [T][d_model]
  * and W_router [n_experts][d_model] (device pointers, dtype, 16-byte aligned;
  * router_bias [n_experts] float32 or NULL) into caller DEVICE buffers:

@@ -53,6 +53,7 @@ class moe_sparse_desc(ctypes.Structure):
         ("gemv_max_tokens", ctypes.c_int32),
         ("gather_max_density", ctypes.c_float),
         ("score", ctypes.c_int32),
+        ("out_f32", ctypes.c_int32),
     ]
 
 

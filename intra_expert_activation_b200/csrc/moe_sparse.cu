@@ -177,6 +177,7 @@ moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
   }
   if (d->path < MOE_PATH_AUTO || d->path > MOE_PATH_SPARSE_TC_ALLROWS) { err = "unknown path"; return MOE_ERR_INVALID; }
   if (d->score != MOE_SCORE_H && d->score != MOE_SCORE_GATE) { err = "unknown score"; return MOE_ERR_INVALID; }
+  if (d->out_f32 != 0 && d->out_f32 != 1) { err = "out_f32 must be 0 or 1"; return MOE_ERR_INVALID; }
   if (!bf16 && (d->path == MOE_PATH_SPARSE_TC || d->path == MOE_PATH_SPARSE_TC_ALLROWS)) {
     err = "tensor-core down paths need bf16";
     return MOE_ERR_UNSUPPORTED;
@@ -664,7 +665,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     stage_ran[6] = true;
   }
   mark(7);
-  e = moe::launch_combine(dm, c->ws, out, c->bf16, st);
+  e = moe::launch_combine(dm, c->ws, out, c->bf16 && !c->desc.out_f32, st);
   if (e != cudaSuccess) return cuda_fail(c, e, "combine launch");
   stage_ran[7] = true;
   mark(8);

@@ -25,6 +25,7 @@
 //   records perm / slot_of and copies the x row to X_perm[slot]; extra warps
 //   zero the padding slots.
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -32,13 +33,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxExperts = 256;
+constexpr int kMaxExperts = kTopkMaxExperts;
 constexpr int kSmallTokens = 4;  // single-CTA routing (and permute) up to this batch
-
-// Total order used by the top-k: larger logit first, then lower index.
-__device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
-  return va > vb || (va == vb && ea < eb);
-}
 
 // 16-byte vectors of x / W_router rows, widened to fp32 (exactly).
 template <typename TX>
@@ -371,57 +367,18 @@ __device__ __forceinline__ float row_dot(const TX* a, const TX* b, int d, int la
   return acc;
 }
 
-// Top-k of one token's logits (one warp): the k largest, equal logits to the
-// lower expert index; softmax over all experts; weights p / sum(p_sel) or p.
-// Writes topk_idx / topk_w of token `tok` and the chosen experts to sel[0..k).
+// Top-k of one token's logits (one warp, topk_warp): the k largest, equal
+// logits to the lower expert index; softmax over all experts; weights
+// p / sum(p_sel) or p. Writes topk_idx / topk_w of token `tok` and the chosen
+// experts to sel[0..k).
 __device__ __forceinline__ void topk_token(const Dims& dm, const Workspace& ws, const float* lgt,
                                            int tok, int lane, int* sel) {
-  const int E = dm.E, k = dm.k;
-  float v[kMaxExperts / 32];
-#pragma unroll
-  for (int j = 0; j < kMaxExperts / 32; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = e < E ? lgt[e] : -INFINITY;
-  }
-  float mx = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < kMaxExperts / 32; ++j) mx = fmaxf(mx, v[j]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float z = 0.f;
-#pragma unroll
-  for (int j = 0; j < kMaxExperts / 32; ++j)
-    if (lane + 32 * j < E) z += expf(v[j] - mx);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-
-  int my_e = -1;
-  float my_p = 0.f, psum = 0.f;
-  for (int i = 0; i < k; ++i) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && better(v[j], e, bv, be)) { bv = v[j]; be = e; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-    }
-#pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j)
-      if (lane + 32 * j == be) v[j] = -INFINITY;
-    const float p = expf(bv - mx) / z;
-    psum += p;
-    if (lane == i) { my_e = be; my_p = p; }
-  }
+  const int k = dm.k;
+  const TopkResult r = topk_warp(lgt, dm.E, k, lane);
   if (lane < k) {
-    ws.topk_idx[tok * k + lane] = my_e;
-    ws.topk_w[tok * k + lane] = dm.renorm ? my_p / psum : my_p;
-    sel[lane] = my_e;
+    ws.topk_idx[tok * k + lane] = r.my_e;
+    ws.topk_w[tok * k + lane] = dm.renorm ? r.my_p / r.psum : r.my_p;
+    sel[lane] = r.my_e;
   }
 }
 

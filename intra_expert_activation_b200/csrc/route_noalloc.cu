@@ -1,8 +1,8 @@
 // moe_sparse_route_noalloc: the layer's routing step (logits, softmax, top-k,
 // stable grouping of the (token, expert) pairs by expert) for callers that
-// must not allocate device memory, for example code that runs while a CUDA
-// graph is being captured, plug-ins that live inside another framework's
-// fixed memory plan, or serving loops that reserve all memory up front. It
+// must not allocate device memory, for example plug-ins that live inside
+// another framework's fixed memory plan, or serving loops that reserve all
+// device memory up front and treat a later allocation as a failure. It
 // computes what the forward's router computes, into caller buffers, and keeps
 // its scratch (per-CTA expert histograms, per-pair ranks, a completion
 // ticket) in one file-scope device array instead of a context workspace.
@@ -13,6 +13,7 @@
 #include <string>
 
 #include "kernels.h"
+#include "topk.cuh"
 #include "moe_sparse.h"
 
 namespace moe {
@@ -70,10 +71,6 @@ __device__ __forceinline__ void load8<float>(const float* p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-__device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
-  return va > vb || (va == vb && ea < eb);
-}
-
 template <typename TX>
 __global__ void __launch_bounds__(kThreads) route_noalloc_kernel(NaArgs a) {
   __shared__ float lg[16][kMaxE + 1];
@@ -113,52 +110,14 @@ __global__ void __launch_bounds__(kThreads) route_noalloc_kernel(NaArgs a) {
   __syncthreads();
 
   // top-k per token: the k largest logits, ties to the lower expert index
+  // (NaN logits rank as -inf; the ids are distinct and in [0, E))
   for (int t = warp; t < tb; t += kWarps) {
-    float v[kMaxE / 32];
-#pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) {
-      const int e = lane + 32 * j;
-      v[j] = e < E ? lg[t][e] : -INFINITY;
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) mx = fmaxf(mx, v[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float z = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j)
-      if (lane + 32 * j < E) z += expf(v[j] - mx);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    int my_e = -1;
-    float my_p = 0.f, psum = 0.f;
-    for (int i = 0; i < k; ++i) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < kMaxE / 32; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && better(v[j], e, bv, be)) { bv = v[j]; be = e; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-      }
-#pragma unroll
-      for (int j = 0; j < kMaxE / 32; ++j)
-        if (lane + 32 * j == be) v[j] = -INFINITY;
-      const float p = expf(bv - mx) / z;
-      psum += p;
-      if (lane == i) { my_e = be; my_p = p; }
-    }
+    const moe::TopkResult r = moe::topk_warp(lg[t], E, k, lane);
     if (lane < k) {
       const int tok = tok0 + t;
-      a.topk_idx[tok * k + lane] = my_e;
-      a.topk_w[tok * k + lane] = a.renorm ? my_p / psum : my_p;
-      sel[t * k + lane] = my_e;
+      a.topk_idx[tok * k + lane] = r.my_e;
+      a.topk_w[tok * k + lane] = a.renorm ? r.my_p / r.psum : r.my_p;
+      sel[t * k + lane] = r.my_e;
     }
   }
   __syncthreads();

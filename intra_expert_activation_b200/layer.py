@@ -34,7 +34,7 @@ class MoESparseLayer:
                  max_tokens: int, renormalize: bool = True, n_shared: int = 0,
                  d_ff_shared: int = 0, dtype: str = "bf16", path: str = "auto",
                  debug: bool = False, device: int = 0, gemv_max_tokens: int = 0,
-                 gather_max_density: float = 0.0, score: str = "h"):
+                 gather_max_density: float = 0.0, score: str = "h", out_f32: bool = False):
         self.lib = _lib.load()
         self.torch_dtype, code = _DT[dtype]
         self.dtype = dtype
@@ -44,8 +44,10 @@ class MoESparseLayer:
         self.desc = _lib.moe_sparse_desc(
             d_model, d_ff, n_experts, top_k_max, max_tokens, int(renormalize), n_shared,
             d_ff_shared, code, _lib.PATHS[path], int(debug), device, gemv_max_tokens,
-            gather_max_density, _lib.SCORES[score])
+            gather_max_density, _lib.SCORES[score], int(out_f32))
         self.score = score
+        # out: float32 (the combine's sums, unrounded) or the layer's dtype
+        self.out_dtype = torch.float32 if out_f32 else self.torch_dtype
         self.ctx = ctypes.c_void_p()
         _lib.check(self.lib.moe_sparse_init(ctypes.byref(self.desc), ctypes.byref(self.ctx)),
                    "moe_sparse_init")
@@ -89,9 +91,9 @@ class MoESparseLayer:
             self._check(router_bias, "router_bias", torch.float32)
         T = x.shape[0]
         if out is None:
-            out = torch.empty((T, self.d_model), dtype=self.torch_dtype, device=self.device)
+            out = torch.empty((T, self.d_model), dtype=self.out_dtype, device=self.device)
         else:
-            self._check(out, "out")
+            self._check(out, "out", self.out_dtype)
         _lib.check(self.lib.moe_sparse_forward(
             self.ctx, _ptr(x), T, _ptr(W_router), _ptr(router_bias), _ptr(W_gate), _ptr(W_up),
             _ptr(W_down), float(tau), int(top_k), _ptr(out), self._stream(stream)),

@@ -14,8 +14,12 @@ Execution", Technical Summary > Methodology > System Implementation in
 vLLM]; this split is the standard tensor-parallel split of an FFN.)
 
 The per-rank layer is the C-ABI library's; the all-reduce is the process
-group's (NCCL over NVLink on GPUs). Partial outputs are reduced in fp32 by
-default and rounded to the layer's dtype once.
+group's (NCCL over NVLink on GPUs). With the default fp32 reduction each
+rank's layer writes its partial output in fp32 straight from the combine's
+sums (desc.out_f32, no rounding), the all-reduce adds the partials in fp32,
+and the sum is rounded to the layer's dtype once. With another reduce_dtype
+the partials are written in the layer's dtype and reduced in reduce_dtype:
+two roundings.
 """
 
 from __future__ import annotations
@@ -57,11 +61,16 @@ class DffShardedLayer:
         if d_ff % self.world or (n_shared and d_ff_shared % self.world):
             raise ValueError("d_ff (and d_ff_shared) must be divisible by the group size")
         self.reduce_dtype = reduce_dtype
+        if reduce_dtype == torch.float32:
+            layer_kw.setdefault("out_f32", True)  # partials leave the layer unrounded
         factory = layer_factory or MoESparseLayer
         self.layer = factory(d_model, d_ff // self.world, n_experts, top_k_max, max_tokens,
                              n_shared=n_shared,
                              d_ff_shared=d_ff_shared // self.world if n_shared else 0,
                              **layer_kw)
+        # the dtype of the returned output: the layer's own (bf16 / fp32), or
+        # that of the partials for a layer without one
+        self.result_dtype = getattr(self.layer, "torch_dtype", None)
 
     def shard(self, W: torch.Tensor) -> torch.Tensor:
         """This rank's rows of a full [experts][d_ff][d_model] weight."""
@@ -77,8 +86,9 @@ class DffShardedLayer:
                 router_bias: Optional[torch.Tensor] = None) -> torch.Tensor:
         part = self.layer.forward(x, W_router, W_gate, W_up, W_down, tau, top_k,
                                   router_bias=router_bias)
+        final = self.result_dtype or part.dtype
         if self.world == 1:
-            return part
+            return part.to(final)
         acc = part.to(self.reduce_dtype)
         dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=self.group)
-        return acc.to(part.dtype)
+        return acc.to(final)

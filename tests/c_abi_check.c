@@ -7,7 +7,7 @@
 
 #include "moe_sparse.h"
 
-_Static_assert(sizeof(moe_sparse_desc) == 15 * 4, "moe_sparse_desc layout");
+_Static_assert(sizeof(moe_sparse_desc) == 16 * 4, "moe_sparse_desc layout");
 _Static_assert(sizeof(moe_stats) == 12 * 8, "moe_stats layout");
 
 static int fails = 0;
@@ -31,6 +31,7 @@ int main(void) {
   d.dtype = MOE_BF16;
   d.path = MOE_PATH_AUTO;
   d.score = MOE_SCORE_H;
+  d.out_f32 = 0;
   CHECK(moe_sparse_validate_desc(&d) == MOE_OK);
 
   size_t bytes = 0;
@@ -46,6 +47,9 @@ int main(void) {
   CHECK(moe_sparse_validate_desc(&bad) != MOE_OK);
   bad = d;
   bad.score = 7;
+  CHECK(moe_sparse_validate_desc(&bad) == MOE_ERR_INVALID);
+  bad = d;
+  bad.out_f32 = 2;
   CHECK(moe_sparse_validate_desc(&bad) == MOE_ERR_INVALID);
   CHECK(moe_sparse_validate_desc(NULL) == MOE_ERR_INVALID);
 

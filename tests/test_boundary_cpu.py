@@ -52,7 +52,7 @@ def test_only_the_abi_is_exported():
 
 
 def test_struct_sizes_match_header():
-    assert ctypes.sizeof(_lib.moe_sparse_desc) == 15 * 4
+    assert ctypes.sizeof(_lib.moe_sparse_desc) == 16 * 4
     assert ctypes.sizeof(_lib.moe_stats) == 12 * 8
 
 
@@ -82,6 +82,7 @@ def test_valid_desc_accepted(lib):
     (dict(dtype=_lib.MOE_F32, d_model=256, d_ff=512, path=3), _lib.MOE_ERR_UNSUPPORTED),
     (dict(gather_max_density=1.5), _lib.MOE_ERR_INVALID),
     (dict(gemv_max_tokens=-2), _lib.MOE_ERR_INVALID),
+    (dict(out_f32=3), _lib.MOE_ERR_INVALID),
 ])
 def test_bad_desc_rejected(lib, kw, code):
     d = good_desc(**kw)

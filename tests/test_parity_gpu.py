@@ -153,6 +153,30 @@ def test_tau_infinity_leaves_shared_only(small_shared):
     _check(layer, small_shared, x, math.inf, ts, "bf16")
 
 
+@pytest.mark.parametrize("T", [3, 37])
+@pytest.mark.parametrize("path", ["auto", "dense"])
+def test_nan_token_routes_to_valid_experts(small, T, path):
+    """A token whose x row is NaN gets the experts 0..k-1 (NaN logits rank as
+    -inf and an expert is chosen once), and every other token's routing,
+    active set and output match the oracle run without that token."""
+    bad = 1
+    x = make_tokens(SMALL.d_model, T, 23, "bf16")
+    tau, _ = _calibrated(small, x, 0.7)
+    xn = x.clone()
+    xn[bad] = float("nan")
+    layer = make_layer(SMALL, 64, path=path)
+    gpu = run_gpu(layer, small, xn, tau)
+    assert gpu["topk_idx"][bad].tolist() == list(range(SMALL.top_k))
+    keep = [t for t in range(T) if t != bad]
+    k = SMALL.top_k
+    pairs = [t * k + i for t in keep for i in range(k)]
+    sub = {"out": gpu["out"][keep], "topk_idx": gpu["topk_idx"][keep],
+           "topk_w": gpu["topk_w"][keep], "active_bits": gpu["active_bits"][pairs]}
+    ref = oracle_forward(small, x[keep], tau, dense=(path == "dense"))
+    compare(sub, ref, tau, 0.0, "bf16", dw=small, dense=(path == "dense"))
+    assert layer.status() == 0
+
+
 def test_empty_batch_is_a_noop(small):
     layer = make_layer(SMALL, 16)
     out = torch.full((0, SMALL.d_model), 7.0, dtype=torch.bfloat16, device="cuda")

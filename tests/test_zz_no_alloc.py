@@ -1,16 +1,15 @@
 """The allocation-free routing entry point (moe_sparse_route_noalloc).
 
-Some callers cannot call cudaMalloc: code that runs while a CUDA graph is
-being captured, plug-ins that live inside another framework's fixed memory
-plan, serving loops that reserve all device memory up front. For them the
+Some callers cannot call cudaMalloc: plug-ins that live inside another
+framework's fixed memory plan, and serving loops that reserve all device
+memory up front and treat any later allocation as a failure. For them the
 library offers the router step with its scratch in a fixed device array.
-This test calls it through the C ABI twice in a row and checks its routing
+The GPU tests call it through the C ABI twice in a row and check its routing
 against the routing that moe_sparse_forward reports for the same inputs,
-plus the validity of the grouping it returns. The file is named so that
-pytest collects it last.
+plus the validity of the grouping it returns; the CPU tests check that bad
+arguments are refused before any CUDA call. The file is named so that pytest
+collects it last.
 """
-
-import ctypes
 
 import numpy as np
 import pytest
@@ -18,8 +17,6 @@ import torch
 
 from moe_inputs import LayerShape, make_tokens, make_weights
 from intra_expert_activation_b200 import MoESparseLayer, _lib
-
-pytestmark = pytest.mark.gpu
 
 CASES = [
     (LayerShape(d_model=512, n_experts=8, top_k=2, d_ff=256, renormalize=True, dtype="bf16",
@@ -48,6 +45,7 @@ def _route_noalloc(lib, x, Wr, bias, sh, T):
     return [t.cpu().numpy() for t in (idx, w, off, slot, perm)]
 
 
+@pytest.mark.gpu
 @pytest.mark.parametrize("sh,T,seed", CASES)
 def test_route_noalloc_matches_forward_routing(sh, T, seed):
     if not torch.cuda.is_available():
@@ -85,14 +83,80 @@ def test_route_noalloc_matches_forward_routing(sh, T, seed):
         assert np.array_equal(a, b)
 
 
-def test_route_noalloc_rejects_oversized_batches():
+@pytest.mark.gpu
+def test_route_noalloc_nan_rows_get_distinct_valid_experts():
+    """A token whose x row holds NaN (every logit NaN) or +inf gets k distinct
+    experts, the lowest ids, as NaN logits rank as -inf; the other tokens
+    route exactly as without it."""
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
     lib = _lib.load()
-    z = ctypes.c_void_p(0)
-    st = lib.moe_sparse_route_noalloc(None, 5000, 512, None, None, 8, 2, 1, _lib.MOE_BF16,
-                                      None, None, None, None, None, None)
-    assert st == _lib.MOE_ERR_UNSUPPORTED
-    assert b"4096" in lib.moe_sparse_last_error(None)
-    st = lib.moe_sparse_route_noalloc(None, 4, 512, None, None, 300, 2, 1, _lib.MOE_BF16,
-                                      None, None, None, None, None, None)
-    assert st == _lib.MOE_ERR_UNSUPPORTED
-    assert z.value is None
+    sh, T = CASES[1][0], 40
+    w = make_weights(sh, 34)
+    x = make_tokens(sh.d_model, T, 34, sh.dtype).cuda()
+    d = lambda t: None if t is None else t.cuda().contiguous()
+    clean = _route_noalloc(lib, x, d(w.W_router), d(w.router_bias), sh, T)
+    bad = x.clone()
+    bad[3] = float("nan")
+    bad[17, 5] = float("inf")
+    for _ in range(2):
+        idx, wt, off, slot, perm = _route_noalloc(lib, bad, d(w.W_router), d(w.router_bias),
+                                                  sh, T)
+        k, E = sh.top_k, sh.n_experts
+        assert (idx >= 0).all() and (idx < E).all()
+        for t in (3, 17):
+            assert len(set(idx[t].tolist())) == k
+        assert idx[3].tolist() == list(range(k))
+        rest = [t for t in range(T) if t not in (3, 17)]
+        assert np.array_equal(idx[rest], clean[0][rest])
+        assert np.array_equal(np.sort(slot), np.arange(T * k))
+        counts = np.bincount(idx.ravel(), minlength=E)
+        assert np.array_equal(off, np.concatenate([[0], np.cumsum(counts)]))
+
+
+def _call(lib, x, T, d, E, k, dtype, bufs):
+    return lib.moe_sparse_route_noalloc(x, T, d, bufs, None, E, k, 1, dtype, bufs, bufs, bufs,
+                                        bufs, bufs, None)
+
+
+@pytest.mark.parametrize("args,code,msg", [
+    # T, d_model, n_experts, top_k, dtype
+    ((5000, 512, 8, 2, "bf16"), "MOE_ERR_UNSUPPORTED", b"4096"),
+    ((4, 512, 300, 2, "bf16"), "MOE_ERR_UNSUPPORTED", b"n_experts"),
+    ((4, 512, 8, 0, "bf16"), "MOE_ERR_INVALID", b"top_k"),
+    ((4, 512, 8, 9, "bf16"), "MOE_ERR_INVALID", b"top_k"),
+    ((4, 512, 32, 17, "bf16"), "MOE_ERR_INVALID", b"top_k"),
+    ((4, 512, 8, 2, 7), "MOE_ERR_INVALID", b"dtype"),
+    ((4, 384, 8, 2, "bf16"), "MOE_ERR_UNSUPPORTED", b"multiple of 256"),
+    ((4, 192, 8, 2, "f32"), "MOE_ERR_UNSUPPORTED", b"multiple of 256"),
+    ((-1, 512, 8, 2, "bf16"), "MOE_ERR_INVALID", b"T < 0"),
+])
+def test_route_noalloc_rejects_bad_arguments(args, code, msg):
+    """Argument errors return before any CUDA call, with a message (CPU)."""
+    lib = _lib.load()
+    T, d, E, k, dt = args
+    dtype = {"bf16": _lib.MOE_BF16, "f32": _lib.MOE_F32}.get(dt, dt)
+    # non-NULL stand-ins: the checks return before anything is dereferenced
+    st = _call(lib, 0x1000, T, d, E, k, dtype, 0x2000)
+    assert st == getattr(_lib, code)
+    assert msg in lib.moe_sparse_last_error(None)
+
+
+def test_route_noalloc_rejects_null_and_misaligned_pointers():
+    lib = _lib.load()
+    st = lib.moe_sparse_route_noalloc(0x1000, 4, 512, 0x2000, None, 8, 2, 1, _lib.MOE_BF16,
+                                      0x3000, 0x4000, None, 0x5000, 0x6000, None)
+    assert st == _lib.MOE_ERR_INVALID
+    assert b"expert_offsets" in lib.moe_sparse_last_error(None)
+    st = lib.moe_sparse_route_noalloc(0x1000, 4, 512, 0x2000, None, 8, 2, 1, _lib.MOE_BF16,
+                                      None, 0x4000, 0x7000, 0x5000, 0x6000, None)
+    assert st == _lib.MOE_ERR_INVALID
+    assert b"NULL" in lib.moe_sparse_last_error(None)
+    st = lib.moe_sparse_route_noalloc(0x1008, 4, 512, 0x2000, None, 8, 2, 1, _lib.MOE_BF16,
+                                      0x3000, 0x4000, 0x7000, 0x5000, 0x6000, None)
+    assert st == _lib.MOE_ERR_INVALID
+    assert b"16-byte aligned" in lib.moe_sparse_last_error(None)
+    st = lib.moe_sparse_route_noalloc(0x1000, 4, 512, 0x2004, None, 8, 2, 1, _lib.MOE_F32,
+                                      0x3000, 0x4000, 0x7000, 0x5000, 0x6000, None)
+    assert st == _lib.MOE_ERR_INVALID
+    assert b"16-byte aligned" in lib.moe_sparse_last_error(None)
