@@ -82,6 +82,10 @@ def parse():
                     help="skip the end-to-end run with host buffers")
     ap.add_argument("--eager", action="store_true",
                     help="time eager API calls instead of replaying a captured CUDA graph")
+    ap.add_argument("--reps", type=int, default=50,
+                    help="graph replays timed one by one per latency point (median, p10, p90)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the sparsity sweep (Mixtral shape, sparse vs own dense path)")
     return ap.parse_args()
 
 
@@ -264,6 +268,106 @@ def run_reference(args, world, rank):
     return 0
 
 
+# ------------------------------------------------------------------ latency points
+
+def replay_stats(fwd, dev, warmup: int, reps: int) -> dict:
+    """Layer latency of one forward: a CUDA graph of `fwd` replayed `reps`
+    times, each replay between its own pair of CUDA events on the replaying
+    stream; median, p10 and p90 in microseconds."""
+    fwd()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        fwd()
+    torch.cuda.synchronize(dev)
+    for _ in range(warmup):
+        g.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    us = np.array([1e3 * a.elapsed_time(b) for a, b in ev])
+    del g
+    return {"median": round(float(np.median(us)), 2), "p10": round(float(np.percentile(us, 10)), 2),
+            "p90": round(float(np.percentile(us, 90)), 2), "reps": reps}
+
+
+SWEEP_POINTS = {  # (T, target sparsity) per score
+    "h": [(1, 0.0), (1, 0.5), (1, 0.7), (1, 0.9), (16, 0.0), (16, 0.5), (16, 0.7), (16, 0.9),
+          (128, 0.0), (128, 0.9), (512, 0.0), (512, 0.9)],
+    "gate": [(1, 0.0), (1, 0.5), (1, 0.7), (1, 0.9), (16, 0.0), (16, 0.5), (16, 0.7), (16, 0.9)],
+}
+
+
+def run_sweep(dev, local, warmup: int, reps: int, w_host=None) -> dict:
+    """Sparsity sweep on the Mixtral-shaped layer (d_model 4096, 8 experts
+    top-2, d_ff 14336, bf16, weights seed 4): tau calibrated on the 512-token
+    batch at each target sparsity, the smaller batches its prefixes. Every
+    point is the graph-replayed layer latency of the sparse path against the
+    library's own dense path (same kernels, no threshold, every row) at the
+    same T, for the |h| score and for the gate score."""
+    from intra_expert_activation_b200 import MoESparseLayer
+    wl = WORKLOADS["mixtral_sweep"]
+    sh = wl.shape
+    w_host = w_host or make_weights(sh, wl.weight_seed)
+    W = {k: getattr(w_host, k).to(dev).contiguous() for k in ("W_router", "W_gate", "W_up",
+                                                              "W_down")}
+    xs = {T: make_tokens(sh.d_model, T, wl.token_seed, sh.dtype).to(dev)
+          for T in sorted({T for pts in SWEEP_POINTS.values() for T, _ in pts})}
+
+    def point(T, path, score, tau):
+        L = MoESparseLayer(sh.d_model, sh.d_ff, sh.n_experts, sh.top_k, T,
+                           renormalize=sh.renormalize, dtype=sh.dtype, path=path, device=local,
+                           score=score)
+        out = torch.empty((T, sh.d_model), dtype=torch.bfloat16, device=dev)
+
+        def fwd():
+            L.forward(xs[T], W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau,
+                      sh.top_k, out=out)
+        lat = replay_stats(fwd, dev, warmup, reps)
+        fwd()
+        st = L.stats()
+        assert L.status() == 0, "device status word set"
+        L.close()
+        return lat, st
+
+    dense = {}
+    for T in xs:
+        lat, st = point(T, "dense", "h", 0.0)
+        dense[T] = {"us": lat, "rows": st["down_rows_read"]}
+    points = []
+    for score, pts in SWEEP_POINTS.items():
+        for T, q in pts:
+            tau, _, calib = load_tau("mixtral_sweep", q, score)
+            lat, st = point(T, "auto", score, tau)
+            meas = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
+            points.append({
+                "score": score, "T": T, "target_sparsity": q, "sparsity": round(meas, 4),
+                "tau": tau, "us": lat, "dense_us": dense[T]["us"],
+                "speedup": round(dense[T]["us"]["median"] / lat["median"], 3),
+                "down_rows_read": st["down_rows_read"], "up_rows_read": st["up_rows_read"],
+                "gate_up_rows_read": st["gate_up_rows_read"],
+                "down_rows_dense": dense[T]["rows"],
+                "groups": {"gemv": st["n_groups_gemv"], "tc_allrows": st["n_groups_tc_allrows"],
+                           "tc_gather": st["n_groups_tc_gather"]},
+            })
+    summary = {}
+    for score in SWEEP_POINTS:
+        for T in (1, 16):
+            row = [p for p in points if p["score"] == score and p["T"] == T]
+            summary[f"{score}_T{T}"] = {f"{p['target_sparsity']:.1f}": p["speedup"] for p in row}
+    return {"workload": "mixtral_sweep", "reps": reps, "speedup_vs_dense": summary, "points": points,
+            "timing": "graph replays, each between its own CUDA events; median/p10/p90 us; "
+                      "touched expert weights exceed L2 (no flush)"}
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_ours(args, world, rank, local):
@@ -346,31 +450,25 @@ def run_ours(args, world, rank, local):
         return per
 
     def per_batch_us(L):
-        """Layer latency per decode batch: K replays of a graph of one forward."""
+        """Layer latency per decode batch: --reps replays of a graph of one
+        forward, each timed between its own events (median, p10, p90)."""
         res = []
         for x, o in zip(xs, outs):
-            def one():
+            def one(x=x, o=o):
                 L.forward(x, W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau,
                           sh.top_k, router_bias=W["router_bias"], out=o)
-            one()
-            torch.cuda.synchronize(dev)
-            side = torch.cuda.Stream(dev)
-            side.wait_stream(stream)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=side):
-                one()
-            for _ in range(args.warmup):
-                g.replay()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize(dev)
-            a.record(stream)
-            for _ in range(args.steps):
-                g.replay()
-            b.record(stream)
-            torch.cuda.synchronize(dev)
-            res.append(1e3 * a.elapsed_time(b) / args.steps)
-            del g
+            res.append(replay_stats(one, dev, args.warmup, args.reps))
         return res
+
+    sweep_w = {}
+    sweep_on = (not args.no_sweep and world == 1 and args.workload == "mixtral_decode"
+                and args.score == "h" and not args.tokens)
+    if sweep_on:  # the sweep's weights are drawn on the host while the GPU works
+        def gen():
+            sweep_w["w"] = make_weights(WORKLOADS["mixtral_sweep"].shape,
+                                        WORKLOADS["mixtral_sweep"].weight_seed)
+        sweep_thread = threading.Thread(target=gen, daemon=True)
+        sweep_thread.start()
 
     sparse = make("auto")
     for _ in range(args.warmup):
@@ -424,7 +522,7 @@ def run_ours(args, world, rank, local):
 
     per_T = []
     gate_bytes_tot = gate_ms_tot = down_bytes_tot = down_ms_tot = 0.0
-    up_bytes_tot = up_ms_tot = gate_flops_tot = 0.0
+    up_bytes_tot = up_ms_tot = gate_flops_tot = gemv_bytes_tot = gemv_ms_tot = 0.0
     for i, T in enumerate(tokens):
         st = stats[i]
         P = T * sh.top_k
@@ -437,20 +535,31 @@ def run_ours(args, world, rank, local):
                 + P * sh.d_ff * esize
             if sh.n_shared:
                 g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
-        d_bytes = st["down_rows_read"] * sh.d_model * esize
-        u_bytes = st["up_rows_read"] * sh.d_model * esize
+        rb = sh.d_model * esize
+        u_bytes = st["up_rows_read"] * rb
         u_ms = avg_stage(per_fwd, i, "updown_gemv")  # gate score: fused sparse up + down
         up_bytes_tot += u_bytes * args.steps
         up_ms_tot += u_ms * args.steps
         g_ms = avg_stage(per_fwd, i, "gate_up")
-        d_ms = avg_stage(per_fwd, i, "down_gemv") + avg_stage(per_fwd, i, "down_tc") \
-            + avg_stage(per_fwd, i, "updown_gemv")
+        # the down kernels, each counted only when it had rows to stream (a launch
+        # that finds no group of its kind is not down-projection work): the row
+        # stream (GEMV; with the gate score the fused kernel, which reads each
+        # union row of W_up and of W_down) and the tensor-core path
+        gemv_rows = st["down_rows_gemv"]
+        tc_rows = st["down_rows_read"] - gemv_rows
+        gemv_ms = avg_stage(per_fwd, i, "updown_gemv" if args.score == "gate" else "down_gemv")
+        gemv_bytes = gemv_rows * rb * (2 if args.score == "gate" else 1)
+        tc_ms = avg_stage(per_fwd, i, "down_tc")
+        tc_bytes = tc_rows * rb
+        d_ms = (gemv_ms if gemv_rows else 0.0) + (tc_ms if tc_rows else 0.0)
+        d_bytes = (gemv_bytes if gemv_rows else 0) + (tc_bytes if tc_rows else 0)
+        if gemv_rows:
+            gemv_bytes_tot += gemv_bytes * args.steps
+            gemv_ms_tot += gemv_ms * args.steps
         fwd_ms = sum(avg_stage(per_fwd, i, s) for s in per_fwd[0]) if per_fwd else 0.0
         fwd_dense = sum(avg_stage(per_dense, i, s) for s in per_dense[0]) if per_dense else None
         d_dense = (avg_stage(per_dense, i, "down_gemv") + avg_stage(per_dense, i, "down_tc")) \
             if per_dense else None
-        if args.score == "gate":  # the fused kernel streams W_up and W_down rows
-            d_bytes += u_bytes
         # gate/up flops: 2 matrices (1 for gate-only rows) x 2 x tokens x d per loaded row
         g_flops = 2.0 * sh.d_model * (P * sh.d_ff * (1 if args.score == "gate" and
                                                       st["n_groups_tc_allrows"] == 0 else 2)
@@ -464,10 +573,14 @@ def run_ours(args, world, rank, local):
         sp = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
         per_T.append({
             "T": T, "sparsity": round(sp, 4), "experts_touched": touched,
-            "layer_us_graph": round(lat_sparse[i], 2),
-            "dense_layer_us_graph": None if lat_dense[i] is None else round(lat_dense[i], 2),
+            "layer_us_graph": lat_sparse[i]["median"],
+            "layer_us_graph_p10_p90": [lat_sparse[i]["p10"], lat_sparse[i]["p90"]],
+            "dense_layer_us_graph": None if lat_dense[i] is None else lat_dense[i]["median"],
+            "dense_layer_us_graph_p10_p90": None if lat_dense[i] is None else
+            [lat_dense[i]["p10"], lat_dense[i]["p90"]],
             "speedup_vs_dense_graph": None if lat_dense[i] is None else
-            round(lat_dense[i] / lat_sparse[i], 3),
+            round(lat_dense[i]["median"] / lat_sparse[i]["median"], 3),
+            "down_rows_gemv": gemv_rows,
             "down_rows_read": st["down_rows_read"],
             "down_rows_dense": touched * sh.d_ff,
             "up_rows_read": st["up_rows_read"],
@@ -481,6 +594,9 @@ def run_ours(args, world, rank, local):
             "speedup_vs_dense": None if not fwd_dense else round(fwd_dense / fwd_ms, 3),
             "gate_up_GBps": round(g_bytes / (g_ms * 1e-3) / 1e9, 1) if g_ms else None,
             "down_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1) if d_ms else None,
+            "down_gemv_GBps": round(gemv_bytes / (gemv_ms * 1e-3) / 1e9, 1)
+            if gemv_rows and gemv_ms else None,
+            "down_tc_GBps": round(tc_bytes / (tc_ms * 1e-3) / 1e9, 1) if tc_rows and tc_ms else None,
             # the fused kernel reads each active row of W_up and of W_down once
             "updown_GBps": round(2 * u_bytes / (u_ms * 1e-3) / 1e9, 1) if u_ms else None,
             "dense_down_us": None if d_dense is None else round(1e3 * d_dense, 2),
@@ -493,6 +609,7 @@ def run_ours(args, world, rank, local):
     g_traffic = None if not traffic_ok or args.score != "h" else \
         round(GATE_UP_TRAFFIC["ratio"] * gate_bytes_tot / n_gate_launches)
     d_ach = down_bytes_tot / (down_ms_tot * 1e-3) / 1e9 if down_ms_tot else 0.0
+    gv_ach = gemv_bytes_tot / (gemv_ms_tot * 1e-3) / 1e9 if gemv_ms_tot else 0.0
     # the gate/up kernel is HBM-bound below the ridge (decode, few tokens per
     # expert) and tensor-bound above it (prefill): grade it on its own bound
     tpeak, tpeak_kind = tensor_peak()
@@ -553,6 +670,11 @@ def run_ours(args, world, rank, local):
                "sample": f"one step: decode batches T={tokens} of {args.workload} through the "
                          f"fp64 numpy oracle on {cores} host threads ({t:.1f} s)"}
 
+    sweep = None
+    if sweep_on:
+        sweep_thread.join()
+        sweep = run_sweep(dev, local, args.warmup, args.reps, sweep_w.get("w"))
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -565,6 +687,12 @@ def run_ours(args, world, rank, local):
                               "bound": "hbm",
                               "achieved": round(d_ach, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(d_ach / peak, 4), "peak_kind": peak_kind},
+            "roofline_down_gemv": None if not gemv_ms_tot else
+            {"kernel": "updown_gemv" if args.score == "gate" else "down_gemv",
+             "bound": "hbm", "achieved": round(gv_ach, 1), "peak": peak, "unit": "GB/s",
+             "frac": round(gv_ach / peak, 4), "peak_kind": peak_kind,
+             "bytes": "union rows streamed by the row stream (W_up and W_down rows with the "
+                      "gate score), batches where it had rows"},
             "roofline_updown": None if args.score != "gate" else
             {"kernel": "updown_gemv (gate score: W_up + W_down rows actually read)",
              "bound": "hbm", "achieved": round(2 * u_ach, 1), "peak": peak, "unit": "GB/s",
@@ -579,6 +707,7 @@ def run_ours(args, world, rank, local):
             "launch": "eager" if args.eager else "cuda_graph",
             "kernel_times": "second timed pass of the same steps with per-stage CUDA events",
             "clocks": clk,
+            "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     del g_sparse

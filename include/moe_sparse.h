@@ -143,6 +143,8 @@ typedef struct {
   int64_t n_experts_touched;  /* routed experts with at least one token */
   int64_t up_rows_read;       /* W_up rows streamed by the sparse up projection (gate score) */
   int64_t gate_up_rows_read;  /* W_gate + W_up rows loaded by the gate/up projection */
+  int64_t down_rows_gemv;     /* of down_rows_read, the rows streamed by the row-stream (GEMV)
+                                 kernel, once per pass of up to 8 tokens */
 } moe_stats;
 
 typedef struct moe_sparse_ctx moe_sparse_ctx;

@@ -61,7 +61,7 @@ class moe_stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "n_routed_h", "n_routed_active", "n_shared_h", "n_shared_active", "down_rows_read",
         "n_groups", "n_groups_gemv", "n_groups_tc_gather", "n_groups_tc_allrows",
-        "n_experts_touched", "up_rows_read", "gate_up_rows_read")]
+        "n_experts_touched", "up_rows_read", "gate_up_rows_read", "down_rows_gemv")]
 
 
 _vp = ctypes.c_void_p
@@ -90,6 +90,11 @@ SIGNATURES = {
     "moe_sparse_destroy": (ctypes.c_int, [_vp]),
 }
 
+# include/moe_sparse_check.h: exported by the bounds-checked build only
+CHECK_SIGNATURES = {
+    "moe_sparse_check_wait_timeout": (ctypes.c_int, [_vp, ctypes.c_uint32, _i32, _vp]),
+}
+
 _LIB = None
 
 
@@ -106,6 +111,11 @@ def load() -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+        for name, (res, args) in CHECK_SIGNATURES.items():  # checked build only
+            if hasattr(lib, name):
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
         _LIB = lib
     return _LIB
 

@@ -155,7 +155,39 @@ __global__ void debug_gather_kernel(Dims dm, Workspace ws, int32_t* topk_idx, fl
   }
 }
 
+#if MOE_CHECK
+// Checked build only: exercises the kernels' bounded waits with an arrival
+// that never comes. which = 0: an mbarrier that expects one arrival, waited
+// on by warp 0 through warp_wait; which = 1: a flag in global memory that
+// nothing sets, waited on through wait_flag. Either wait gives up after
+// `limit` probes, records MOE_ERR_DEVICE_TIMEOUT in the status word and the
+// kernel returns.
+__device__ int g_flag_never_set = 0;
+__global__ void wait_timeout_kernel(int* status, uint32_t limit, int which) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (which == 0) {
+    if (threadIdx.x < 32) warp_wait(&bar, 0, &abort_flag, status, 0, limit);
+  } else if (threadIdx.x == 0) {
+    wait_flag(&g_flag_never_set, &abort_flag, status, limit);
+  }
+}
+#endif
+
 }  // namespace
+
+#if MOE_CHECK
+cudaError_t launch_wait_timeout(int* status, uint32_t limit, int which, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 64, 0, st>>>(status, limit, which);
+  return cudaGetLastError();
+}
+#endif
 
 cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st) {
   return launch_k(union_scan_kernel, dm.groups_max, kScanThreads, 0, st, dm, ws);

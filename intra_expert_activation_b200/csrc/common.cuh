@@ -80,17 +80,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Gives up after
-// about a second: sets *abort, records MOE_ERR_DEVICE_TIMEOUT and returns
-// false, so that no kernel can hang the GPU on a lost arrival.
+// about a second (limit probes; the kernels keep the default, the checked
+// build's timeout test passes a small one): sets *abort, records
+// MOE_ERR_DEVICE_TIMEOUT and returns false, so that no kernel can hang the
+// GPU on a lost arrival.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status, int tight = 0) {
+                                          int* status, int tight = 0,
+                                          uint32_t limit = kSpinLimit) {
   // optionally first a tight run of probes (each may suspend the thread
   // briefly in hardware), for waits that are short and on the critical path;
   // then probes with growing sleeps up to the limit
   for (int i = 0; i < tight; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     __nanosleep(i < 64 ? 20 : 200);
@@ -103,10 +106,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // One lane of the warp waits; the outcome is broadcast, so the warp never
 // diverges around a later __syncwarp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status, int tight = 0) {
+                                          int* status, int tight = 0,
+                                          uint32_t limit = kSpinLimit) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, tight) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, tight, limit) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Bounded wait for another CTA's release flag (acquire), at most limit
+// probes (about a second by default); on expiry as mbar_wait.
+__device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort, int* status,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v) return true;
+    if (*abort) return false;
+    __nanosleep(i < 64 ? 20 : 200);
+  }
+  *abort = 1;
+  report_error(status, kErrDeviceTimeout);
+  return false;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -205,20 +205,6 @@ __device__ __forceinline__ void epi_finish(const GateUpTcParams& p, const UnitIn
   }
 }
 
-// Bounded wait for another CTA's release flag (acquire).
-__device__ bool wait_flag(const int* f, volatile int* abort, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
-    if (v) return true;
-    if (*abort) return false;
-    __nanosleep(i < 64 ? 20 : 200);
-  }
-  *abort = 1;
-  report_error(status, kErrDeviceTimeout);
-  return false;
-}
-
 // The four epilogue warps only (named barrier 1).
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 

@@ -81,7 +81,7 @@ enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUse
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
                kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
-               kCntUpRows = 8, kCntGateUpRows = 9, kCntWords = 10 };
+               kCntUpRows = 8, kCntGateUpRows = 9, kCntGemvRows = 10, kCntWords = 11 };
 
 // kPathCand: GEMV or all-rows TC, chosen after gate/up (cand_takes_gemv)
 enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3, kPathCand = 4 };
@@ -239,6 +239,11 @@ cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStr
 size_t down_tc_smem_bytes(int b_bytes, int stages);
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
                            cudaStream_t st);
+#if defined(MOE_CHECK) && MOE_CHECK
+// Checked build: a one-CTA kernel whose bounded wait (0: mbarrier, 1: global
+// flag) never completes and gives up after `limit` probes.
+cudaError_t launch_wait_timeout(int* status, uint32_t limit, int which, cudaStream_t st);
+#endif
 cudaError_t launch_debug_gather(const Dims& dm, const Workspace& ws, int32_t* topk_idx,
                                 float* topk_w, uint32_t* bits, uint32_t* bits_shared,
                                 cudaStream_t st);

@@ -16,6 +16,9 @@
 
 #include "kernels.h"
 #include "moe_sparse.h"
+#if defined(MOE_CHECK) && MOE_CHECK
+#include "moe_sparse_check.h"
+#endif
 
 using moe::Dims;
 using moe::Workspace;
@@ -721,6 +724,7 @@ moe_status moe_sparse_get_stats(moe_sparse_ctx* c, moe_stats* s, void* stream) {
   s->n_experts_touched = meta[moe::kMetaExpertsTouched];
   s->up_rows_read = (int64_t)cnt[moe::kCntUpRows];
   s->gate_up_rows_read = (int64_t)cnt[moe::kCntGateUpRows];
+  s->down_rows_gemv = (int64_t)cnt[moe::kCntGemvRows];
   return MOE_OK;
 }
 
@@ -812,6 +816,21 @@ const char* moe_sparse_stage_name(int32_t i) {
 const char* moe_sparse_last_error(const moe_sparse_ctx* c) {
   return c ? c->err.c_str() : g_init_error.c_str();
 }
+
+#if defined(MOE_CHECK) && MOE_CHECK
+moe_status moe_sparse_check_wait_timeout(moe_sparse_ctx* c, uint32_t limit, int32_t which,
+                                         void* stream) {
+  if (!c) return MOE_ERR_INVALID;
+  if (which != 0 && which != 1) return fail(c, MOE_ERR_INVALID, "which must be 0 or 1");
+  if (limit < 1 || limit > moe::kSpinLimit)
+    return fail(c, MOE_ERR_INVALID, "limit must be in 1..kSpinLimit");
+  DeviceGuard dg(c->desc.device);
+  const cudaError_t e =
+      moe::launch_wait_timeout(c->ws.status, limit, which, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "wait_timeout launch");
+  return MOE_OK;
+}
+#endif
 
 moe_status moe_sparse_destroy(moe_sparse_ctx* c) {
   if (!c) return MOE_OK;

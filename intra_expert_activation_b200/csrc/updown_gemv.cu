@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     atomicAdd(ws.counters + kCntUpRows, static_cast<unsigned long long>(start.rows));
     atomicAdd(ws.counters + kCntDownRows, static_cast<unsigned long long>(start.rows));
+    atomicAdd(ws.counters + kCntGemvRows, static_cast<unsigned long long>(start.rows));
   }
   __syncthreads();
   const uint32_t smem_s = smem_u32(smem);

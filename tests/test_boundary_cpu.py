@@ -12,6 +12,7 @@ from intra_expert_activation_b200 import _lib
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moe_sparse.h")
+CHECK_HEADER = os.path.join(ROOT, "include", "moe_sparse_check.h")
 
 
 @pytest.fixture(scope="module")
@@ -22,8 +23,8 @@ def lib():
     return _lib.load()
 
 
-def declared_functions():
-    src = open(HEADER).read()
+def declared_functions(header=HEADER):
+    src = open(header).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(moe_sparse_\w+)\s*\(", src)))
 
@@ -53,7 +54,7 @@ def test_only_the_abi_is_exported():
 
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(_lib.moe_sparse_desc) == 16 * 4
-    assert ctypes.sizeof(_lib.moe_stats) == 12 * 8
+    assert ctypes.sizeof(_lib.moe_stats) == 13 * 8
 
 
 def test_valid_desc_accepted(lib):
@@ -172,7 +173,10 @@ def test_checked_build_exports_the_same_abi():
     assert path.endswith("libmoe_sparse_check.so") and os.path.exists(path)
     out = os.popen(f"nm -D --defined-only {path}").read()
     syms = {l.split()[-1] for l in out.splitlines() if " T " in l}
-    assert {s for s in syms if s.startswith("moe_")} == set(declared_functions())
+    # the ABI plus the checked build's test hook (include/moe_sparse_check.h)
+    check_only = set(declared_functions(CHECK_HEADER))
+    assert check_only == set(_lib.CHECK_SIGNATURES)
+    assert {s for s in syms if s.startswith("moe_")} == set(declared_functions()) | check_only
     r = subprocess.run([sys.executable, "-c",
                         "from intra_expert_activation_b200 import _lib; print(_lib.LIB_PATH)"],
                        capture_output=True, text=True, cwd=ROOT,
