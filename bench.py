@@ -460,15 +460,8 @@ def run_ours(args, world, rank, local):
             res.append(replay_stats(one, dev, args.warmup, args.reps))
         return res
 
-    sweep_w = {}
     sweep_on = (not args.no_sweep and world == 1 and args.workload == "mixtral_decode"
                 and args.score == "h" and not args.tokens)
-    if sweep_on:  # the sweep's weights are drawn on the host while the GPU works
-        def gen():
-            sweep_w["w"] = make_weights(WORKLOADS["mixtral_sweep"].shape,
-                                        WORKLOADS["mixtral_sweep"].weight_seed)
-        sweep_thread = threading.Thread(target=gen, daemon=True)
-        sweep_thread.start()
 
     sparse = make("auto")
     for _ in range(args.warmup):
@@ -671,9 +664,8 @@ def run_ours(args, world, rank, local):
                          f"fp64 numpy oracle on {cores} host threads ({t:.1f} s)"}
 
     sweep = None
-    if sweep_on:
-        sweep_thread.join()
-        sweep = run_sweep(dev, local, args.warmup, args.reps, sweep_w.get("w"))
+    if sweep_on:  # after every headline pass: its weights are drawn on the host now
+        sweep = run_sweep(dev, local, args.warmup, args.reps)
 
     if rank == 0:
         line = {

@@ -40,9 +40,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
-// Wait until the previous kernel on the stream has completed and its memory
-// is visible (no-op when the launch had no programmatic dependency).
+// First let the next kernel on the stream launch its CTAs (they take only the
+// resources this grid leaves free, and wait in their own grid_dep_wait until
+// this grid has completed), then wait until the previous kernel on the stream
+// has completed and its memory is visible (no-op when the launch had no
+// programmatic dependency). Every CTA calls it before it exits, so a grid
+// completes only after its predecessor has.
 __device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 

@@ -12,10 +12,10 @@
 namespace moe {
 
 // Every kernel is launched with programmatic stream serialization: its CTAs
-// may be scheduled while the previous kernel on the stream drains, and they
-// call grid_dep_wait() (griddepcontrol.wait) before touching global memory,
-// so the launch latency overlaps the predecessor's tail. MOE_PDL=0 in the
-// environment turns it off.
+// may be scheduled as soon as every CTA of the previous kernel on the stream
+// has started (each signals it at its start), and they call grid_dep_wait()
+// (griddepcontrol.wait) before touching global memory, so the launch latency
+// overlaps the predecessor's run. MOE_PDL=0 in the environment turns it off.
 bool pdl_enabled();
 
 template <typename... KArgs, typename... Args>
