@@ -48,14 +48,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int MT = R::MT;
   constexpr int ES = static_cast<int>(sizeof(TW));
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ Start start;
-  __shared__ long long sm_warp[kThreads / 32];
+  __shared__ StartSmem ss;
+  const Start& start = ss.st;
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ uint16_t list[kListRows];
   __shared__ int abort_flag;
 
   grid_dep_wait();
-  find_start(dm, ws, MT, &start, sm_warp);
+  find_start(dm, ws, MT, ss);
   if (start.rows <= 0 || start.i < 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t ld = static_cast<size_t>(dm.slots_total);
     const char* ht = static_cast<const char*>(ws.ht);
     Walk k;
-    walk_begin(dm, ws, start, k, MT);
+    walk_begin(dm, ss, k, MT);
     int s = 0;  // stages filled
     bool ok = true;
     for (bool last = false; ok && !last;) {
