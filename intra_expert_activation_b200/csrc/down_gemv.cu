@@ -32,6 +32,12 @@
 // (zeroed by the router) with vector fp32 atomics: the partials of a unit are
 // summed in arrival order, so results agree to fp32 rounding, not bitwise,
 // between runs on this path.
+//
+// Direct combine (dm.direct_combine: every group of the forward is on this
+// path and T is small): the flush adds w x the sums of a slot straight into
+// its token's output accumulator row Y[token] (w: the slot's combine weight,
+// 1 for shared experts), and the last CTA to finish (a ticket) writes out
+// from those rows, so no combine kernel runs.
 #include "gemv_consumers.cuh"
 
 namespace moe {
@@ -40,10 +46,92 @@ namespace {
 
 constexpr int kStageExtra = kBatch * kHBytes + 16;   // per stage after the rows: h | meta
 
+// Direct combine: the output row and combine weight of slot s (routed: the
+// token the router placed there and its weight; shared: weight 1).
+__device__ __forceinline__ void slot_target(const Dims& dm, const Workspace& ws, int s, int& tok,
+                                            float& w) {
+  if (s < dm.slots_routed) {
+    tok = __ldcg(ws.perm + s);
+    w = __ldcg(ws.slot_w + s);
+  } else {
+    tok = (s - dm.slots_routed) % dm.T_pad;
+    w = 1.f;
+  }
+  if (!moe_in_bounds(ws.status, tok >= 0 && tok < dm.T)) tok = 0;  // checked build
+}
+
+// Where a consumer lane's sums of the current unit go under direct combine.
+template <typename TW>
+struct Direct;
+template <>
+struct Direct<__nv_bfloat16> {  // one token per lane (Rows::flush_token)
+  float* row;
+  float w;
+  bool on;
+  __device__ void load(const Dims& dm, const Workspace& ws, int slot, int mt, int col0, int lane) {
+    const int t = Rows<__nv_bfloat16>::flush_token(lane);
+    on = t < mt;
+    row = ws.y;
+    w = 0.f;
+    if (on) {
+      int tok;
+      slot_target(dm, ws, slot + t, tok, w);
+      row = ws.y + (size_t)tok * dm.d + col0;
+    }
+  }
+  __device__ void flush(Rows<__nv_bfloat16>& r, int, int lane) { r.flush_to(row, w, on, lane); }
+};
+template <>
+struct Direct<float> {  // every token of the pass per lane
+  static constexpr int MT = Rows<float>::MT;
+  float* row[MT];
+  float w[MT];
+  __device__ void load(const Dims& dm, const Workspace& ws, int slot, int mt, int col0, int) {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      row[t] = ws.y;
+      w[t] = 0.f;
+      if (t < mt) {
+        int tok;
+        slot_target(dm, ws, slot + t, tok, w[t]);
+        row[t] = ws.y + (size_t)tok * dm.d + col0;
+      }
+    }
+  }
+  __device__ void flush(Rows<float>& r, int mt, int lane) { r.flush_rows(row, w, mt, lane); }
+};
+
+// Direct combine, every thread of every CTA: after this CTA's sums are out,
+// take the ticket; the last CTA writes out[t][c] = Y[t][c] for t < T.
+__device__ void direct_finish(const Dims& dm, const Workspace& ws, void* out, int out_bf16) {
+  __shared__ int is_last;
+  __threadfence();  // this thread's sums are visible before the ticket
+  __syncthreads();
+  if (threadIdx.x == 0)
+    is_last = atomicAdd(ws.meta + kMetaDownDone, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int n4 = dm.T * dm.d / 4;
+  const float4* y4 = reinterpret_cast<const float4*>(ws.y);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = __ldcg(y4 + i);
+    if (out_bf16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&lo);
+      u.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(out)[i] = u;
+    } else {
+      reinterpret_cast<float4*>(out)[i] = v;
+    }
+  }
+}
+
 template <typename TW>
 __global__ void __launch_bounds__(kThreads, 1)
     down_gemv_kernel(Dims dm, Workspace ws, const TW* __restrict__ Wd,
-                     const TW* __restrict__ Wds) {
+                     const TW* __restrict__ Wds, void* out, int out_bf16) {
   using R = Rows<TW>;
   constexpr int MT = R::MT;
   constexpr int ES = static_cast<int>(sizeof(TW));
@@ -56,7 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   grid_dep_wait();
   find_start(dm, ws, MT, ss);
-  if (start.rows <= 0 || start.i < 0) return;
+  if (start.rows <= 0 || start.i < 0) {  // uniform
+    if (dm.direct_combine) direct_finish(dm, ws, out, out_bf16);
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int row_bytes = d * ES;
@@ -155,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ consumers
     R rows;
     rows.zero();
+    Direct<TW> dir;
     int cur_tag = -1, cur_slot = 0, cur_mt = 0, cur_col0 = 0;
     for (int s = 0;; ++s) {
       const int b = s % NS;
@@ -171,13 +263,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool mine = phase < n_phase && (s % n_phase) == phase;
       if (meta.x != cur_tag && (mine || meta.x < 0)) {
         if (cur_tag >= 0) {
-          rows.flush(ws.y + (size_t)cur_slot * d + cur_col0, d, cur_mt, lane);
+          if (dm.direct_combine)
+            dir.flush(rows, cur_mt, lane);
+          else
+            rows.flush(ws.y + (size_t)cur_slot * d + cur_col0, d, cur_mt, lane);
           rows.zero();
         }
         cur_tag = meta.x;
         cur_slot = meta.z;
         cur_mt = mt;
         cur_col0 = (cb * kBlockBytes + slice * kSliceBytes) / ES;
+        // the new unit's output rows and weights, loaded long before its flush
+        if (dm.direct_combine && cur_tag >= 0) dir.load(dm, ws, cur_slot, cur_mt, cur_col0, lane);
       }
       if (mine && meta.y > 0)
         rows.consume(smem_s + b * geo.stage + slice * kSliceBytes, stg + slice * kSliceBytes,
@@ -187,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (meta.x < 0) break;
     }
   }
+  if (dm.direct_combine) direct_finish(dm, ws, out, out_bf16);
 }
 
 }  // namespace
@@ -197,7 +295,8 @@ size_t down_gemv_smem_bytes(int d, bool bf16) {
 }
 
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
-                             const void* Wds, bool bf16, int n_sms, cudaStream_t st) {
+                             const void* Wds, bool bf16, int n_sms, void* out, bool out_bf16,
+                             cudaStream_t st) {
   const cudaError_t e = bf16 ? smem_limit(down_gemv_kernel<__nv_bfloat16>, kSmemBudget)
                              : smem_limit(down_gemv_kernel<float>, kSmemBudget);
   if (e != cudaSuccess) return e;
@@ -205,9 +304,11 @@ cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd
   const size_t smem = down_gemv_smem_bytes(dm.d, bf16);
   if (bf16)
     return launch_k(down_gemv_kernel<__nv_bfloat16>, grid, kThreads, smem, st, dm, ws,
-                    static_cast<const __nv_bfloat16*>(Wd), static_cast<const __nv_bfloat16*>(Wds));
+                    static_cast<const __nv_bfloat16*>(Wd), static_cast<const __nv_bfloat16*>(Wds),
+                    out, out_bf16 ? 1 : 0);
   return launch_k(down_gemv_kernel<float>, grid, kThreads, smem, st, dm, ws,
-                  static_cast<const float*>(Wd), static_cast<const float*>(Wds));
+                  static_cast<const float*>(Wd), static_cast<const float*>(Wds), out,
+                  out_bf16 ? 1 : 0);
 }
 
 }  // namespace moe

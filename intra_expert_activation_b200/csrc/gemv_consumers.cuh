@@ -72,21 +72,28 @@ struct Rows<__nv_bfloat16> {
   // into Y with 8-byte vector atomics (no shared-memory staging, so the ring
   // of stages gets that space).
   __device__ void flush(float* y, int d, int mt, int lane) {
-    const int g = lane >> 2, c2 = 2 * (lane & 3);
+    const int tok = 2 * (lane & 3) + ((lane >> 2) & 1);
+    flush_to(y + (size_t)tok * d, 1.f, tok < mt, lane);
+  }
+  // The token of this lane in the flush (its sums go to that token's row).
+  __device__ static int flush_token(int lane) { return 2 * (lane & 3) + ((lane >> 2) & 1); }
+  // Adds w x the sums of this lane's token (flush_token) into the row yrow
+  // (at the warp's first column); nothing when !on.
+  __device__ void flush_to(float* yrow, float w, bool on, int lane) {
+    const int g = lane >> 2;
     const bool odd = g & 1;
-    const int tok = c2 + odd;
-    float* yt = y + (size_t)tok * d + (g & ~1);
+    float* yt = yrow + (g & ~1);
 #pragma unroll
     for (int i = 0; i < kTiles; ++i) {
       const float s0 = odd ? acc[i][0] : acc[i][1];
       const float s1 = odd ? acc[i][2] : acc[i][3];
       const float r0 = __shfl_xor_sync(0xffffffffu, s0, 4);
       const float r1 = __shfl_xor_sync(0xffffffffu, s1, 4);
-      if (tok < mt) {
+      if (on) {
         const float2 a = odd ? make_float2(r0, acc[i][1]) : make_float2(acc[i][0], r0);
         const float2 b = odd ? make_float2(r1, acc[i][3]) : make_float2(acc[i][2], r1);
-        red_add_v2(yt + 16 * i, a.x, a.y);
-        red_add_v2(yt + 16 * i + 8, b.x, b.y);
+        red_add_v2(yt + 16 * i, w * a.x, w * a.y);
+        red_add_v2(yt + 16 * i + 8, w * b.x, w * b.y);
       }
     }
   }
@@ -142,6 +149,17 @@ struct Rows<float> {
       if (t < mt) {
         const float2 a = unpack2(acc[t][0]), b = unpack2(acc[t][1]);
         red_add_v4(y + (size_t)t * d + lane * 4, a.x, a.y, b.x, b.y);
+      }
+    }
+  }
+  // Adds w[t] x the sums of token t into the row yrow[t] (at the warp's
+  // first column) for t < mt.
+  __device__ void flush_rows(float* const (&yrow)[MT], const float (&w)[MT], int mt, int lane) {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      if (t < mt) {
+        const float2 a = unpack2(acc[t][0]), b = unpack2(acc[t][1]);
+        red_add_v4(yrow[t] + lane * 4, w[t] * a.x, w[t] * a.y, w[t] * b.x, w[t] * b.y);
       }
     }
   }

@@ -76,7 +76,9 @@ __host__ __device__ inline bool cand_takes_gemv(int union_rows, int passes, int 
 
 // meta[] words written by the router's scan
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
-            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6, kMetaWords = 16 };
+            kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
+            kMetaDownDone = 7,  // row-stream CTAs finished (direct combine ticket)
+            kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
@@ -115,7 +117,14 @@ struct Dims {
   int score_gate;     // 1: active iff |SiLU(g)| > tau, sparse up projection for GEMV groups
   int tc_grid;        // CTAs of this forward's tensor-core down launch
   int tc_part_units;  // capacity of the tensor-core down part buffers (units), 0: none
+  // 1: every group of this forward is on the row stream (and T <= kDirectMax):
+  // the row stream adds w x its sums straight into the output accumulator
+  // rows Y[0..T) (zeroed by the router) and its last CTA writes out; no
+  // combine launch
+  int direct_combine;
 };
+
+constexpr int kDirectMax = 16;  // tokens up to which the row stream combines directly
 
 // K parts per tensor-core down unit (group, 128-column slice). A unit reads
 // all of its group's rows for its columns, and an SM streams at most about
@@ -175,6 +184,7 @@ struct Workspace {
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)
   int* tc_list;                 // [groups_max] groups on a tensor-core path (count in meta)
   int* y_zero;                  // [E+1] 1: expert's Y rows (last: shared experts') start at zero
+  float* slot_w;                // [slots_routed] combine weight of each routed slot
   int* sk_flags;                // [sk_ctas] gate/up: CTA c published its split-unit partial
   float* sk_part;               // [2 * sk_ctas][2][128][n_max] gate/up split-unit partial sums
   int* tc_ticket;               // [tc_part_units] parts of a TC down unit done (cleared by the router)
@@ -234,7 +244,8 @@ cudaError_t launch_gate_up_simt(const Dims& dm, const Workspace& ws, const float
                                 cudaStream_t st);
 cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st);
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
-                             const void* Wds, bool bf16, int n_sms, cudaStream_t st);
+                             const void* Wds, bool bf16, int n_sms, void* out, bool out_bf16,
+                             cudaStream_t st);
 cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st);
 size_t down_tc_smem_bytes(int b_bytes, int stages);
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,

@@ -153,7 +153,7 @@ struct Layout {
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero, bSkFlags, bSkPart,
+           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero, bSlotW, bSkFlags, bSkPart,
            bTcTicket, bTcPart, bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
@@ -250,6 +250,7 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
   sz[bYZero] = sizeof(int) * (c.E + 1);
+  sz[bSlotW] = sizeof(float) * c.slots_routed;
   // gate/up split units (bf16): one flag per CTA and two partial slots per CTA,
   // for up to 2 x 160 CTAs (2 per SM) when the groups hold <= 32 tokens, else 160
   {
@@ -442,6 +443,7 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
   w.y_zero = reinterpret_cast<int*>(b + o[bYZero]);
+  w.slot_w = reinterpret_cast<float*>(b + o[bSlotW]);
   w.sk_flags = reinterpret_cast<int*>(b + o[bSkFlags]);
   w.sk_part = reinterpret_cast<float*>(b + o[bSkPart]);
   w.tc_ticket = reinterpret_cast<int*>(b + o[bTcTicket]);
@@ -535,6 +537,10 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
                          std::min(T, moe::kGroupMax) <= cap.gemv_max);
   const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
+  // every group on the |h|-score row stream and a small batch: the row stream
+  // combines directly into the output (no combine launch)
+  const bool out_bf16 = c->bf16 && !c->desc.out_f32;
+  dm.direct_combine = need_gemv && !need_tc && !dm.score_gate && T <= moe::kDirectMax ? 1 : 0;
   // the tensor-core down launch's grid is fixed here: the router's layout
   // and the kernel both derive the units' K parts from it
   const int tc_ctas_per_sm = n_max <= 64 ? 2 : 1;
@@ -639,7 +645,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   }
   mark(5);
   if (need_gemv && !dm.score_gate) {
-    e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, st);
+    e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, out, out_bf16, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_gemv launch");
     stage_ran[5] = true;
   }
@@ -668,9 +674,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     stage_ran[6] = true;
   }
   mark(7);
-  e = moe::launch_combine(dm, c->ws, out, c->bf16 && !c->desc.out_f32, st);
-  if (e != cudaSuccess) return cuda_fail(c, e, "combine launch");
-  stage_ran[7] = true;
+  if (!dm.direct_combine) {
+    e = moe::launch_combine(dm, c->ws, out, out_bf16, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "combine launch");
+    stage_ran[7] = true;
+  }
   mark(8);
   int nl = 0;
   for (int i = 0; i < kStages; ++i) nl += stage_ran[i];

@@ -23,7 +23,8 @@
 // permute_kernel, one warp per pair: slot = expert_off[e] + base[cta][e] +
 //   rank, so slots are ordered by (token, choice) within each expert; it
 //   records perm / slot_of and copies the x row to X_perm[slot]; extra warps
-//   zero the padding slots.
+//   mark the padding slots in perm (their X_perm rows are never used: every
+//   kernel masks the columns of tokens past a group's count).
 #include "common.cuh"
 #include "topk.cuh"
 
@@ -325,7 +326,8 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     ws.counters[kCntRoutedH] = (unsigned long long)T * k * (unsigned long long)dm.F;
     ws.counters[kCntSharedH] =
         (unsigned long long)S * (unsigned long long)T * (unsigned long long)dm.Fs;
-    ws.meta[kMetaDone] = 0;  // ticket counter for the next forward
+    ws.meta[kMetaDone] = 0;      // ticket counter for the next forward
+    ws.meta[kMetaDownDone] = 0;  // the row stream's direct-combine ticket
   }
   __syncthreads();
   for (int x = tid; x <= E; x += blockDim.x) ws.expert_off[x] = poff[x];
@@ -369,16 +371,18 @@ __device__ __forceinline__ float row_dot(const TX* a, const TX* b, int d, int la
 
 // Top-k of one token's logits (one warp, topk_warp): the k largest, equal
 // logits to the lower expert index; softmax over all experts; weights
-// p / sum(p_sel) or p. Writes topk_idx / topk_w of token `tok` and the chosen
-// experts to sel[0..k).
+// p / sum(p_sel) or p. Writes topk_idx / topk_w of token `tok`, the chosen
+// experts to sel[0..k) and, if given, their weights to selw[0..k).
 __device__ __forceinline__ void topk_token(const Dims& dm, const Workspace& ws, const float* lgt,
-                                           int tok, int lane, int* sel) {
+                                           int tok, int lane, int* sel, float* selw = nullptr) {
   const int k = dm.k;
   const TopkResult r = topk_warp(lgt, dm.E, k, lane);
   if (lane < k) {
+    const float w = dm.renorm ? r.my_p / r.psum : r.my_p;
     ws.topk_idx[tok * k + lane] = r.my_e;
-    ws.topk_w[tok * k + lane] = dm.renorm ? r.my_p / r.psum : r.my_p;
+    ws.topk_w[tok * k + lane] = w;
     sel[lane] = r.my_e;
+    if (selw) selw[lane] = w;
   }
 }
 
@@ -587,29 +591,33 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
     if (lane == 0) {
       ws.perm[slot] = t;
       ws.slot_of[item] = slot;
+      ws.slot_w[slot] = __ldcg(ws.topk_w + item);
     }
     uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * dm.d);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * dm.d);
     copy_row(dst, src, nv, lane);
-    if (__ldcg(ws.y_zero + e)) {  // the GEMV path adds split partials into Y
+    if (!dm.direct_combine && __ldcg(ws.y_zero + e)) {  // the GEMV path adds split partials into Y
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)slot * dm.d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   } else if (item < P + E) {
+    // padding slots: marked in perm; their X_perm rows are left as they are
+    // (every kernel masks the columns of tokens past a group's count)
     const int e = item - P;
     const int s0 = __ldcg(ws.expert_off + e) + __ldcg(ws.expert_cnt + e);
     const int s1 = __ldcg(ws.expert_off + e + 1);
-    for (int s = s0; s < s1; ++s) {
-      if (lane == 0) ws.perm[s] = -1;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)s * dm.d);
-      for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-    }
+    for (int s = s0 + lane; s < s1; s += 32) ws.perm[s] = -1;
   } else if (item < P + E + dm.S * dm.T) {
-    if (!__ldcg(ws.y_zero + E)) return;
+    if (dm.direct_combine || !__ldcg(ws.y_zero + E)) return;
     const int q = item - P - E;
     const int sh = q / dm.T, t = q % dm.T;
     float4* yz =
         reinterpret_cast<float4*>(ws.y + (size_t)(dm.slots_routed + sh * dm.T_pad + t) * dm.d);
+    for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (dm.direct_combine && item < P + E + dm.S * dm.T + dm.T) {
+    // direct combine: the output accumulator rows Y[0..T) start at zero
+    const int t = item - P - E - dm.S * dm.T;
+    float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)t * dm.d);
     for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
@@ -627,6 +635,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __shared__ float lg[kSmallTokens][kMaxExperts + 1];
   __shared__ float lpart[4][kSmallTokens][kMaxExperts];  // split-d partial logits
   __shared__ int sel[kSmallTokens * 16];
+  __shared__ float selw[kSmallTokens * 16];
   __shared__ int slot_s[kSmallTokens * 16];
   __shared__ int cnt[kMaxExperts];
   __shared__ int poff[kMaxExperts + 1];
@@ -659,7 +668,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   }
   __syncthreads();
   for (int t = warp; t < T; t += kSmallWarps)
-    topk_token(dm, ws, lg[t], t, lane, sel + t * k);
+    topk_token(dm, ws, lg[t], t, lane, sel + t * k, selw + t * k);
   __syncthreads();
   // stable rank of pair p among earlier pairs of the same expert
   for (int p = tid; p < P; p += kSmallThreads) {
@@ -678,6 +687,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     slot_s[p] = slot;
     ws.perm[slot] = p / k;
     ws.slot_of[p] = slot;
+    ws.slot_w[slot] = selw[p];
   }
   __syncthreads();
   // copies: one warp per pair, then padding slots, then shared Y rows
@@ -688,19 +698,22 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * d);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(p / k) * d);
     copy_row(dst, src, nv, lane);
-    if (ws.y_zero[sel[p]]) {
+    if (!dm.direct_combine && ws.y_zero[sel[p]]) {
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)slot * d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  for (int e = warp; e < E; e += kSmallWarps) {
-    for (int sl = poff[e] + cnt[e]; sl < poff[e + 1]; ++sl) {
-      if (lane == 0) ws.perm[sl] = -1;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)sl * d);
-      for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+  if (dm.direct_combine) {  // the output accumulator rows Y[0..T) start at zero
+    for (int t = warp; t < T; t += kSmallWarps) {
+      float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)t * d);
+      for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  if (ws.y_zero[E]) {
+  // padding slots: marked in perm; their X_perm rows are left as they are
+  // (every kernel masks the columns of tokens past a group's count)
+  for (int e = warp; e < E; e += kSmallWarps)
+    for (int sl = poff[e] + cnt[e] + lane; sl < poff[e + 1]; sl += 32) ws.perm[sl] = -1;
+  if (!dm.direct_combine && ws.y_zero[E]) {
     for (int q = warp; q < dm.S * T; q += kSmallWarps) {
       const int sh = q / T, t = q % T;
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)(dm.slots_routed + sh * dm.T_pad + t) * d);
@@ -772,7 +785,7 @@ cudaError_t launch_route(const Dims& dm, const Workspace& ws, const void* x, con
 
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st) {
-  const int items = dm.T * dm.k + dm.E + dm.S * dm.T;
+  const int items = dm.T * dm.k + dm.E + dm.S * dm.T + (dm.direct_combine ? dm.T : 0);
   const int grid = (items + 7) / 8;
   const int tpc = route_tokens_per_cta(dm, bf16 ? 2 : 4);
   if (bf16)
