@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kThreads)
                               : Wu + static_cast<size_t>(gr.expert) * F_e * d;
     const float* X = shared ? x : xperm;
     const float th = shared ? tau_shared : tau;
-    const bool gate_only = dm.score_gate != 0;
+    const bool gate_only = dm.sparse_up != 0;
 
     for (int t = threadIdx.x; t < gr.m; t += kThreads) tok_bits[t] = 0u;
     if (threadIdx.x == 0) uni = 0u;
@@ -80,11 +80,12 @@ __global__ void __launch_bounds__(kThreads)
           gs += __shfl_xor_sync(0xffffffffu, gs, o);
           us += __shfl_xor_sync(0xffffffffu, us, o);
         }
-        // gate score: active iff |SiLU(g)| > tau, and the masked SiLU(g) is
-        // stored for the sparse up kernel (every fp32 group is on the GEMV path)
+        // gate score: active iff |SiLU(g)| > tau; with the sparse up
+        // projection the masked SiLU(g) is stored for the fused up + down
+        // kernel (every fp32 group is on the GEMV path), else the masked h
         const float sg = silu_f32(gs);
         const float h = gate_only ? sg : sg * us;
-        const bool act = dense || fabsf(gate_only ? sg : h) > th;
+        const bool act = dense || fabsf(dm.score_gate ? sg : h) > th;
         if (lane == 0) {
           ht[static_cast<size_t>(j) * ld + gr.slot0 + t] = act ? h : 0.f;
           if (act) atomicOr(&tok_bits[t], 1u << (j & 31));

@@ -77,7 +77,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, 
     ui.shared = 1;
   }
   ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
-  ui.gate_only = p.dm.score_gate && __ldcg(p.ws.group_path + g) == kPathGemv;
+  ui.gate_only = p.dm.sparse_up && __ldcg(p.ws.group_path + g) == kPathGemv;
   ui.F_e = ui.shared ? p.dm.Fs : p.dm.F;
   const int e_local = ui.shared ? ui.gr.expert - p.dm.E : ui.gr.expert;
   ui.wrow = e_local * ui.F_e + ui.nt * kNeuronTile;

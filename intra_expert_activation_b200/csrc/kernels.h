@@ -114,7 +114,10 @@ struct Dims {
   int no_tc;          // 1: no tensor-core down path (fp32 layers): every group on GEMV
   int n_sms;          // streaming multiprocessors of the device
   int sk_ctas;        // capacity of the gate/up split-unit flags (CTAs), 0: no split units
-  int score_gate;     // 1: active iff |SiLU(g)| > tau, sparse up projection for GEMV groups
+  int score_gate;     // 1: active iff |SiLU(g)| > tau
+  int sparse_up;      // 1 (gate score, tau > 0): GEMV groups compute the up projection only
+                      // for their active rows (gate-only GEMM, then the fused up + down
+                      // row stream); 0: the up projection is dense
   int tc_grid;        // CTAs of this forward's tensor-core down launch
   int tc_part_units;  // capacity of the tensor-core down part buffers (units), 0: none
   // 1: every group of this forward is on the row stream (and T <= kDirectMax):

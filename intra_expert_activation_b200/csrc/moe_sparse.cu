@@ -537,10 +537,15 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
                          std::min(T, moe::kGroupMax) <= cap.gemv_max);
   const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
+  // gate score: the GEMV groups' up projection is sparse (only the active
+  // rows) when the threshold can leave rows out; at tau <= 0 every neuron
+  // whose SiLU(g) is non-zero is active, so the dense up projection (gate and
+  // up in one GEMM) reads the same rows faster
+  dm.sparse_up = dm.score_gate && tau > 0.f ? 1 : 0;
   // every group on the |h|-score row stream and a small batch: the row stream
   // combines directly into the output (no combine launch)
   const bool out_bf16 = c->bf16 && !c->desc.out_f32;
-  dm.direct_combine = need_gemv && !need_tc && !dm.score_gate && T <= moe::kDirectMax ? 1 : 0;
+  dm.direct_combine = need_gemv && !need_tc && !dm.sparse_up && T <= moe::kDirectMax ? 1 : 0;
   // the tensor-core down launch's grid is fixed here: the router's layout
   // and the kernel both derive the units' K parts from it
   const int tc_ctas_per_sm = n_max <= 64 ? 2 : 1;
@@ -608,7 +613,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     // gate score: gate-only units take two K-blocks per stage; the second
     // activation region costs a stage of the pipeline when groups are larger
     // than 16 tokens (measured at T = 32: 303 -> 358 us), so only below that
-    p.b_blocks = dm.score_gate && n_max <= 16 ? 2 : 1;
+    p.b_blocks = dm.sparse_up && n_max <= 16 ? 2 : 1;
     const size_t stage_bytes = 32768 + (size_t)p.b_blocks * n_max * 128;
     p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
     const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages, p.b_blocks);
@@ -637,14 +642,14 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   }
   mark(4);
 
-  if (need_gemv && dm.score_gate) {  // GEMV groups: fused sparse up + down over the active rows
+  if (need_gemv && dm.sparse_up) {  // GEMV groups: fused sparse up + down over the active rows
     e = moe::launch_updown_gemv(dm, c->ws, W_up, c->Wus, W_down, c->Wds, x, c->bf16, c->n_sms,
                                 st);
     if (e != cudaSuccess) return cuda_fail(c, e, "updown_gemv launch");
     stage_ran[4] = true;
   }
   mark(5);
-  if (need_gemv && !dm.score_gate) {
+  if (need_gemv && !dm.sparse_up) {
     e = moe::launch_down_gemv(dm, c->ws, W_down, c->Wds, c->bf16, c->n_sms, out, out_bf16, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_gemv launch");
     stage_ran[5] = true;
