@@ -46,6 +46,19 @@ namespace {
 
 constexpr int kStageExtra = kBatch * kHBytes + 16;   // per stage after the rows: h | meta
 
+// Column blocks of this kernel. Wide (bf16 rows of a multiple of 1 KB,
+// d_model % 512 == 0): rows up to 8 KB (d_model <= 4096) come in one bulk
+// copy per row and each consumer warp owns a 1 KB slice (32 sixteen-column
+// tiles); whole-row copies stream faster than two 4 KB halves fetched apart.
+// Otherwise (fp32, and bf16 rows of an odd number of 512-byte slices): 4 KB
+// blocks and 512-byte slices.
+template <bool WIDE>
+struct Blocks {
+  static constexpr int kBlock = WIDE ? 8192 : kBlockBytes;
+  static constexpr int kSlice = WIDE ? 1024 : kSliceBytes;
+};
+__host__ __device__ inline bool wide_rows(int d, bool bf16) { return bf16 && d % 512 == 0; }
+
 // Direct combine: the output row and combine weight of slot s (routed: the
 // token the router placed there and its weight; shared: weight 1).
 __device__ __forceinline__ void slot_target(const Dims& dm, const Workspace& ws, int s, int& tok,
@@ -79,7 +92,10 @@ struct Direct<__nv_bfloat16> {  // one token per lane (Rows::flush_token)
       row = ws.y + (size_t)tok * dm.d + col0;
     }
   }
-  __device__ void flush(Rows<__nv_bfloat16>& r, int, int lane) { r.flush_to(row, w, on, lane); }
+  template <class R>
+  __device__ void flush(R& r, int, int lane) {
+    r.flush_to(row, w, on, lane);
+  }
 };
 template <>
 struct Direct<float> {  // every token of the pass per lane
@@ -98,7 +114,10 @@ struct Direct<float> {  // every token of the pass per lane
       }
     }
   }
-  __device__ void flush(Rows<float>& r, int mt, int lane) { r.flush_rows(row, w, mt, lane); }
+  template <class R>
+  __device__ void flush(R& r, int mt, int lane) {
+    r.flush_rows(row, w, mt, lane);
+  }
 };
 
 // Direct combine, every thread of every CTA: after this CTA's sums are out,
@@ -128,22 +147,23 @@ __device__ void direct_finish(const Dims& dm, const Workspace& ws, void* out, in
   }
 }
 
-template <typename TW>
+template <typename TW, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     down_gemv_kernel(Dims dm, Workspace ws, const TW* __restrict__ Wd,
                      const TW* __restrict__ Wds, void* out, int out_bf16) {
-  using R = Rows<TW>;
+  using B = Blocks<WIDE>;
+  using R = Rows<TW, B::kSlice / 32>;
   constexpr int MT = R::MT;
   constexpr int ES = static_cast<int>(sizeof(TW));
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ StartSmem ss;
-  const Start& start = ss.st;
+  __shared__ Start start;
+  __shared__ long long sm_warp[kThreads / 32];
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ uint16_t list[kListRows];
   __shared__ int abort_flag;
 
   grid_dep_wait();
-  find_start(dm, ws, MT, ss);
+  find_start(dm, ws, MT, &start, sm_warp);
   if (start.rows <= 0 || start.i < 0) {  // uniform
     if (dm.direct_combine) direct_finish(dm, ws, out, out_bf16);
     return;
@@ -151,9 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int row_bytes = d * ES;
-  const Geometry geo = geometry(row_bytes, kStageExtra);
+  const Geometry geo = geometry(row_bytes, kStageExtra, B::kBlock);
   const int NS = geo.n_stages;
-  const int n_blocks = (row_bytes + kBlockBytes - 1) / kBlockBytes;
+  const int n_blocks = (row_bytes + B::kBlock - 1) / B::kBlock;
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < NS; ++b) {
@@ -175,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t ld = static_cast<size_t>(dm.slots_total);
     const char* ht = static_cast<const char*>(ws.ht);
     Walk k;
-    walk_begin(dm, ss, k, MT);
+    walk_begin(dm, ws, start, k, MT);
     int s = 0;  // stages filled
     bool ok = true;
     for (bool last = false; ok && !last;) {
@@ -186,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TW* wexp = k.expert >= dm.E ? Wds + (size_t)(k.expert - dm.E) * dm.Fs * d
                                         : Wd + (size_t)k.expert * dm.F * d;
       for (int cb = 0; cb < (last ? 1 : n_blocks) && ok; ++cb) {
-        const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
+        const int cbytes = min(B::kBlock, row_bytes - cb * B::kBlock);
         for (int pos = 0; pos < n_list || (last && pos == 0); pos += kBatch) {
           const int b = s % NS;
           if (s >= NS && !warp_wait(empty + b, ((s / NS) + 1) & 1, &abort_flag, ws.status, kTight)) {
@@ -228,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cp_async16(hdst + 16, hsrc + 16);
               }
               bulk_load(stg_s + lane * geo.stride,
-                        wexp + (size_t)j * d + cb * (kBlockBytes / ES), cbytes,
+                        wexp + (size_t)j * d + cb * (B::kBlock / ES), cbytes,
                         smem_u32(full + b));
             }
             cp_async_arrive(smem_u32(full + b));
@@ -254,10 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* stg = smem + b * geo.stage;
       const int4 meta = *reinterpret_cast<const int4*>(stg + kBatch * geo.stride + kBatch * kHBytes);
       const int cb = meta.w >> 8, mt = meta.w & 255;
-      const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
+      const int cbytes = min(B::kBlock, row_bytes - cb * B::kBlock);
       // this warp's slice of the block; with narrow blocks several warps
       // share a slice and take alternate stages
-      const int n_slices = cbytes / kSliceBytes;
+      const int n_slices = cbytes / B::kSlice;
       const int n_phase = n_slices >= kConsumers ? 1 : kConsumers / n_slices;
       const int slice = warp % n_slices, phase = warp / n_slices;
       const bool mine = phase < n_phase && (s % n_phase) == phase;
@@ -272,12 +292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         cur_tag = meta.x;
         cur_slot = meta.z;
         cur_mt = mt;
-        cur_col0 = (cb * kBlockBytes + slice * kSliceBytes) / ES;
+        cur_col0 = (cb * B::kBlock + slice * B::kSlice) / ES;
         // the new unit's output rows and weights, loaded long before its flush
         if (dm.direct_combine && cur_tag >= 0) dir.load(dm, ws, cur_slot, cur_mt, cur_col0, lane);
       }
       if (mine && meta.y > 0)
-        rows.consume(smem_s + b * geo.stage + slice * kSliceBytes, stg + slice * kSliceBytes,
+        rows.consume(smem_s + b * geo.stage + slice * B::kSlice, stg + slice * B::kSlice,
                      geo.stride, stg + kBatch * geo.stride, meta.y, mt, lane);
       __syncwarp();  // every lane has read the stage
       if (lane == 0) mbar_arrive(empty + b);
@@ -290,25 +310,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t down_gemv_smem_bytes(int d, bool bf16) {
-  const Geometry g = geometry(d * (bf16 ? 2 : 4), kStageExtra);
+  const int block = wide_rows(d, bf16) ? Blocks<true>::kBlock : Blocks<false>::kBlock;
+  const Geometry g = geometry(d * (bf16 ? 2 : 4), kStageExtra, block);
   return static_cast<size_t>(g.n_stages) * g.stage;
 }
+
+namespace {
+template <typename TW, bool WIDE>
+cudaError_t launch_dg(const Dims& dm, const Workspace& ws, const void* Wd, const void* Wds,
+                      int n_sms, void* out, bool out_bf16, cudaStream_t st) {
+  const cudaError_t e = smem_limit(down_gemv_kernel<TW, WIDE>, kSmemBudget);
+  if (e != cudaSuccess) return e;
+  const int grid = n_sms;  // one CTA per SM
+  const size_t smem = down_gemv_smem_bytes(dm.d, sizeof(TW) == 2);
+  return launch_k(down_gemv_kernel<TW, WIDE>, grid, kThreads, smem, st, dm, ws,
+                  static_cast<const TW*>(Wd), static_cast<const TW*>(Wds), out, out_bf16 ? 1 : 0);
+}
+}  // namespace
 
 cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd,
                              const void* Wds, bool bf16, int n_sms, void* out, bool out_bf16,
                              cudaStream_t st) {
-  const cudaError_t e = bf16 ? smem_limit(down_gemv_kernel<__nv_bfloat16>, kSmemBudget)
-                             : smem_limit(down_gemv_kernel<float>, kSmemBudget);
-  if (e != cudaSuccess) return e;
-  const int grid = n_sms;  // one CTA per SM
-  const size_t smem = down_gemv_smem_bytes(dm.d, bf16);
-  if (bf16)
-    return launch_k(down_gemv_kernel<__nv_bfloat16>, grid, kThreads, smem, st, dm, ws,
-                    static_cast<const __nv_bfloat16*>(Wd), static_cast<const __nv_bfloat16*>(Wds),
-                    out, out_bf16 ? 1 : 0);
-  return launch_k(down_gemv_kernel<float>, grid, kThreads, smem, st, dm, ws,
-                  static_cast<const float*>(Wd), static_cast<const float*>(Wds), out,
-                  out_bf16 ? 1 : 0);
+  if (!bf16) return launch_dg<float, false>(dm, ws, Wd, Wds, n_sms, out, out_bf16, st);
+  if (wide_rows(dm.d, true))
+    return launch_dg<__nv_bfloat16, true>(dm, ws, Wd, Wds, n_sms, out, out_bf16, st);
+  return launch_dg<__nv_bfloat16, false>(dm, ws, Wd, Wds, n_sms, out, out_bf16, st);
 }
 
 }  // namespace moe

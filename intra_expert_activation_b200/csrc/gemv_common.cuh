@@ -17,7 +17,7 @@ namespace {
 constexpr int kConsumers = 8;
 constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
 constexpr int kBatch = 8;            // rows per stage (the mma's K)
-constexpr int kSliceBytes = 512;     // row bytes per consumer warp
+constexpr int kSliceBytes = 512;     // row bytes per consumer warp (4 KB column blocks)
 constexpr int kBlockBytes = kConsumers * kSliceBytes;  // column block: 4 KB of a row
 constexpr int kRowPad = 16;          // row stride = block bytes + 16
 constexpr int kMaxStages = 6;
@@ -86,15 +86,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Stage geometry for a row of row_bytes: the column block (<= 4 KB), the
-// stage size (kBatch rows at the padded stride, then `extra` bytes of
+// Stage geometry for a row of row_bytes: the column block (<= block_max),
+// the stage size (kBatch rows at the padded stride, then `extra` bytes of
 // per-stage data) and the number of stages that fit the budget.
 struct Geometry {
   int block, stride, stage, n_stages;
 };
-__host__ __device__ inline Geometry geometry(int row_bytes, int extra) {
+__host__ __device__ inline Geometry geometry(int row_bytes, int extra,
+                                             int block_max = kBlockBytes) {
   Geometry g;
-  g.block = row_bytes < kBlockBytes ? row_bytes : kBlockBytes;
+  g.block = row_bytes < block_max ? row_bytes : block_max;
   g.stride = g.block + kRowPad;
   g.stage = kBatch * g.stride + extra;
   g.n_stages = kSmemBudget / g.stage;
@@ -117,11 +118,6 @@ __device__ __forceinline__ bool consumers_any(bool v) {
   return r != 0;
 }
 
-// Bitmap words a thread loads in the start search (every word of a group at
-// once: F_e / 32 <= 2048 words for d_ff <= 65536, over >= 256 threads).
-constexpr int kStartWords = 8;
-constexpr int kWordCache = 2048;  // the start group's words, kept for the producer
-
 // Where a CTA's share of the row sequence starts.
 struct Start {
   int i;        // GEMV list index of the first group
@@ -130,17 +126,7 @@ struct Start {
   uint32_t m;   // mask of the rows of word w that are still to come
   int rows;     // rows of this CTA
   int g, row;   // the first group and the row within its pass
-  int n_gv;     // GEMV groups of this forward
   Group gr;     // the first group's record
-};
-
-// Shared memory of the start search: the result, the scan's per-warp sums,
-// and the start group's bitmap words (valid when the group has at most
-// kWordCache words), which the producer's walk reads instead of L2.
-struct StartSmem {
-  Start st;
-  long long warp_sum[32];
-  uint32_t words[kWordCache];
 };
 
 // The producer's walk over its CTA's rows: group list index, pass, next word
@@ -152,8 +138,6 @@ struct Walk {
   int n_gv;  // GEMV groups
   int g, words, passes, slot0, m_tok, expert, xrow0;  // unit data of group i
   int serial;  // increments whenever the unit (group, pass) changes
-  int cache_g;               // group whose words are in `cache` (-1: none)
-  const uint32_t* cache;     // the start search's word cache (shared memory)
 };
 
 // Unit data of group g (record gr).
@@ -169,18 +153,16 @@ __device__ __forceinline__ void walk_set_group(const Dims& dm, Walk& k, int g, c
 }
 
 // The producer's walk from the CTA's start (no global loads).
-__device__ __forceinline__ void walk_begin(const Dims& dm, const StartSmem& ss, Walk& k, int MT) {
-  const Start& st = ss.st;
+__device__ __forceinline__ void walk_begin(const Dims& dm, const Workspace& ws, const Start& st,
+                                           Walk& k, int MT) {
   k.i = st.i;
   k.p = st.p;
   k.w = st.w;
   k.m = st.m;
   k.left = st.rows;
-  k.n_gv = st.n_gv;
+  k.n_gv = min(__ldcg(ws.meta + kMetaGemvCount), kListMax);
   k.serial = 0;
   walk_set_group(dm, k, st.g, st.gr, MT);
-  k.cache_g = k.words <= kWordCache ? st.g : -1;
-  k.cache = ss.words;
 }
 
 // Loads group i's unit data; false past the end of the GEMV list.
@@ -234,9 +216,7 @@ __device__ int walk_next(const Dims& dm, const Workspace& ws, Walk& k, uint16_t*
       continue;
     }
     const int word = k.w + lane;
-    uint32_t bits = word >= k.words ? 0u
-                    : k.g == k.cache_g ? k.cache[word]
-                                       : __ldcg(ws.union_bits + (size_t)k.g * dm.fw + word);
+    uint32_t bits = word < k.words ? __ldcg(ws.union_bits + (size_t)k.g * dm.fw + word) : 0u;
     if (lane == 0) bits &= k.m;
     const int c = __popc(bits);
     int incl = c;
@@ -273,11 +253,10 @@ __device__ int walk_next(const Dims& dm, const Workspace& ws, Walk& k, uint16_t*
 }
 
 // The CTA's share of rows and where it starts. Every thread calls it.
-__device__ void find_start(const Dims& dm, const Workspace& ws, int MT, StartSmem& ss) {
+__device__ void find_start(const Dims& dm, const Workspace& ws, int MT, Start* st,
+                           long long* sm_warp) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = blockDim.x / 32;
-  Start* st = &ss.st;
-  long long* sm_warp = ss.warp_sum;
   // the first list entries are read while the list length is still in
   // flight (they are inside the list's capacity either way)
   const int g_spec = tid < dm.groups_max ? __ldcg(ws.gemv_list + tid) : 0;
@@ -289,7 +268,6 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, StartSme
   if (tid == 0) {
     st->i = -1;
     st->rows = 0;
-    st->n_gv = n_gv;
   }
   for (int sweep = one ? 1 : 0; sweep < 2; ++sweep) {
     long long carry = 0;
@@ -354,47 +332,39 @@ __device__ void find_start(const Dims& dm, const Workspace& ws, int MT, StartSme
   __syncthreads();
   if (st->rows <= 0 || st->i < 0) return;  // uniform
   // the bitmap word holding row st->row of group st->g: every thread loads
-  // its kStartWords consecutive words of the group at once (one pass over L2
-  // for the whole group), keeps them in the word cache for the producer, and
-  // a CTA-wide prefix sum of their row counts in word order finds the word
-  const int g = st->g, words = st->w, skip = st->row;
-  uint32_t bw[kStartWords];
-  int c = 0;
-#pragma unroll
-  for (int q = 0; q < kStartWords; ++q) {
-    const int word = tid * kStartWords + q;
-    bw[q] = word < words ? __ldcg(ws.union_bits + (size_t)g * dm.fw + word) : 0u;
-    c += __popc(bw[q]);
-  }
-#pragma unroll
-  for (int q = 0; q < kStartWords; ++q) {
-    const int word = tid * kStartWords + q;
-    if (word < words && word < kWordCache) ss.words[word] = bw[q];
-  }
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
+  // one word of a window of blockDim words (all loads in flight together),
+  // a CTA-wide prefix sum of their row counts finds the word
+  const int g = st->g, words = st->w;
+  int skip = st->row;
   int* cnt_w = reinterpret_cast<int*>(sm_warp);
-  if (lane == 31) cnt_w[warp] = incl;
-  __syncthreads();  // also: every thread has read st->w before its owner rewrites it
-  int before = 0;
-  for (int w = 0; w < warp; ++w) before += cnt_w[w];
-  int excl = before + incl - c;
-  if (excl <= skip && skip < excl + c) {  // this thread's words hold the first row
+  for (int w0 = 0; w0 < words; w0 += blockDim.x) {
+    const int word = w0 + tid;
+    const uint32_t bits = word < words ? __ldcg(ws.union_bits + (size_t)g * dm.fw + word) : 0u;
+    const int c = __popc(bits);
+    int incl = c;
 #pragma unroll
-    for (int q = 0; q < kStartWords; ++q) {
-      const int cq = __popc(bw[q]);
-      if (excl <= skip && skip < excl + cq) {
-        uint32_t m = bw[q];
-        for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
-        st->w = tid * kStartWords + q;
-        st->m = m;
-      }
-      excl += cq;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
     }
+    if (lane == 31) cnt_w[warp] = incl;
+    __syncthreads();  // also: every thread has read st->w before its owner rewrites it
+    int before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int x = cnt_w[w];
+      if (w < warp) before += x;
+      total += x;
+    }
+    const int excl = before + incl - c;
+    if (excl <= skip && skip < excl + c) {  // this thread's word holds the first row
+      uint32_t m = bits;
+      for (int t = 0; t < skip - excl; ++t) m &= m - 1;  // drop the rows before it
+      st->w = word;
+      st->m = m;
+    }
+    __syncthreads();  // cnt_w is rewritten by the next window
+    if (skip < total) break;  // uniform
+    skip -= total;
   }
   __syncthreads();
 }

@@ -13,14 +13,16 @@ constexpr int kTok = 8;         // token columns of the mma (passes hold up to 8
 constexpr int kTokStride = kTok;  // floats per row of an fp32 h array [row][token]
 constexpr int kHBytes = 32;          // h bytes per row slot: 8 x bf16 (16 B used) or 8 x fp32
 
-template <typename TW>
+// TILES: 16-column tiles of a consumer warp's slice (bf16: 16 for a
+// 512-byte slice, 32 for 1 KB); the fp32 rows take 512-byte slices.
+template <typename TW, int TILES = 16>
 struct Rows;
 
 // bf16: tensor-core multiply of the landed rows.
-template <>
-struct Rows<__nv_bfloat16> {
+template <int TILES>
+struct Rows<__nv_bfloat16, TILES> {
   static constexpr int MT = kGemvTokens;  // tokens per pass
-  static constexpr int kTiles = 16;       // 16-column tiles of the warp's 256 columns
+  static constexpr int kTiles = TILES;    // 16-column tiles of the warp's slice
   float acc[kTiles][4];
 
   __device__ void zero() {
@@ -100,8 +102,8 @@ struct Rows<__nv_bfloat16> {
 };
 
 // fp32: packed fp32x2 FMAs, 4 columns per lane, up to 8 tokens.
-template <>
-struct Rows<float> {
+template <int TILES>
+struct Rows<float, TILES> {
   static constexpr int MT = 8;
   uint64_t acc[MT][2];
 

@@ -623,11 +623,127 @@ __global__ void __launch_bounds__(256) permute_kernel(Dims dm, Workspace ws, con
 }
 
 // Small batches (T <= kSmallTokens): the whole routing step in one CTA of
-// 16 warps with no cross-CTA ticket: logits, top-k, in-order stable ranks,
-// layout, and the permute copies of the x rows (and zeroing of the Y rows
-// that GEMV splits add into).
+// 16 warps with no cross-CTA ticket and three CTA barriers: logits (every
+// warp), top-k (a warp per token), the layout (warp 0, small_layout), then
+// the permute copies of the x rows and the zeroing of the Y rows that the
+// row stream adds into.
 constexpr int kSmallThreads = 512;
 constexpr int kSmallWarps = kSmallThreads / 32;
+
+// Shared memory of the small-batch layout.
+struct SmallLayout {
+  int cnt[kMaxExperts];       // pairs per expert
+  int gidx[kMaxExperts];      // group (= 8-slot block) of each touched expert
+  int gpath[kMaxExperts + 8]; // path of each group (routed, then shared)
+  int yzero[kMaxExperts + 1]; // 1: the expert's Y rows start at zero (last: shared)
+};
+
+// The layout of a batch of T <= kSmallTokens tokens, by one warp. Every
+// touched expert holds at most 4 pairs, so it is one group in one block of
+// kSlotAlign slots, in expert order; each shared expert is one group of T
+// tokens. Writes the same records as build_layout (groups, paths, lists,
+// cleared union counts, meta, counters) and each pair's slot (slot_s; perm,
+// slot_of, slot_w, padding marks). cnt[] must be zero on entry.
+__device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel,
+                             const float* selw, int* slot_s, SmallLayout& L, int lane) {
+  const int E = dm.E, T = dm.T, k = dm.k, S = dm.S, P = T * k;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int p = lane; p < P; p += 32) atomicAdd(&L.cnt[sel[p]], 1);
+  __syncwarp();
+  // touched experts in expert order: group index and path
+  int n_touched = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const int c = e < E ? L.cnt[e] : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
+    if (c > 0) {
+      const int g = n_touched + __popc(bal & lt);
+      const int path = group_path_of(dm, c);
+      L.gidx[e] = g;
+      L.gpath[g] = path;
+      Group gr;
+      gr.expert = e;
+      gr.slot0 = g * kSlotAlign;
+      gr.m = c;
+      gr.xrow0 = g * kSlotAlign;
+      ws.groups[g] = gr;
+      ws.group_path[g] = path;
+      ws.union_cnt[g] = 0;
+      // padding slots of the block: marked in perm (their X_perm rows are
+      // never used: every kernel masks the columns past a group's count)
+      for (int r = c; r < kSlotAlign; ++r) ws.perm[g * kSlotAlign + r] = -1;
+    }
+    if (e < E) L.yzero[e] = c > 0 && on_gemv_list(group_path_of(dm, c));
+    n_touched += __popc(bal);
+  }
+  const int n_groups = n_touched + S;
+  if (lane < S) {  // shared experts: one group of all T tokens each
+    const int g = n_touched + lane;
+    const int path = group_path_of(dm, T);
+    L.gpath[g] = path;
+    Group gr;
+    gr.expert = E + lane;
+    gr.slot0 = dm.slots_routed + lane * dm.T_pad;
+    gr.m = T;
+    gr.xrow0 = 0;
+    ws.groups[g] = gr;
+    ws.group_path[g] = path;
+    ws.union_cnt[g] = 0;
+  }
+  __syncwarp();
+  // GEMV and tensor-core lists in group order (a candidate is on both)
+  int n_gv = 0, n_tc = 0, n_cand = 0, n_tc_sh = 0, any_gv_sh = 0;
+  for (int g0 = 0; g0 < n_groups; g0 += 32) {
+    const int g = g0 + lane;
+    const int path = g < n_groups ? L.gpath[g] : kPathNone;
+    const bool gv = g < n_groups && on_gemv_list(path);
+    const bool tc = g < n_groups && on_tc_list(path);
+    const bool cand = g < n_groups && path == kPathCand;
+    const unsigned bgv = __ballot_sync(0xffffffffu, gv), btc = __ballot_sync(0xffffffffu, tc);
+    if (gv) ws.gemv_list[n_gv + __popc(bgv & lt)] = g;
+    if (tc) ws.tc_list[n_tc + __popc(btc & lt)] = g;
+    n_gv += __popc(bgv);
+    n_tc += __popc(btc);
+    n_cand += __popc(__ballot_sync(0xffffffffu, cand));
+    n_tc_sh += __popc(__ballot_sync(0xffffffffu, tc && !cand && g >= n_touched));
+    any_gv_sh |= __ballot_sync(0xffffffffu, gv && g >= n_touched) != 0u;
+  }
+  if (lane == 0) L.yzero[E] = any_gv_sh;
+  // each pair's slot: its expert's block + its rank among the expert's pairs
+  for (int p = lane; p < P; p += 32) {
+    const int e = sel[p];
+    int r = 0;
+    for (int q = 0; q < p; ++q) r += sel[q] == e;
+    int slot = L.gidx[e] * kSlotAlign + r;
+    if (!moe_in_bounds(ws.status, slot >= 0 && slot < dm.slots_routed)) slot = 0;
+    slot_s[p] = slot;
+    ws.perm[slot] = p / k;
+    ws.slot_of[p] = slot;
+    ws.slot_w[slot] = selw[p];
+  }
+  if (lane < kCntWords) {
+    unsigned long long v = 0ull;
+    if (lane == kCntGemv) v = n_gv - n_cand;  // candidates are counted by the kernel that takes them
+    if (lane == kCntTc) v = n_tc - n_cand;
+    if (lane == kCntDownRows && dm.mode != kModeTc)  // the GEMV kernel adds its rows
+      v = (unsigned long long)(n_tc - n_cand - n_tc_sh) * dm.F +
+          (unsigned long long)n_tc_sh * dm.Fs;
+    if (lane == kCntRoutedH) v = (unsigned long long)P * dm.F;
+    if (lane == kCntSharedH) v = (unsigned long long)S * T * dm.Fs;
+    ws.counters[lane] = v;
+  }
+  if (lane == 0) {
+    ws.meta[kMetaRoutedGroups] = n_touched;
+    ws.meta[kMetaGroups] = n_groups;
+    ws.meta[kMetaSlotsUsed] = n_touched * kSlotAlign;
+    ws.meta[kMetaExpertsTouched] = n_touched;
+    ws.meta[kMetaGemvCount] = n_gv;
+    ws.meta[kMetaTcCount] = n_tc;
+    ws.meta[kMetaDone] = 0;
+    ws.meta[kMetaDownDone] = 0;
+  }
+  __syncwarp();
+}
 
 template <typename TX>
 __global__ void __launch_bounds__(kSmallThreads, 1)
@@ -637,8 +753,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __shared__ int sel[kSmallTokens * 16];
   __shared__ float selw[kSmallTokens * 16];
   __shared__ int slot_s[kSmallTokens * 16];
-  __shared__ int cnt[kMaxExperts];
-  __shared__ int poff[kMaxExperts + 1];
+  __shared__ SmallLayout L;
 
   grid_dep_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -657,40 +772,27 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
                                 Wr + (size_t)e * d + (size_t)sl * dsl, dsl, lane);
     if (lane == 0) lpart[sl][t][e] = a;
   }
-  for (int e = tid; e < E; e += kSmallThreads) cnt[e] = 0;
-  if (tid < kCntWords) ws.counters[tid] = 0ull;
+  for (int e = tid; e < E; e += kSmallThreads) L.cnt[e] = 0;
   __syncthreads();
-  for (int i = tid; i < TE; i += kSmallThreads) {
-    const int t = i / E, e = i % E;
-    float a = 0.f;
-    for (int sl = 0; sl < ns; ++sl) a += lpart[sl][t][e];
-    lg[t][e] = a + (bias ? bias[e] : 0.f);
+  if (warp < T) {  // warp t: token t's logits (slices in order, + bias) and top-k
+    for (int e = lane; e < E; e += 32) {
+      float a = 0.f;
+      for (int sl = 0; sl < ns; ++sl) a += lpart[sl][warp][e];
+      lg[warp][e] = a + (bias ? bias[e] : 0.f);
+    }
+    __syncwarp();
+    topk_token(dm, ws, lg[warp], warp, lane, sel + warp * k, selw + warp * k);
+  } else {  // the other warps clear the next kernels' cross-CTA tickets
+    for (int x2 = tid - T * 32; x2 < dm.sk_ctas; x2 += kSmallThreads - T * 32)
+      ws.sk_flags[x2] = 0;
+    for (int x2 = tid - T * 32; x2 < dm.tc_part_units; x2 += kSmallThreads - T * 32)
+      ws.tc_ticket[x2] = 0;
   }
   __syncthreads();
-  for (int t = warp; t < T; t += kSmallWarps)
-    topk_token(dm, ws, lg[t], t, lane, sel + t * k, selw + t * k);
+  if (warp == 0) small_layout(dm, ws, sel, selw, slot_s, L, lane);
   __syncthreads();
-  // stable rank of pair p among earlier pairs of the same expert
-  for (int p = tid; p < P; p += kSmallThreads) {
-    const int e = sel[p];
-    int r = 0;
-    for (int q = 0; q < p; ++q) r += sel[q] == e;
-    slot_s[p] = r;
-    atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  build_layout(dm, ws, cnt, poff);
-  __syncthreads();
-  for (int p = tid; p < P; p += kSmallThreads) {
-    int slot = poff[sel[p]] + slot_s[p];
-    if (!moe_in_bounds(ws.status, slot >= 0 && slot < dm.slots_routed)) slot = 0;
-    slot_s[p] = slot;
-    ws.perm[slot] = p / k;
-    ws.slot_of[p] = slot;
-    ws.slot_w[slot] = selw[p];
-  }
-  __syncthreads();
-  // copies: one warp per pair, then padding slots, then shared Y rows
+  // copies: one warp per pair (x row to X_perm; the Y rows the row stream
+  // adds into start at zero), then the shared experts' Y rows
   constexpr int kVec = 16 / sizeof(TX);
   const int nv = d / kVec, nz = d / 4;
   for (int p = warp; p < P; p += kSmallWarps) {
@@ -698,7 +800,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     uint4* dst = reinterpret_cast<uint4*>(static_cast<TX*>(ws.xperm) + (size_t)slot * d);
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(p / k) * d);
     copy_row(dst, src, nv, lane);
-    if (!dm.direct_combine && ws.y_zero[sel[p]]) {
+    if (!dm.direct_combine && L.yzero[sel[p]]) {
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)slot * d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -708,12 +810,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)t * d);
       for (int i = lane; i < nz; i += 32) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  }
-  // padding slots: marked in perm; their X_perm rows are left as they are
-  // (every kernel masks the columns of tokens past a group's count)
-  for (int e = warp; e < E; e += kSmallWarps)
-    for (int sl = poff[e] + cnt[e] + lane; sl < poff[e + 1]; sl += 32) ws.perm[sl] = -1;
-  if (!dm.direct_combine && ws.y_zero[E]) {
+  } else if (L.yzero[E]) {
     for (int q = warp; q < dm.S * T; q += kSmallWarps) {
       const int sh = q / T, t = q % T;
       float4* yz = reinterpret_cast<float4*>(ws.y + (size_t)(dm.slots_routed + sh * dm.T_pad + t) * d);

@@ -48,8 +48,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(R::MT == MT, "tokens per pass");
   constexpr int ES = static_cast<int>(sizeof(TW));
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ StartSmem ss;
-  const Start& start = ss.st;
+  __shared__ Start start;
+  __shared__ long long sm_warp[kThreads / 32];
   __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
   __shared__ uint16_t list[kListRows];
   __shared__ uint16_t rowj[kListRows];              // the current run's neuron indices
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
 
   grid_dep_wait();
-  find_start(dm, ws, MT, ss);
+  find_start(dm, ws, MT, &start, sm_warp);
   if (start.rows <= 0 || start.i < 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kConsumers) {
     // ------------------------------------------------------------ producer
     Walk k;
-    walk_begin(dm, ss, k, MT);
+    walk_begin(dm, ws, start, k, MT);
     int s = 0;
     bool ok = true;
     for (bool last_run = false; ok && !last_run;) {

@@ -112,6 +112,15 @@ static void check_geometry() {
         CHECK((long long)g.n_stages * g.stage <= kSmemBudget, "d %d smem", d);
         CHECK(g.block <= kBlockBytes && g.block % kSliceBytes == 0, "block %d", g.block);
         CHECK(g.stride % 16 == 0 && g.stage % 16 == 0, "alignment d %d", d);
+        // the down row stream's wide blocks (bf16 rows of a multiple of 1 KB):
+        // up to 8 KB per block, whole 1 KB slices, at least two stages
+        if (es == 2 && d % 512 == 0) {
+          const Geometry w = geometry(row_bytes, extra, 8192);
+          CHECK(w.n_stages >= 2 && w.n_stages <= kMaxStages, "wide d %d stages %d", d, w.n_stages);
+          CHECK((long long)w.n_stages * w.stage <= kSmemBudget, "wide d %d smem", d);
+          CHECK(w.block <= 8192 && w.block % 1024 == 0, "wide block %d", w.block);
+          CHECK(w.stride % 16 == 0 && w.stage % 16 == 0, "wide alignment d %d", d);
+        }
       }
     }
 }
