@@ -121,7 +121,7 @@ typedef struct {
   int32_t gemv_max_tokens;    /* AUTO: groups with <= this many tokens use the GEMV path.
                                  0: automatic -- groups of <= 4 tokens on the GEMV path, and
                                  (|h| score, bf16) groups of 5..8 tokens choose after gate/up:
-                                 the GEMV path if their active-row union is <= 0.9 x d_ff,
+                                 the GEMV path if their active-row union is <= 0.8 x d_ff,
                                  else all rows on the tensor cores */
   float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: never) */
   int32_t score;              /* moe_score (0: MOE_SCORE_H) */

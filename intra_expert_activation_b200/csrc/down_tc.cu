@@ -46,6 +46,15 @@ __device__ __forceinline__ bool epi_all(bool v) {
       : "memory");
   return r != 0;
 }
+// Units in flight between the TMA warp, which takes them from the queue, and
+// the MMA and epilogue warps, which process them in the same order.
+constexpr int kUQ = 4;
+struct UnitQueue {
+  int id[kUQ];                 // unit of each slot, -1: the queue is empty
+  uint64_t full[kUQ];          // the TMA warp published the slot (1 arrival)
+  uint64_t empty[kUQ];         // the MMA warp and the 4 epilogue warps read it (5 arrivals)
+};
+
 constexpr uint32_t kAAtom = 64 * 128;  // one 64-row x 128-byte swizzled atom column
 constexpr uint32_t kABytes = 2 * kAAtom;
 
@@ -94,6 +103,36 @@ __device__ __forceinline__ DownUnit decode(const DownTcParams& p, int u, int n_s
   return du;
 }
 
+// TMA warp: take the next unit from the queue and publish it in slot
+// n % kUQ, once the MMA and epilogue warps have read that slot's previous
+// unit. Returns the unit, -1 when the queue is empty (also published), or -2
+// when a wait gave up.
+__device__ __forceinline__ int uq_take(UnitQueue& uq, int n, int* queue, int n_units,
+                                       volatile int* abort, int* status, int lane) {
+  const int q = n % kUQ;
+  if (n >= kUQ && !warp_wait(&uq.empty[q], ((n / kUQ) - 1) & 1, abort, status)) return -2;
+  int u = 0;
+  if (lane == 0) {
+    u = atomicAdd(queue, 1);
+    if (u >= n_units) u = -1;
+    uq.id[q] = u;
+    mbar_arrive(&uq.full[q]);
+  }
+  return __shfl_sync(0xffffffffu, u, 0);
+}
+
+// MMA and epilogue warps: the n-th unit of this CTA (-1: none left, -2: a
+// wait gave up); the slot is released as soon as it is read.
+__device__ __forceinline__ int uq_next(UnitQueue& uq, int n, volatile int* abort, int* status,
+                                       int lane) {
+  const int q = n % kUQ;
+  if (!warp_wait(&uq.full[q], (n / kUQ) & 1, abort, status)) return -2;
+  const int u = uq.id[q];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&uq.empty[q]);
+  return u;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     down_tc_kernel(const __grid_constant__ DownTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -112,11 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  __shared__ UnitQueue uq;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
+    }
+    for (int q = 0; q < kUQ; ++q) {
+      mbar_init(&uq.full[q], 1);
+      mbar_init(&uq.empty[q], 5);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
@@ -152,7 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     uint32_t it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int n = 0; ok; ++n) {
+      const int u =
+          uq_take(uq, n, p.ws.meta + kMetaTcQueue, n_units, abort_flag, p.ws.status, lane);
+      if (u == -2) ok = false;
+      if (u < 0) break;
       const DownUnit du = decode(p, u, n_slices, ks);
       if (du.cand && !du.skip && du.slice == 0 && du.k0 == 0 && lane == 0) {  // a candidate taken here
         atomicAdd(p.ws.counters + kCntDownRows,
@@ -213,7 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ MMA issuer
     uint32_t it = 0, uidx = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (int n = 0; ok; ++n) {
+      const int u = uq_next(uq, n, abort_flag, p.ws.status, lane);
+      if (u < 0) break;
       const DownUnit du = decode(p, u, n_slices, ks);
       if (du.nk == 0) continue;  // empty union: the epilogue writes zeros
       const int N = (du.gr.m + 15) & ~15;
@@ -258,7 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const int d = p.dm.d;
     uint32_t uidx = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    for (int n = 0;; ++n) {
+      const int u = uq_next(uq, n, abort_flag, p.ws.status, lane);
+      // the four warps leave together (the part path below has barriers)
+      const bool got = ks > 1 ? epi_all(u != -2) : u != -2;
+      if (!got || u < 0) break;
       const DownUnit du = decode(p, u, n_slices, ks);
       const int m = du.gr.m;
       const int col = du.slice * kDownSlice + 32 * q + lane;
@@ -310,26 +364,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
           const float* pb = p.ws.tc_part + static_cast<size_t>(ub) * ks * kTcPartTokens * kDownSlice +
                             32 * q + lane;
-          // 8 tokens x all parts per batch: their loads are in flight together
-          // (one L2 round trip per batch, not one per value)
-          constexpr int kC = 8;
+          // 8 tokens x 6 parts per batch: their loads are in flight together
+          // (one L2 round trip per batch, not one per value); the sums run
+          // in part order
+          constexpr int kC = 8, kP = 6;
           for (int c0 = 0; c0 < m; c0 += kC) {
-            float v[kC][kTcMaxParts];
+            float acc[kC];
+#pragma unroll
+            for (int i = 0; i < kC; ++i) acc[i] = 0.f;
+            for (int p0 = 0; p0 < ks; p0 += kP) {
+              float v[kC][kP];
+#pragma unroll
+              for (int i = 0; i < kC; ++i)
+#pragma unroll
+                for (int pp = 0; pp < kP; ++pp)
+                  v[i][pp] = c0 + i < m && p0 + pp < ks
+                                 ? __ldcg(pb + (static_cast<size_t>(p0 + pp) * kTcPartTokens +
+                                                c0 + i) *
+                                                   kDownSlice)
+                                 : 0.f;
+#pragma unroll
+              for (int i = 0; i < kC; ++i)
+#pragma unroll
+                for (int pp = 0; pp < kP; ++pp) acc[i] += v[i][pp];
+            }
 #pragma unroll
             for (int i = 0; i < kC; ++i)
-#pragma unroll
-              for (int pp = 0; pp < kTcMaxParts; ++pp)
-                v[i][pp] = c0 + i < m && pp < ks
-                               ? __ldcg(pb + (static_cast<size_t>(pp) * kTcPartTokens + c0 + i) *
-                                                 kDownSlice)
-                               : 0.f;
-#pragma unroll
-            for (int i = 0; i < kC; ++i) {
-              float acc = 0.f;
-#pragma unroll
-              for (int pp = 0; pp < kTcMaxParts; ++pp) acc += v[i][pp];  // part order
-              if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = acc;
-            }
+              if (c0 + i < m) yc[static_cast<size_t>(c0 + i) * d] = acc[i];
           }
         }
       }
@@ -352,7 +413,9 @@ size_t down_tc_smem_bytes(int b_bytes, int stages) {
 }
 
 cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st) {
-  const cudaError_t e = smem_limit(down_tc_kernel, 227 * 1024);
+  // the limit covers this launch's dynamic shared memory (the kernel also
+  // has a little static shared memory, so 227 KB of dynamic would not fit)
+  const cudaError_t e = smem_limit(down_tc_kernel, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_k(down_tc_kernel, grid, kThreads, smem, st, p);
 }

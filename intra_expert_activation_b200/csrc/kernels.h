@@ -62,9 +62,10 @@ constexpr int kGemvTokens = 8;      // tokens per GEMV pass (the row-stream mma'
 // their active-row union: the row stream if passes x union rows <=
 // kCandNum / kCandDen x d_ff, else all rows on the tensor cores. The ratio is
 // the measured bandwidth of the row stream over that of the all-rows
-// tensor-core path on the Mixtral-shaped layer.
+// tensor-core path on the Mixtral-shaped layer (about 5.0 and 6.3 TB/s per
+// launch, CUDA-event timed).
 constexpr int kGemvCandMax = 8;
-constexpr int kCandNum = 9, kCandDen = 10;
+constexpr int kCandNum = 4, kCandDen = 5;
 
 // A candidate group (kPathCand) takes the row stream when its passes over
 // the union rows cost less than all F_e rows on the tensor cores; both down
@@ -78,6 +79,7 @@ __host__ __device__ inline bool cand_takes_gemv(int union_rows, int passes, int 
 enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUsed = 3,
             kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
             kMetaDownDone = 7,  // row-stream CTAs finished (direct combine ticket)
+            kMetaTcQueue = 8,   // next tensor-core down unit to hand out
             kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
@@ -134,15 +136,16 @@ constexpr int kDirectMax = 16;  // tokens up to which the row stream combines di
 // 35-40 GB/s, so HBM is only saturated when every SM has work: with few
 // groups most SMs idled (one 117 MB group of the Mixtral-shaped layer = 32
 // units took 108 us). When the units fill less than 3/4 of the grid, each
-// unit's rows are cut into ks parts, ks in 1..kTcMaxParts minimising the
-// rounds per unit of work, ceil(units x ks / grid) / ks (the smaller ks on
-// ties), with at most dm.tc_part_units part units and at least one K-block
-// per part. Parts write fp32 partial sums to the workspace and the last part
-// of a unit to finish (a ticket) adds them in part order into Y, so results
-// do not depend on timing. Only groups of <= kTcPartTokens tokens are cut
-// (decode batches). The router (to clear the tickets) and the kernel
-// evaluate it on the same inputs.
-constexpr int kTcMaxParts = 12;
+// unit's rows are cut into ks parts, enough for about two units per CTA,
+// ks = ceil(2 grid / units) (at most kTcMaxParts, at least one K-block per
+// part, and within dm.tc_part_units part units); the CTAs take units from a
+// queue (an atomic ticket), so the units of the SMs that stream slower are
+// taken over by the others. Parts write fp32 partial sums to the workspace
+// and the last part of a unit to finish (a ticket) adds them in part order
+// into Y, so results do not depend on timing. Only groups of <=
+// kTcPartTokens tokens are cut (decode batches). The router (to clear the
+// tickets) and the kernel evaluate it on the same inputs.
+constexpr int kTcMaxParts = 24;
 constexpr int kTcPartTokens = 64;
 __host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
   if (dm.mode == kModeTc || n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
@@ -152,18 +155,11 @@ __host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
   const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);
   if (4 * base >= 3 * grid) return 1;
   const int f_min = dm.S > 0 && dm.Fs < dm.F ? dm.Fs : dm.F;
-  const int cap = f_min / kKBlock < kTcMaxParts ? f_min / kKBlock : kTcMaxParts;
-  int best = 1;
-  long long bn = (base + grid - 1) / grid, bd = 1;  // rounds per unit of work: bn / bd
-  for (int ks = 2; ks <= cap && base * ks <= dm.tc_part_units; ++ks) {
-    const long long r = (base * ks + grid - 1) / grid;
-    if (r * bd < bn * ks) {
-      best = ks;
-      bn = r;
-      bd = ks;
-    }
-  }
-  return best;
+  long long ks = (2 * grid + base - 1) / base;
+  if (ks > kTcMaxParts) ks = kTcMaxParts;
+  if (ks > f_min / kKBlock) ks = f_min / kKBlock;
+  if (ks > dm.tc_part_units / base) ks = dm.tc_part_units / base;
+  return ks < 1 ? 1 : static_cast<int>(ks);
 }
 
 struct Workspace {

@@ -261,7 +261,7 @@ Layout make_layout(const moe_sparse_desc* d) {
   }
   // tensor-core down units cut along K (bf16, groups of <= 64 tokens): a
   // ticket per unit and a partial-sum block per part unit
-  c.tc_part_units = bf16 ? 640 : 0;
+  c.tc_part_units = bf16 ? 1024 : 0;
   sz[bTcTicket] = sizeof(int) * (size_t)c.tc_part_units;
   sz[bTcPart] = sizeof(float) * (size_t)c.tc_part_units * moe::kTcPartTokens * moe::kDownSlice;
   sz[bActBits] = d->debug ? sizeof(uint32_t) * (size_t)c.slots_total * c.fw : 0;

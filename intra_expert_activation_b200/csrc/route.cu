@@ -328,6 +328,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
         (unsigned long long)S * (unsigned long long)T * (unsigned long long)dm.Fs;
     ws.meta[kMetaDone] = 0;      // ticket counter for the next forward
     ws.meta[kMetaDownDone] = 0;  // the row stream's direct-combine ticket
+    ws.meta[kMetaTcQueue] = 0;   // the tensor-core down kernel's unit queue
   }
   __syncthreads();
   for (int x = tid; x <= E; x += blockDim.x) ws.expert_off[x] = poff[x];
@@ -741,6 +742,7 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
     ws.meta[kMetaTcCount] = n_tc;
     ws.meta[kMetaDone] = 0;
     ws.meta[kMetaDownDone] = 0;
+    ws.meta[kMetaTcQueue] = 0;
   }
   __syncwarp();
 }

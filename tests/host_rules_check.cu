@@ -33,7 +33,7 @@ static void check_ksplit() {
   const int Fs_[] = {128, 384, 768, 1408, 14336, 65536};
   const int Ts[] = {1, 2, 4, 8, 16, 17, 32, 48, 64, 65, 100, 128, 4096};
   const int grids[] = {0, 1, 16, 148, 160, 296, 320, 512};
-  const int units_caps[] = {0, 640};
+  const int units_caps[] = {0, 640, 1024};
   for (int mode : modes)
     for (int d : ds)
       for (int F : Fs_)
@@ -90,7 +90,7 @@ static void check_candidates() {
       bool prev = true;
       for (int u = 0; u <= F; ++u) {
         const bool take = cand_takes_gemv(u, passes, F);
-        CHECK(take == ((long long)u * passes * 10 <= 9LL * F), "F %d u %d", F, u);
+        CHECK(take == ((long long)u * passes * 5 <= 4LL * F), "F %d u %d", F, u);
         CHECK(!take || prev, "not monotone at F %d u %d", F, u);  // once false, stays false
         prev = take;
       }

@@ -324,7 +324,7 @@ def test_mixtral_sweep(sweep, T, q):
 def _expected_down_rows(gpu, F):
     """Rows the automatic per-group switch reads, from the GPU's own active
     sets: groups of <= 4 tokens stream their union; groups of 5..8 tokens
-    stream it iff 10 x union <= 9 x d_ff (one pass of 8 tokens), else all
+    stream it iff 5 x union <= 4 x d_ff (one pass of 8 tokens), else all
     d_ff rows on the tensor cores, as do larger groups."""
     act = unpack_bits(gpu["active_bits"], F)
     idx = gpu["topk_idx"].ravel()
@@ -332,7 +332,7 @@ def _expected_down_rows(gpu, F):
     for e in np.unique(idx):
         m = int((idx == e).sum())
         u = int(act[idx == e].any(axis=0).sum())
-        if m <= 4 or (m <= 8 and 10 * u <= 9 * F):
+        if m <= 4 or (m <= 8 and 5 * u <= 4 * F):
             rows += u
             n_gemv += 1
             cand_gemv += m > 4
