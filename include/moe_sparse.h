@@ -145,6 +145,9 @@ typedef struct {
   int64_t gate_up_rows_read;  /* W_gate + W_up rows loaded by the gate/up projection */
   int64_t down_rows_gemv;     /* of down_rows_read, the rows streamed by the row-stream (GEMV)
                                  kernel, once per pass of up to 8 tokens */
+  int64_t down_rows_fused;    /* of down_rows_read, the rows read by the gate/up kernel's fused
+                                 down projection (row-stream groups of <= 4 tokens, bf16):
+                                 per 128-neuron tile, the tile's active rows */
 } moe_stats;
 
 typedef struct moe_sparse_ctx moe_sparse_ctx;

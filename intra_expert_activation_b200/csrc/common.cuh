@@ -136,6 +136,18 @@ __device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort, int
 
 // ---------------------------------------------------------------- TMA
 
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from global to this CTA's shared memory, completion counted on bar as
+// transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -285,7 +297,76 @@ __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(uint32_t M, uint32_t
   return d;
 }
 
+// ---------------------------------------------------------------- direct combine
+
+// Under Dims::direct_combine the row stream adds w x the sums of a slot straight
+// into its token's output accumulator row Y[token] (zeroed by the router), and
+// the last CTA of the last kernel that adds writes out from those rows.
+
+// The output row and combine weight of slot s (routed: the token the router
+// placed there and its weight; shared: weight 1).
+__device__ __forceinline__ void slot_target(const Dims& dm, const Workspace& ws, int s, int& tok,
+                                            float& w) {
+  if (s < dm.slots_routed) {
+    tok = __ldcg(ws.perm + s);
+    w = __ldcg(ws.slot_w + s);
+  } else {
+    tok = (s - dm.slots_routed) % dm.T_pad;
+    w = 1.f;
+  }
+  if (!moe_in_bounds(ws.status, tok >= 0 && tok < dm.T)) tok = 0;  // checked build
+}
+
+// Direct combine, every thread of every CTA: after this CTA's sums are out,
+// take the ticket; the last CTA writes out[t][c] = Y[t][c] for t < T.
+static __device__ void direct_finish(const Dims& dm, const Workspace& ws, void* out, int out_bf16) {
+  __shared__ int is_last;
+  __threadfence();  // this thread's sums are visible before the ticket
+  __syncthreads();
+  if (threadIdx.x == 0)
+    is_last = atomicAdd(ws.meta + kMetaDownDone, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int n4 = dm.T * dm.d / 4;
+  const float4* y4 = reinterpret_cast<const float4*>(ws.y);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = __ldcg(y4 + i);
+    if (out_bf16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&lo);
+      u.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(out)[i] = u;
+    } else {
+      reinterpret_cast<float4*>(out)[i] = v;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- misc
+
+// Vector fp32 atomic adds (no return value) into global memory.
+__device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// 16 bytes of read-only data that is read once: not kept in L1. Not
+// volatile, so the compiler may schedule it (callers issue several
+// unconditionally before the first use; a load under a branch would be
+// waited for at the branch's join).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
 
 // SiLU(g) = g / (1 + e^-g) with the fast exponential and division intrinsics
 // (a few ulp of fp32; the threshold band is 1e-3 of tau). For g below about

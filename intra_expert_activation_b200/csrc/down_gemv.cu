@@ -59,20 +59,6 @@ struct Blocks {
 };
 __host__ __device__ inline bool wide_rows(int d, bool bf16) { return bf16 && d % 512 == 0; }
 
-// Direct combine: the output row and combine weight of slot s (routed: the
-// token the router placed there and its weight; shared: weight 1).
-__device__ __forceinline__ void slot_target(const Dims& dm, const Workspace& ws, int s, int& tok,
-                                            float& w) {
-  if (s < dm.slots_routed) {
-    tok = __ldcg(ws.perm + s);
-    w = __ldcg(ws.slot_w + s);
-  } else {
-    tok = (s - dm.slots_routed) % dm.T_pad;
-    w = 1.f;
-  }
-  if (!moe_in_bounds(ws.status, tok >= 0 && tok < dm.T)) tok = 0;  // checked build
-}
-
 // Where a consumer lane's sums of the current unit go under direct combine.
 template <typename TW>
 struct Direct;
@@ -119,33 +105,6 @@ struct Direct<float> {  // every token of the pass per lane
     r.flush_rows(row, w, mt, lane);
   }
 };
-
-// Direct combine, every thread of every CTA: after this CTA's sums are out,
-// take the ticket; the last CTA writes out[t][c] = Y[t][c] for t < T.
-__device__ void direct_finish(const Dims& dm, const Workspace& ws, void* out, int out_bf16) {
-  __shared__ int is_last;
-  __threadfence();  // this thread's sums are visible before the ticket
-  __syncthreads();
-  if (threadIdx.x == 0)
-    is_last = atomicAdd(ws.meta + kMetaDownDone, 1) == static_cast<int>(gridDim.x) - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const int n4 = dm.T * dm.d / 4;
-  const float4* y4 = reinterpret_cast<const float4*>(ws.y);
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-    const float4 v = __ldcg(y4 + i);
-    if (out_bf16) {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-      uint2 u;
-      u.x = *reinterpret_cast<uint32_t*>(&lo);
-      u.y = *reinterpret_cast<uint32_t*>(&hi);
-      reinterpret_cast<uint2*>(out)[i] = u;
-    } else {
-      reinterpret_cast<float4*>(out)[i] = v;
-    }
-  }
-}
 
 template <typename TW, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -43,6 +43,22 @@
 // bounded; the parts are added in K order. (Cutting every unit's range
 // evenly instead lowered the DRAM throughput on small-d layers: the whole-
 // unit rounds keep the CTAs in step along K.)
+//
+// Fused down projection (groups of kPathFused: the smallest row-stream
+// groups, dm.fuse_down). Once a unit's h is known, the tile's active rows
+// are final: neuron j of the tile contributes h_j W_down[e][j,:] to the
+// group's outputs and nothing else does [same list, "Fused Up-Down
+// Projection": only the active neurons' weight rows are fetched]. So right
+// after the unit's epilogue (and after its TMEM buffer is handed back to the
+// MMA warp) the four epilogue warps compact the tile's active rows and their
+// h values into shared memory, stream those rows of W_down with 16-byte
+// loads (each warp instruction reads 512 contiguous bytes of a row, 16 rows
+// in flight per thread), multiply on the CUDA cores in fp32 and add the sums
+// into Y with vector fp32 atomics (or, under direct combine, w x the sums
+// into the token's output accumulator row). The next unit's weight tiles
+// stream meanwhile, so the down rows ride on the same pass over HBM, with
+// no second kernel, no second start-up and no second walk over the union
+// bitmaps. h is rounded to bf16 first, as H^T holds it for the down kernels.
 #include "common.cuh"
 
 namespace moe {
@@ -60,6 +76,7 @@ struct UnitInfo {
   int F_e;
   int wrow;       // first weight row in the 2-D [experts*F][d] view
   int gate_only;  // gate score and a GEMV group: the up projection is left to the sparse kernel
+  int fused;      // kPathFused: this kernel also does the unit's down projection
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, int n_rg,
@@ -77,7 +94,9 @@ __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, 
     ui.shared = 1;
   }
   ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
-  ui.gate_only = p.dm.sparse_up && __ldcg(p.ws.group_path + g) == kPathGemv;
+  const int path = __ldcg(p.ws.group_path + g);
+  ui.gate_only = p.dm.sparse_up && path == kPathGemv;
+  ui.fused = path == kPathFused;
   ui.F_e = ui.shared ? p.dm.Fs : p.dm.F;
   const int e_local = ui.shared ? ui.gr.expert - p.dm.E : ui.gr.expert;
   ui.wrow = e_local * ui.F_e + ui.nt * kNeuronTile;
@@ -94,8 +113,17 @@ __device__ __forceinline__ int group_of_unit(int u, int n_rg, int tiles_r, int t
 // one; the n_units mod G leftover units are then cut along K, each into at
 // most kMaxParts parts, over the first P = min(G, leftover x kMaxParts) CTAs:
 // CTA c < P takes iterations [base + Wr c / P, base + Wr (c+1) / P) of the
-// Wr = leftover x K-blocks iterations that start at base.
+// Wr = leftover x K-blocks iterations that start at base. Only a short last
+// round is cut (fewer leftover units than half the grid): a last round that
+// fills most of the grid runs as whole units (measured on the Mixtral-shaped
+// layer: cutting 192 leftover units of 296 slots cost 7 us at T = 8, cutting
+// 8 leftover units saved 15-20 us at T = 32 and 64).
 constexpr int kMaxParts = 4;
+
+__device__ __forceinline__ int whole_units(int n_units, int split) {
+  const int G = gridDim.x;
+  return split && 2 * (n_units % G) < G ? n_units / G * G : n_units;
+}
 
 struct Segs {
   int u, n_full, KB;   // whole units: next one, and how many are whole
@@ -106,7 +134,7 @@ __device__ __forceinline__ Segs segs_begin(int n_units, int KB, int split) {
   Segs s;
   s.KB = KB;
   s.u = blockIdx.x;
-  s.n_full = split ? n_units / gridDim.x * gridDim.x : n_units;
+  s.n_full = whole_units(n_units, split);
   const int left = n_units - s.n_full;
   const int P = min((int)gridDim.x, left * kMaxParts);
   s.i = s.end = 0;
@@ -136,7 +164,7 @@ __device__ __forceinline__ bool segs_next(Segs& s, int& u, int& kb0, int& kb1) {
 
 // CTA holding leftover iteration i.
 __device__ __forceinline__ int cta_of_iter(long long i, int n_units, int KB) {
-  const int n_full = n_units / gridDim.x * gridDim.x;
+  const int n_full = whole_units(n_units, 1);  // only called for cut units
   const int left = n_units - n_full;
   const int P = min((int)gridDim.x, left * kMaxParts);
   const long long base = (long long)n_full * KB, Wr = (long long)left * KB;
@@ -155,12 +183,13 @@ __device__ __forceinline__ float* part_ptr(const GateUpTcParams& p, int slot, in
 // neuron row: masked h to H^T, warp ballots into the union word and counts.
 // The score is |h| or, with the gate score, |SiLU(g)|; a gate-only unit
 // (sparse up projection to follow) stores the masked SiLU(g) in place of h.
+// hv receives the masked values (columns past m hold values of padding rows).
 __device__ __forceinline__ void epi_chunk(const GateUpTcParams& p, const UnitInfo& ui, int word,
                                           int c0, int m, float tau, const float (&gv)[16],
                                           const float (&uv)[16], __nv_bfloat16* row,
-                                          uint32_t& uni, unsigned long long& nact, int lane) {
+                                          uint32_t& uni, unsigned long long& nact, int lane,
+                                          float (&hv)[16]) {
   const int fw = p.dm.fw;
-  float hv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int c = c0 + i;
@@ -208,7 +237,273 @@ __device__ __forceinline__ void epi_finish(const GateUpTcParams& p, const UnitIn
 // The four epilogue warps only (named barrier 1).
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// ------------------------------------------------------------ fused down projection
+
+// Shared-memory scratch of one unit's fused down projection: the tile's
+// active rows in neuron order with their h values (bf16-rounded, zero for
+// the tokens where the row is inactive).
+struct FuseScratch {
+  uint64_t bar[2];            // bulk-copy halves of the ring (last unit of a CTA)
+  float h[kNeuronTile][kFuseTokens];
+  uint8_t rows[kNeuronTile];  // neuron index within the tile
+  int cnt[4];                 // active rows of each epilogue warp's 32 neurons
+};
+constexpr int kFuseCols = 8;      // bf16 columns per thread and load (16 bytes)
+constexpr int kFuseInFlight = 16;  // row loads in flight per thread
+
+// Epilogue warps: place this warp's active neurons (bits of uni; hv their h
+// values, token t in hv[t]) at their rank among the tile's active rows.
+// Returns the tile's active row count. Every epilogue warp calls it.
+__device__ __forceinline__ int fuse_compact(FuseScratch& fs, uint32_t uni,
+                                            const float (&hv)[kFuseTokens], int m, int q,
+                                            int lane) {
+  if (lane == 0) fs.cnt[q] = __popc(uni);
+  epi_sync();
+  int off = 0, R = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int c = fs.cnt[w];
+    off += w < q ? c : 0;
+    R += c;
+  }
+  if ((uni >> lane) & 1u) {
+    const int pos = off + __popc(uni & ((1u << lane) - 1u));
+    fs.rows[pos] = static_cast<uint8_t>(32 * q + lane);
+#pragma unroll
+    for (int t = 0; t < kFuseTokens; ++t)
+      fs.h[pos][t] = t < m ? __bfloat162float(__float2bfloat16_rn(hv[t])) : 0.f;
+  }
+  epi_sync();
+  return R;
+}
+
+// acc[t][8 k + i] += h[t] * w[i] for the 8 bf16 values w of v.
+template <int MT, int KC>
+__device__ __forceinline__ void fuse_fma(float (&acc)[MT][KC * kFuseCols], int k, const uint4& v,
+                                         const float* h) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  float w[kFuseCols];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // bf16 -> fp32: the high half of a 32-bit word
+    w[2 * i] = __uint_as_float(u[i] << 16);
+    w[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+  float hh[MT];
+  if constexpr (MT == 4) {
+    const float4 h4 = *reinterpret_cast<const float4*>(h);
+    hh[0] = h4.x; hh[1] = h4.y; hh[2] = h4.z; hh[3] = h4.w;
+  } else {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) hh[t] = h[t];
+  }
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int i = 0; i < kFuseCols; ++i)
+      acc[t][k * kFuseCols + i] = fmaf(hh[t], w[i], acc[t][k * kFuseCols + i]);
+}
+
+// The unit's down projection over its R compacted rows, by the 128 epilogue
+// threads (tid 0..127). Thread tid owns columns 8 tid + 1024 k + [0, 8) for
+// k < KC of every 1024 KC-column block of d and the group's MT token slots
+// (m <= MT). Each batch issues kFuseInFlight 16-byte loads (kFuseInFlight /
+// KC rows, KC pieces of 2 KB of each) before using the first: with KC = 4 the
+// 128 threads request whole 8 KB rows (d = 4096) at once, which streams
+// faster than 2 KB pieces of many rows; the accumulators (MT x KC x 8) stay
+// at 32 registers.
+template <int MT, int KC>
+__device__ void fuse_cols(const GateUpTcParams& p, const UnitInfo& ui, const FuseScratch& fs,
+                          int R, int tid) {
+  constexpr int RB = kFuseInFlight / KC;  // rows per batch
+  const int d = p.dm.d, m = ui.gr.m;
+  const __nv_bfloat16* W = (ui.shared ? p.wds : p.wd) + static_cast<size_t>(ui.wrow) * d;
+  float* yrow[MT];
+  float wt[MT];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+    yrow[t] = nullptr;
+    wt[t] = 1.f;
+    if (t < m) {
+      int tok = ui.gr.slot0 + t;
+      if (p.dm.direct_combine) slot_target(p.dm, p.ws, ui.gr.slot0 + t, tok, wt[t]);
+      yrow[t] = p.ws.y + static_cast<size_t>(tok) * d;
+    }
+  }
+  for (int c0 = tid * kFuseCols; c0 < d; c0 += 128 * kFuseCols * KC) {
+    float acc[MT][KC * kFuseCols];
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int i = 0; i < KC * kFuseCols; ++i) acc[t][i] = 0.f;
+    const __nv_bfloat16* wc = W + c0;
+    for (int r = 0; r < R; r += RB) {
+      // all loads of the batch are issued before the first is used (rows past
+      // R re-read the last row, which is not multiplied)
+      uint4 v[RB][KC];
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const int rr = min(r + u, R - 1);
+        const __nv_bfloat16* wr = wc + static_cast<size_t>(fs.rows[rr]) * d;
+#pragma unroll
+        for (int k = 0; k < KC; ++k) v[u][k] = ld_stream_v4(wr + k * 128 * kFuseCols);
+      }
+#pragma unroll
+      for (int u = 0; u < RB; ++u)
+        if (r + u < R)
+#pragma unroll
+          for (int k = 0; k < KC; ++k) fuse_fma<MT, KC>(acc, k, v[u][k], fs.h[r + u]);
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+      if (t < m) {
+        const float w = wt[t];
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+          float* y = yrow[t] + c0 + k * 128 * kFuseCols;
+          const float* a = acc[t] + k * kFuseCols;
+          red_add_v4(y, w * a[0], w * a[1], w * a[2], w * a[3]);
+          red_add_v4(y + 4, w * a[4], w * a[5], w * a[6], w * a[7]);
+        }
+      }
+  }
+}
+
+constexpr int kFuseHalfMax = 32;  // rows per half of the ring in the bulk path
+
+// The CTA's last unit (its weight ring is idle: every copy landed and every
+// MMA that read the ring has completed): the unit's R active rows, whole
+// (d = 1024 KC, rows of 2 KB KC), come into the ring by bulk copies, H rows
+// per half, the two halves alternating, so that up to 2 H rows are in flight
+// while the 128 threads multiply the landed half from shared memory (thread
+// tid reads 16 bytes at 2 KB k + 16 tid of a row: conflict-free). Thread tid
+// owns the same columns as in fuse_cols; MT <= 2 keeps the accumulators at
+// <= 64 registers.
+template <int MT, int KC>
+__device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, FuseScratch& fs,
+                               int R, int tid, uint8_t* ring, uint32_t ring_bytes,
+                               volatile int* abort_flag) {
+  const int d = p.dm.d, m = ui.gr.m;
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 2;
+  const int H = min(static_cast<int>(ring_bytes / row_bytes) / 2, kFuseHalfMax);
+  const int nb = (R + H - 1) / H;
+  const __nv_bfloat16* W = (ui.shared ? p.wds : p.wd) + static_cast<size_t>(ui.wrow) * d;
+  auto issue = [&](int b) {  // thread 0: batch b into half b & 1
+    const int h = b & 1, r0 = b * H, n = min(H, R - r0);
+    mbar_arrive_expect_tx(&fs.bar[h], static_cast<uint32_t>(n) * row_bytes);
+    for (int i = 0; i < n; ++i)
+      bulk_load(smem_u32(ring + static_cast<size_t>(h * H + i) * row_bytes),
+                W + static_cast<size_t>(fs.rows[r0 + i]) * d, row_bytes, smem_u32(&fs.bar[h]));
+  };
+  int issued = 0;  // thread 0: batches issued
+  if (tid == 0) {
+    issue(0);
+    issued = 1;
+    if (nb > 1) {
+      issue(1);
+      issued = 2;
+    }
+  }
+  float acc[MT][KC * kFuseCols];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int i = 0; i < KC * kFuseCols; ++i) acc[t][i] = 0.f;
+  bool ok = true;
+  for (int b = 0; b < nb; ++b) {
+    // every epilogue warp runs every batch (named barrier), skipping the
+    // work once a wait has failed
+    const int h = b & 1;
+    if (ok && !warp_wait(&fs.bar[h], (b >> 1) & 1, abort_flag, p.ws.status)) ok = false;
+    if (ok) {
+      const int r0 = b * H, n = min(H, R - r0);
+      const uint8_t* base = ring + static_cast<size_t>(h * H) * row_bytes + tid * 16;
+      for (int i = 0; i < n; ++i) {
+        const float* hr = fs.h[r0 + i];
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(base + i * row_bytes + k * 2048);
+          fuse_fma<MT, KC>(acc, k, v, hr);
+        }
+      }
+    }
+    epi_sync();  // the half is read: it may be refilled
+    if (tid == 0 && b + 2 < nb && !*abort_flag) {
+      issue(b + 2);
+      issued = b + 3;
+    }
+  }
+  if (tid == 0 && *abort_flag) {
+    // copies still in flight land before the CTA may exit: wait (bounded) for
+    // the last batch issued on each half
+    volatile int never = 0;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int lb = issued - 1 - ((issued - 1 - hh) & 1);
+      if (lb >= 0) mbar_wait(&fs.bar[hh], (lb >> 1) & 1, &never, p.ws.status);
+    }
+  }
+  if (!ok) return;
+  const int c0 = tid * kFuseCols;
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+    if (t < m) {
+      int tok = ui.gr.slot0 + t;
+      float w = 1.f;
+      if (p.dm.direct_combine) slot_target(p.dm, p.ws, ui.gr.slot0 + t, tok, w);
+      float* yrow = p.ws.y + static_cast<size_t>(tok) * d;
+#pragma unroll
+      for (int k = 0; k < KC; ++k) {
+        float* y = yrow + c0 + k * 128 * kFuseCols;
+        const float* a = acc[t] + k * kFuseCols;
+        red_add_v4(y, w * a[0], w * a[1], w * a[2], w * a[3]);
+        red_add_v4(y + 4, w * a[4], w * a[5], w * a[6], w * a[7]);
+      }
+    }
+}
+
+// A kPathFused unit after its epilogue, every epilogue warp: compaction, the
+// down projection of the active rows, and a barrier that frees the scratch.
+// uni / hv: this warp's union word and its lane's h values (token t in
+// hv[t]); a warp whose wait failed passes uni = 0. last: the CTA has no
+// further unit (the ring may be used for bulk copies of the rows).
+__device__ __forceinline__ void fuse_unit(const GateUpTcParams& p, const UnitInfo& ui,
+                                          FuseScratch& fs, uint32_t uni,
+                                          const float (&hv)[kFuseTokens], int q, int lane,
+                                          bool last, uint8_t* ring, uint32_t ring_bytes,
+                                          volatile int* abort_flag) {
+  const int m = ui.gr.m;
+  const int R = fuse_compact(fs, uni, hv, m, q, lane);
+  const int tid = 32 * q + lane;
+  if (R > 0) {
+    const int d = p.dm.d;
+    const bool bulk = last && m <= 2 && ring_bytes >= 4u * static_cast<uint32_t>(d);
+    if (bulk && d == 4096) {
+      if (m == 1) fuse_rows_bulk<1, 4>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
+      else fuse_rows_bulk<2, 4>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
+    } else if (bulk && d == 2048) {
+      fuse_rows_bulk<2, 2>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
+    } else if (bulk && d == 1024) {
+      fuse_rows_bulk<2, 1>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
+    } else if (m == 1 && d % 4096 == 0) {
+      fuse_cols<1, 4>(p, ui, fs, R, tid);
+    } else if (m <= 2 && d % 2048 == 0) {
+      fuse_cols<2, 2>(p, ui, fs, R, tid);
+    } else if (m == 1) {
+      fuse_cols<1, 1>(p, ui, fs, R, tid);
+    } else if (m == 2) {
+      fuse_cols<2, 1>(p, ui, fs, R, tid);
+    } else {
+      fuse_cols<4, 1>(p, ui, fs, R, tid);
+    }
+  }
+  if (tid == 0) {  // W_down rows this unit read
+    atomicAdd(p.ws.counters + kCntDownRows, static_cast<unsigned long long>(R));
+    atomicAdd(p.ws.counters + kCntFusedRows, static_cast<unsigned long long>(R));
+  }
+  epi_sync();
+}
+
+// Two CTAs per SM for groups of <= 32 tokens: at most 168 registers a thread.
+__global__ void __launch_bounds__(kThreads, 2)
     gate_up_tc_kernel(const __grid_constant__ GateUpTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -228,6 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* fix_ok = abort_flag + 1;  // the parked unit's parts are all published
+  FuseScratch* fscr = reinterpret_cast<FuseScratch*>(
+      (reinterpret_cast<uintptr_t>(tmem_slot) + 16 + 15) & ~static_cast<uintptr_t>(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -242,6 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tempty + b, 4);
     }
     mbar_init(drain, 1);
+    if (p.dm.fuse_down) {
+      mbar_init(&fscr->bar[0], 1);
+      mbar_init(&fscr->bar[1], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -408,6 +709,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && !warp_wait(tfull + b, tph, abort_flag, p.ws.status)) ok = false;
       const bool whole = kb0 == 0 && kb1 == KB;
       const bool last_part = !whole && kb1 == KB;
+      uint32_t uni = 0;       // this warp's union word (fused down projection)
+      float hv[kFuseTokens];  // this lane's masked h of the first tokens
+#pragma unroll
+      for (int i = 0; i < kFuseTokens; ++i) hv[i] = 0.f;
       if (ok) {
         tc_fence_after();
         const float tau = ui.shared ? p.tau_shared : p.tau;
@@ -417,7 +722,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* row = ht + static_cast<size_t>(j) * ld + ui.gr.slot0;
         const uint32_t tg = tmem_base + lane_off + b * buf_cols;
         const uint32_t tu = tg + n_max;
-        uint32_t uni = 0;
         unsigned long long nact = 0;
         const int slot = last_part ? gridDim.x + blockIdx.x : blockIdx.x;
         for (int c0 = 0; c0 < N; c0 += 16) {
@@ -438,7 +742,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uv[i] = __uint_as_float(ur[i]);
           }
           if (whole) {
-            epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane);
+            float hc[16];
+            epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane, hc);
+            if (c0 == 0)
+#pragma unroll
+              for (int i = 0; i < kFuseTokens; ++i) hv[i] = hc[i];
           } else {  // a part of a split unit: park its sums
             float4* pg = reinterpret_cast<float4*>(part_ptr(p, slot, 0, c0 / 16, row_i));
             float4* pu = reinterpret_cast<float4*>(part_ptr(p, slot, 1, c0 / 16, row_i));
@@ -459,6 +767,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + b);
+      // the TMEM buffer is back with the MMA warp: the next unit's tiles
+      // stream while this one's active W_down rows are read
+      if (whole && ui.fused) {
+        Segs rest = sg;  // no segment and no parked unit after this one: the ring is idle
+        int u2, a2, b2;
+        const bool last = park_u < 0 && !segs_next(rest, u2, a2, b2);
+        fuse_unit(p, ui, *fscr, ok ? uni : 0u, hv, q, lane, last, smem, stages * stage_bytes,
+                  abort_flag);
+      }
       if (!whole && !last_part) {
         // an earlier part: publish it for the CTA that holds the unit's end
         __threadfence();
@@ -491,6 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* row = ht + static_cast<size_t>(j) * ld + ui.gr.slot0;
         uint32_t uni = 0;
         unsigned long long nact = 0;
+        float hv[kFuseTokens];
         for (int c0 = 0; c0 < N; c0 += 16) {
           float gv[16], uv[16];
 #pragma unroll
@@ -506,11 +824,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               uv[4 * i] += c.x; uv[4 * i + 1] += c.y; uv[4 * i + 2] += c.z; uv[4 * i + 3] += c.w;
             }
           }
-          epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane);
+          float hc[16];
+          epi_chunk(p, ui, word, c0, m, tau, gv, uv, row, uni, nact, lane, hc);
+          if (c0 == 0)
+#pragma unroll
+            for (int i = 0; i < kFuseTokens; ++i) hv[i] = hc[i];
         }
         epi_finish(p, ui, g, word, uni, nact, lane);
         if (q == 0 && lane == 0)
           atomicAdd(p.ws.counters + kCntGateUpRows, (ui.gate_only ? 1ull : 2ull) * kNeuronTile);
+        if (ui.fused)
+          fuse_unit(p, ui, *fscr, uni, hv, q, lane, true, smem, stages * stage_bytes, abort_flag);
       }
     }
   }
@@ -521,17 +845,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
+  // direct combine with no row-stream launch after this one: the last CTA
+  // writes out from the accumulator rows
+  if (p.dm.fuse_finish) direct_finish(p.dm, p.ws, p.out, p.out_bf16);
 }
 
 }  // namespace
 
-size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks) {
+size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks, bool fuse) {
   const size_t stage_bytes = 2 * kABytes + static_cast<size_t>(b_blocks) * n_max * 128;
-  return 1024 + stages * stage_bytes + (2 * stages + 5) * sizeof(uint64_t) + 16;
+  return 1024 + stages * stage_bytes + (2 * stages + 5) * sizeof(uint64_t) + 16 +
+         (fuse ? 16 + sizeof(FuseScratch) : 0);
 }
 
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st) {
-  const cudaError_t e = smem_limit(gate_up_tc_kernel, 227 * 1024);
+  // the launch's own size: the kernel has a little static shared memory too,
+  // and the opt-in limit covers both
+  const cudaError_t e = smem_limit(gate_up_tc_kernel, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_k(gate_up_tc_kernel, grid, kThreads, smem, st, p);
 }

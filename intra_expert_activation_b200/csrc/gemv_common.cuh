@@ -25,15 +25,6 @@ constexpr int kSmemBudget = 200 * 1024;  // ring of stages (6 stages of 4 KB blo
 constexpr int kListRows = 256;       // producer's row list (uint16 neuron indices)
 constexpr int kTight = 4096;         // barrier probes before sleeping: stages arrive every few us
 
-__device__ __forceinline__ void red_add_v2(float* p, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
-}
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
 // Packed pair of fp32 values and d = a * b + d on both halves.
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
   uint64_t r;
@@ -73,17 +64,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 // barrier's expected count includes this arrival).
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16) from global to shared memory,
-// completion counted on bar as transaction bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
 }
 
 // Stage geometry for a row of row_bytes: the column block (<= block_max),

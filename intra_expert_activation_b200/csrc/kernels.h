@@ -11,11 +11,12 @@
 
 namespace moe {
 
-// Every kernel is launched with programmatic stream serialization: its CTAs
-// may be scheduled as soon as every CTA of the previous kernel on the stream
-// has started (each signals it at its start), and they call grid_dep_wait()
-// (griddepcontrol.wait) before touching global memory, so the launch latency
-// overlaps the predecessor's run. MOE_PDL=0 in the environment turns it off.
+// Every kernel is launched with programmatic stream serialization: its
+// launch is set up while the previous kernel on the stream drains (its CTAs
+// are scheduled as the predecessor's CTAs exit), and they call
+// grid_dep_wait() (griddepcontrol.wait) before touching global memory, so
+// part of the launch latency overlaps the predecessor's tail. MOE_PDL=0 in
+// the environment turns it off.
 bool pdl_enabled();
 
 template <typename... KArgs, typename... Args>
@@ -85,10 +86,19 @@ enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUse
 // counters[] (u64), reset by the router's scan every forward
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
                kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
-               kCntUpRows = 8, kCntGateUpRows = 9, kCntGemvRows = 10, kCntWords = 11 };
+               kCntUpRows = 8, kCntGateUpRows = 9, kCntGemvRows = 10, kCntFusedRows = 11,
+               kCntWords = 12 };
 
-// kPathCand: GEMV or all-rows TC, chosen after gate/up (cand_takes_gemv)
-enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3, kPathCand = 4 };
+// kPathCand: GEMV or all-rows TC, chosen after gate/up (cand_takes_gemv).
+// kPathFused: a row-stream group whose down projection the gate/up kernel
+// does itself, per 128-neuron tile, right after the tile's epilogue
+// (Dims::fuse_down); it is on neither down kernel's list.
+enum GroupPath { kPathNone = 0, kPathGemv = 1, kPathTcGather = 2, kPathTcAll = 3, kPathCand = 4,
+                 kPathFused = 5 };
+
+// Groups of at most kFuseTokens tokens on the row stream are fused into the
+// gate/up kernel when Dims::fuse_down is set.
+constexpr int kFuseTokens = 4;
 
 // Requested path (mirrors moe_path in the public header).
 enum Mode { kModeAuto = 0, kModeDense = 1, kModeGemv = 2, kModeTc = 3, kModeTcAll = 4 };
@@ -127,6 +137,13 @@ struct Dims {
   // rows Y[0..T) (zeroed by the router) and its last CTA writes out; no
   // combine launch
   int direct_combine;
+  // 1: row-stream groups of <= kFuseTokens tokens take kPathFused: the gate/up
+  // kernel multiplies each tile's active W_down rows by its h values and adds
+  // the sums into Y (bf16 layers, |h| score or a dense up projection)
+  int fuse_down;
+  // 1 (with direct_combine): no row-stream launch follows the gate/up kernel,
+  // so its last CTA (a ticket) writes out from the accumulator rows
+  int fuse_finish;
 };
 
 constexpr int kDirectMax = 16;  // tokens up to which the row stream combines directly
@@ -211,6 +228,10 @@ struct GateUpTcParams {
   uint32_t tmem_cols;          // allocated TMEM columns
   int split;                   // 1: the leftover units after whole rounds are cut along K
   int b_blocks;                // activation regions per stage: 2 with the gate score, else 1
+  const __nv_bfloat16* wd;     // [E*F][d] W_down (fused down projection, kPathFused groups)
+  const __nv_bfloat16* wds;    // [S*Fs][d] shared experts' W_down
+  void* out;                   // [T][d] layer output (dm.fuse_finish)
+  int out_bf16;                // out's type: 1 bf16, 0 fp32
 };
 
 // ------------------------------------------------------------ down (tcgen05)
@@ -233,7 +254,9 @@ bool route_is_small(const Dims& dm);
 cudaError_t launch_permute(const Dims& dm, const Workspace& ws, const void* x, bool bf16,
                            cudaStream_t st);
 cudaError_t launch_gate_up_tc(const GateUpTcParams& p, int grid, size_t smem, cudaStream_t st);
-size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks);
+// Dynamic shared memory of a gate/up launch; `fuse`: room for the fused
+// down projection's row list and h values.
+size_t gate_up_tc_smem_bytes(int n_max, int stages, int b_blocks, bool fuse);
 cudaError_t launch_updown_gemv(const Dims& dm, const Workspace& ws, const void* Wu,
                                const void* Wus, const void* Wd, const void* Wds, const void* x,
                                bool bf16, int n_sms, cudaStream_t st);

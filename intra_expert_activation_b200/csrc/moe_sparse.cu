@@ -65,6 +65,17 @@ bool split_enabled() {
   }();
   return on;
 }
+
+// Down projection of the smallest row-stream groups inside the gate/up kernel
+// (MOE_FUSE_DOWN=0 turns it off and sends them to the row-stream kernel, for
+// comparisons).
+bool fuse_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_FUSE_DOWN");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 }  // namespace moe
 
 namespace {
@@ -149,6 +160,7 @@ struct Layout {
   Dims cap;
   size_t off[32];
   size_t total;
+  long long sk_cols = 0;  // gate/up split partials: capacity in CTAs x MMA N (columns)
 };
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
@@ -251,13 +263,15 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bTcList] = sizeof(int) * c.groups_max;
   sz[bYZero] = sizeof(int) * (c.E + 1);
   sz[bSlotW] = sizeof(float) * c.slots_routed;
-  // gate/up split units (bf16): one flag per CTA and two partial slots per CTA,
-  // for up to 2 x 160 CTAs (2 per SM) when the groups hold <= 32 tokens, else 160
+  // gate/up split units (bf16): one flag per CTA and two partial slots per CTA
+  // of MMA N columns each: 2 x 160 CTAs (2 per SM) for groups of <= 32 tokens,
+  // 160 CTAs for larger ones (cut only up to 64 tokens)
   {
-    const int nm = std::min(roundup(std::min(c.T, moe::kGroupMax), 16), 64);  // cut only <= 64
-    c.sk_ctas = bf16 ? (nm <= 32 ? 320 : 160) : 0;
+    const int nm = std::min(roundup(std::min(c.T, moe::kGroupMax), 16), 64);
+    c.sk_ctas = bf16 ? 320 : 0;
+    L.sk_cols = bf16 ? std::max(320LL * std::min(nm, 32), 160LL * nm) : 0;
     sz[bSkFlags] = sizeof(int) * (size_t)c.sk_ctas;
-    sz[bSkPart] = sizeof(float) * (size_t)2 * c.sk_ctas * 2 * moe::kNeuronTile * nm;
+    sz[bSkPart] = sizeof(float) * (size_t)2 * L.sk_cols * 2 * moe::kNeuronTile;
   }
   // tensor-core down units cut along K (bf16, groups of <= 64 tokens): a
   // ticket per unit and a partial-sum block per part unit
@@ -532,20 +546,50 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
                   cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
   const bool dense = c->desc.path == MOE_PATH_DENSE;
   const int mode = c->desc.path;
-  const bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
+  const int tmax = std::min(T, moe::kGroupMax);  // no group holds more tokens
+  bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
-                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
-                         std::min(T, moe::kGroupMax) <= cap.gemv_max);
-  const int n_max = roundup(std::min(T, moe::kGroupMax), 16);
+                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) && tmax <= cap.gemv_max);
+  const int n_max = roundup(tmax, 16);
   // gate score: the GEMV groups' up projection is sparse (only the active
   // rows) when the threshold can leave rows out; at tau <= 0 every neuron
   // whose SiLU(g) is non-zero is active, so the dense up projection (gate and
   // up in one GEMM) reads the same rows faster
   dm.sparse_up = dm.score_gate && tau > 0.f ? 1 : 0;
-  // every group on the |h|-score row stream and a small batch: the row stream
-  // combines directly into the output (no combine launch)
+  // gate/up units (group x 128-neuron tile) at most, and the launch's CTAs
+  const int gu_units_max =
+      (P / moe::kGroupMax + std::min(cap.E, P)) * (cap.F / moe::kNeuronTile) +
+      cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) * (cap.Fs / moe::kNeuronTile);
+  const int gu_ctas_per_sm = n_max <= 32 ? 2 : 1;
+  // (with fewer units than CTA slots, one unit per CTA: cutting the units
+  // along K over the full grid to even out the SMs measured slower, 120 vs
+  // 108 us per layer at T = 1 on the Mixtral-shaped layer)
+  const int gu_grid = std::max(1, std::min(gu_units_max, gu_ctas_per_sm * c->n_sms));
+  // row-stream groups of <= kFuseTokens tokens: down projection inside the
+  // gate/up kernel (bf16, dense up projection, automatic or dense path), when
+  // no CTA has more than one unit to finish, so that the down rows stream
+  // after the CTA's weight tiles. With several units per CTA the down rows
+  // would share HBM with the next units' tiles through 16-byte loads, which
+  // stream slower than the row-stream kernel's bulk copies (measured at
+  // T = 8 on the Mixtral-shaped layer: 384 vs 363 us per layer); with one
+  // unit per CTA the fusion saves the row-stream launch and its start-up
+  // (T = 1: 110 vs 120 us).
+  dm.fuse_down = c->bf16 && !dm.sparse_up && (mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
+                 gu_units_max <= gu_grid && moe::fuse_enabled() ? 1 : 0;
+  if (dm.fuse_down) {
+    // the row-stream kernel is only needed for groups the fusion leaves:
+    // unfused row-stream groups and candidates
+    const bool big_gemv = std::min(tmax, cap.gemv_max) > moe::kFuseTokens;
+    const bool cand = cap.gemv_cand > cap.gemv_max && tmax > cap.gemv_max;
+    need_gemv = big_gemv || cand;
+  }
+  // every group on the |h|-score row stream (fused or not) and a small
+  // batch: the row stream combines directly into the output (no combine
+  // launch); with no row-stream launch the gate/up kernel writes out
   const bool out_bf16 = c->bf16 && !c->desc.out_f32;
-  dm.direct_combine = need_gemv && !need_tc && !dm.sparse_up && T <= moe::kDirectMax ? 1 : 0;
+  dm.direct_combine =
+      (need_gemv || dm.fuse_down) && !need_tc && !dm.sparse_up && T <= moe::kDirectMax ? 1 : 0;
+  dm.fuse_finish = dm.direct_combine && !need_gemv ? 1 : 0;
   // the tensor-core down launch's grid is fixed here: the router's layout
   // and the kernel both derive the units' K parts from it
   const int tc_ctas_per_sm = n_max <= 64 ? 2 : 1;
@@ -608,23 +652,29 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     const uint32_t buf = 2u * n_max;
     p.nbuf = 2 * buf <= 512 ? 2 : 1;
     p.tmem_cols = pow2_at_least(p.nbuf * buf);
-    const int ctas_per_sm = n_max <= 32 ? 2 : 1;
-    const size_t budget = ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
+    const size_t budget = gu_ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
     // gate score: gate-only units take two K-blocks per stage; the second
     // activation region costs a stage of the pipeline when groups are larger
     // than 16 tokens (measured at T = 32: 303 -> 358 us), so only below that
     p.b_blocks = dm.sparse_up && n_max <= 16 ? 2 : 1;
     const size_t stage_bytes = 32768 + (size_t)p.b_blocks * n_max * 128;
-    p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
-    const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages, p.b_blocks);
-    const int units_max = (P / moe::kGroupMax + std::min(cap.E, P)) * (cap.F / moe::kNeuronTile) +
-                          cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) *
-                              (cap.Fs / moe::kNeuronTile);
-    const int grid = std::max(1, std::min(units_max, ctas_per_sm * c->n_sms));
+    const size_t fuse_bytes =
+        moe::gate_up_tc_smem_bytes(n_max, 0, p.b_blocks, dm.fuse_down) -
+        moe::gate_up_tc_smem_bytes(n_max, 0, p.b_blocks, false);
+    p.stages = (int)std::min<size_t>(8, (budget - 2048 - fuse_bytes) / stage_bytes);
+    const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages, p.b_blocks, dm.fuse_down);
+    p.wd = static_cast<const __nv_bfloat16*>(W_down);
+    p.wds = static_cast<const __nv_bfloat16*>(c->Wds);
+    p.out = out;
+    p.out_bf16 = out_bf16 ? 1 : 0;
+    const int grid = gu_grid;
     // leftover units are cut along K only for groups of <= 64 tokens: with
     // 128-token groups (prefill) the parts' accumulators cost more than the
     // uneven last round (measured: +24 us at T = 4096, d = 2048)
-    p.split = moe::split_enabled() && n_max <= 64 && grid <= cap.sk_ctas ? 1 : 0;
+    p.split = moe::split_enabled() && n_max <= 64 && grid <= cap.sk_ctas &&
+                      (long long)grid * n_max <= c->lay.sk_cols
+                  ? 1
+                  : 0;
     e = moe::launch_gate_up_tc(p, grid, smem, st);
   } else {
     e = moe::launch_gate_up_simt(dm, c->ws, static_cast<const float*>(x),
@@ -738,6 +788,7 @@ moe_status moe_sparse_get_stats(moe_sparse_ctx* c, moe_stats* s, void* stream) {
   s->up_rows_read = (int64_t)cnt[moe::kCntUpRows];
   s->gate_up_rows_read = (int64_t)cnt[moe::kCntGateUpRows];
   s->down_rows_gemv = (int64_t)cnt[moe::kCntGemvRows];
+  s->down_rows_fused = (int64_t)cnt[moe::kCntFusedRows];
   return MOE_OK;
 }
 

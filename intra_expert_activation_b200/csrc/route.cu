@@ -80,7 +80,8 @@ __device__ __forceinline__ int group_path_of(const Dims& dm, int m) {
   if (dm.no_tc || dm.mode == kModeGemv) return kPathGemv;
   if (dm.mode == kModeTc) return kPathTcAll;  // gathered or not: decided by the union scan
   if (dm.mode == kModeTcAll) return kPathTcAll;
-  if (m <= dm.gemv_max) return kPathGemv;  // auto and dense
+  if (m <= dm.gemv_max)  // auto and dense; the smallest groups inside the gate/up kernel
+    return dm.fuse_down && m <= kFuseTokens ? kPathFused : kPathGemv;
   return m <= dm.gemv_cand ? kPathCand : kPathTcAll;
 }
 
@@ -193,7 +194,14 @@ __device__ __forceinline__ void block_exclusive_scan(int (&v)[N], int (&total)[N
 __device__ __forceinline__ int on_gemv_list(int path) {
   return path == kPathGemv || path == kPathCand;
 }
-__device__ __forceinline__ int on_tc_list(int path) { return path != kPathGemv; }
+__device__ __forceinline__ int on_tc_list(int path) {
+  return path == kPathTcAll || path == kPathTcGather || path == kPathCand;
+}
+// The group's Y rows receive atomic adds (row stream, fused or not), so they
+// start at zero.
+__device__ __forceinline__ int adds_into_y(int path) {
+  return on_gemv_list(path) || path == kPathFused;
+}
 
 // ng groups of gsz tokens (a multiple of kSlotAlign; the last one has
 // m_last), each at most kGroupMax.
@@ -241,7 +249,8 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
   // ---- pass 1: slots, groups, GEMV / TC list positions
   // kGemv / kTc: list lengths (a candidate group is in both lists); kCand:
   // candidates; kTcSharedDef: shared groups whose all-rows TC path is fixed now
-  enum { kSlots, kGroups, kGemv, kTc, kCand, kRoutedGroups, kTcSharedDef, kTouched, kN };
+  // kFused: groups whose down projection runs inside the gate/up kernel
+  enum { kSlots, kGroups, kGemv, kTc, kCand, kRoutedGroups, kTcSharedDef, kTouched, kFused, kN };
   int v[kN] = {}, tot[kN];
   EntryCut cut[kPer];
 #pragma unroll
@@ -254,6 +263,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     const int n_gemv = (c.ng - 1) * on_gemv_list(c.path_full) + on_gemv_list(c.path_last);
     const int n_tc = (c.ng - 1) * on_tc_list(c.path_full) + on_tc_list(c.path_last);
     const int n_cand = (c.ng - 1) * (c.path_full == kPathCand) + (c.path_last == kPathCand);
+    v[kFused] += (c.ng - 1) * (c.path_full == kPathFused) + (c.path_last == kPathFused);
     if (q < E) {
       v[kSlots] += (c.me + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
       v[kRoutedGroups] += c.ng;
@@ -291,10 +301,8 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
           ws.groups[g] = gr;
           ws.group_path[g] = path;
           ws.union_cnt[g] = 0;
-          if (on_gemv_list(path)) {
-            any_gemv = 1;
-            ws.gemv_list[gv++] = g;
-          }
+          any_gemv |= adds_into_y(path);
+          if (on_gemv_list(path)) ws.gemv_list[gv++] = g;
           if (on_tc_list(path)) ws.tc_list[tc++] = g;
         }
       }
@@ -317,7 +325,7 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
     ws.meta[kMetaGemvCount] = tot[kGemv];
     ws.meta[kMetaTcCount] = tot[kTc];
     // candidates are counted by the down kernel that takes them
-    ws.counters[kCntGemv] = tot[kGemv] - tot[kCand];
+    ws.counters[kCntGemv] = tot[kGemv] - tot[kCand] + tot[kFused];
     ws.counters[kCntTc] = tot[kTc] - tot[kCand];
     if (dm.mode != kModeTc)  // the GEMV kernel adds its rows
       ws.counters[kCntDownRows] =
@@ -674,7 +682,7 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
       // never used: every kernel masks the columns past a group's count)
       for (int r = c; r < kSlotAlign; ++r) ws.perm[g * kSlotAlign + r] = -1;
     }
-    if (e < E) L.yzero[e] = c > 0 && on_gemv_list(group_path_of(dm, c));
+    if (e < E) L.yzero[e] = c > 0 && adds_into_y(group_path_of(dm, c));
     n_touched += __popc(bal);
   }
   const int n_groups = n_touched + S;
@@ -693,7 +701,7 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
   }
   __syncwarp();
   // GEMV and tensor-core lists in group order (a candidate is on both)
-  int n_gv = 0, n_tc = 0, n_cand = 0, n_tc_sh = 0, any_gv_sh = 0;
+  int n_gv = 0, n_tc = 0, n_cand = 0, n_tc_sh = 0, any_gv_sh = 0, n_fz = 0;
   for (int g0 = 0; g0 < n_groups; g0 += 32) {
     const int g = g0 + lane;
     const int path = g < n_groups ? L.gpath[g] : kPathNone;
@@ -707,7 +715,8 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
     n_tc += __popc(btc);
     n_cand += __popc(__ballot_sync(0xffffffffu, cand));
     n_tc_sh += __popc(__ballot_sync(0xffffffffu, tc && !cand && g >= n_touched));
-    any_gv_sh |= __ballot_sync(0xffffffffu, gv && g >= n_touched) != 0u;
+    n_fz += __popc(__ballot_sync(0xffffffffu, g < n_groups && path == kPathFused));
+    any_gv_sh |= __ballot_sync(0xffffffffu, g < n_groups && adds_into_y(path) && g >= n_touched) != 0u;
   }
   if (lane == 0) L.yzero[E] = any_gv_sh;
   // each pair's slot: its expert's block + its rank among the expert's pairs
@@ -724,7 +733,7 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
   }
   if (lane < kCntWords) {
     unsigned long long v = 0ull;
-    if (lane == kCntGemv) v = n_gv - n_cand;  // candidates are counted by the kernel that takes them
+    if (lane == kCntGemv) v = n_gv - n_cand + n_fz;  // candidates: counted by the kernel that takes them
     if (lane == kCntTc) v = n_tc - n_cand;
     if (lane == kCntDownRows && dm.mode != kModeTc)  // the GEMV kernel adds its rows
       v = (unsigned long long)(n_tc - n_cand - n_tc_sh) * dm.F +

@@ -3,6 +3,7 @@ workload at its full size, on small layers that span several tiles with
 ragged tails, with each down-projection path forced, and on edge cases."""
 
 import math
+import os
 
 import numpy as np
 import pytest
@@ -323,12 +324,15 @@ def test_mixtral_sweep(sweep, T, q):
 
 def _expected_down_rows(gpu, F):
     """Rows the automatic per-group switch reads, from the GPU's own active
-    sets: groups of <= 4 tokens stream their union; groups of 5..8 tokens
-    stream it iff 5 x union <= 4 x d_ff (one pass of 8 tokens), else all
-    d_ff rows on the tensor cores, as do larger groups."""
+    sets: groups of <= 4 tokens stream their union (inside the gate/up kernel,
+    tile by tile, unless MOE_FUSE_DOWN=0); groups of 5..8 tokens stream it
+    iff 5 x union <= 4 x d_ff (one pass of 8 tokens), else all d_ff rows on
+    the tensor cores, as do larger groups. Returns (rows, GEMV groups, TC
+    groups, candidates on the row stream, candidates on the tensor cores,
+    rows of the fused groups)."""
     act = unpack_bits(gpu["active_bits"], F)
     idx = gpu["topk_idx"].ravel()
-    rows = n_gemv = n_tc = cand_gemv = cand_tc = 0
+    rows = n_gemv = n_tc = cand_gemv = cand_tc = fused = 0
     for e in np.unique(idx):
         m = int((idx == e).sum())
         u = int(act[idx == e].any(axis=0).sum())
@@ -336,11 +340,56 @@ def _expected_down_rows(gpu, F):
             rows += u
             n_gemv += 1
             cand_gemv += m > 4
+            fused += u if m <= 4 else 0
         else:
             rows += F
             n_tc += 1
             cand_tc += m <= 8
-    return rows, n_gemv, n_tc, cand_gemv, cand_tc
+    return rows, n_gemv, n_tc, cand_gemv, cand_tc, fused
+
+
+def _fuses(shape, T):
+    """Whether a forward of T tokens fuses the down projection of its groups
+    of <= 4 tokens into the gate/up kernel: only when the gate/up launch has
+    a CTA for every possible unit (group x 128-neuron tile), two CTAs per SM
+    for groups of <= 32 tokens, and the fusion is not turned off."""
+    if os.environ.get("MOE_FUSE_DOWN") == "0":
+        return False
+    P = T * shape.top_k
+    units = (P // 128 + min(shape.n_experts, P)) * (shape.d_ff // 128)
+    if shape.n_shared:
+        units += shape.n_shared * ((T + 127) // 128) * (shape.d_ff_shared // 128)
+    per_sm = 2 if min(T, 128) <= 32 else 1
+    return units <= per_sm * torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("name,T", [("mixtral_decode", 1), ("many_small_experts", 1),
+                                    ("many_small_experts", 4), ("shared_routed_prefill", 2),
+                                    ("shared_routed_prefill", 4)])
+def test_fused_down_matches_row_stream(name, T):
+    """Small batches whose gate/up units fit one per CTA: the gate/up kernel's
+    fused down projection (automatic path) and the row-stream kernel (path
+    forced to the GEMV kernel) multiply the same bf16 h values by the same
+    W_down rows with fp32 sums in different orders, so their fp32 outputs
+    agree to fp32 rounding and read the same rows, and both match the oracle
+    (routed groups of 1-4 tokens, d = 4096 and 2048, shared experts)."""
+    if os.environ.get("MOE_FUSE_DOWN") == "0":
+        pytest.skip("fused down projection turned off")
+    wl, dw = workload_weights(name)
+    assert _fuses(wl.shape, T)  # every case here has one gate/up unit per CTA at most
+    q = wl.sparsities[0]
+    tau, ts = tau_of(name, q)
+    x = workload_tokens(wl, T)
+    fused = run_gpu(make_layer(wl.shape, 64, out_f32=True), dw, x, tau, ts)
+    gemv = run_gpu(make_layer(wl.shape, 64, path="sparse_gemv", out_f32=True), dw, x, tau, ts)
+    a, b = fused["out"], gemv["out"]
+    assert np.array_equal(fused["active_bits"], gemv["active_bits"])
+    scale = np.abs(b).max()
+    assert np.abs(a - b).max() <= 1e-5 * scale, (np.abs(a - b).max(), scale)
+    sf, sg = fused["stats"], gemv["stats"]
+    assert sf["down_rows_fused"] == sf["down_rows_read"] == sg["down_rows_gemv"] > 0
+    assert sf["down_rows_gemv"] == 0 and sg["down_rows_fused"] == 0
+    compare(fused, oracle_forward(dw, x, tau, ts), tau, ts, "bf16", dw=dw)
 
 
 def test_candidate_groups_choose_by_union(sweep):
@@ -355,9 +404,10 @@ def test_candidate_groups_choose_by_union(sweep):
         tau, _ = tau_of("mixtral_sweep", q)
         layer = make_layer(wl.shape, 512)
         gpu, _, _ = _check(layer, dw, workload_tokens(wl, 24), tau, 0.0, "bf16")
-        rows, n_gemv, n_tc, cand_gemv, cand_tc = _expected_down_rows(gpu, F)
+        rows, n_gemv, n_tc, cand_gemv, cand_tc, fused = _expected_down_rows(gpu, F)
         st = gpu["stats"]
         assert st["down_rows_read"] == rows
+        assert st["down_rows_fused"] == (fused if _fuses(wl.shape, 24) else 0)
         assert st["n_groups_gemv"] == n_gemv and st["n_groups_tc_allrows"] == n_tc
         seen_gemv += cand_gemv
         seen_tc += cand_tc
