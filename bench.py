@@ -671,7 +671,19 @@ def run_ours(args, world, rank, local):
                          f"fp64 numpy oracle on {cores} host threads ({t:.1f} s)"}
 
     sweep = None
-    if sweep_on:  # after every headline pass: its weights are drawn on the host now
+    if sweep_on:
+        # after every headline pass, with the headline's layer, graph and device
+        # tensors released first: the sweep's layers then run in the same clean
+        # device memory state from point to point (its own weights are drawn on
+        # the host now)
+        del g_sparse
+        sparse.close()
+        sparse = g_sparse = None
+        W.clear()
+        xs.clear()
+        outs.clear()
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
         sweep = run_sweep(dev, local, args.warmup, args.reps)
 
     if rank == 0:
@@ -709,8 +721,9 @@ def run_ours(args, world, rank, local):
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
-    del g_sparse
-    sparse.close()
+    if sparse is not None:
+        del g_sparse
+        sparse.close()
     return 0
 
 
