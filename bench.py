@@ -331,33 +331,42 @@ def run_sweep(dev, local, warmup: int, reps: int, w_host=None) -> dict:
         def fwd():
             L.forward(xs[T], W["W_router"], W["W_gate"], W["W_up"], W["W_down"], tau,
                       sh.top_k, out=out)
+        clk = Clocks(local)
         lat = replay_stats(fwd, dev, warmup, reps)
+        c = clk.stop()
+        lat["sm_mhz"] = c.get("sm_mhz")
+        lat["clock_reasons"] = c.get("reasons")
         fwd()
         st = L.stats()
         assert L.status() == 0, "device status word set"
         L.close()
         return lat, st
 
+    # batch by batch, smallest first (the large batches run the tensor cores
+    # hardest and are measured last), each batch's dense point just before
+    # its sparse points; every point records the SM clock it ran at
     dense = {}
-    for T in xs:
+    points = []
+    for T in sorted(xs):
         lat, st = point(T, "dense", "h", 0.0)
         dense[T] = {"us": lat, "rows": st["down_rows_read"]}
-    points = []
-    for score, pts in SWEEP_POINTS.items():
-        for T, q in pts:
-            tau, _, calib = load_tau("mixtral_sweep", q, score)
-            lat, st = point(T, "auto", score, tau)
-            meas = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
-            points.append({
-                "score": score, "T": T, "target_sparsity": q, "sparsity": round(meas, 4),
-                "tau": tau, "us": lat, "dense_us": dense[T]["us"],
-                "speedup": round(dense[T]["us"]["median"] / lat["median"], 3),
-                "down_rows_read": st["down_rows_read"], "up_rows_read": st["up_rows_read"],
-                "gate_up_rows_read": st["gate_up_rows_read"],
-                "down_rows_dense": dense[T]["rows"],
-                "groups": {"gemv": st["n_groups_gemv"], "tc_allrows": st["n_groups_tc_allrows"],
-                           "tc_gather": st["n_groups_tc_gather"]},
-            })
+        for score, pts in SWEEP_POINTS.items():
+            for T2, q in pts:
+                if T2 != T:
+                    continue
+                tau, _, calib = load_tau("mixtral_sweep", q, score)
+                lat, st = point(T, "auto", score, tau)
+                meas = 1.0 - st["n_routed_active"] / max(st["n_routed_h"], 1)
+                points.append({
+                    "score": score, "T": T, "target_sparsity": q, "sparsity": round(meas, 4),
+                    "tau": tau, "us": lat, "dense_us": dense[T]["us"],
+                    "speedup": round(dense[T]["us"]["median"] / lat["median"], 3),
+                    "down_rows_read": st["down_rows_read"], "up_rows_read": st["up_rows_read"],
+                    "gate_up_rows_read": st["gate_up_rows_read"],
+                    "down_rows_dense": dense[T]["rows"],
+                    "groups": {"gemv": st["n_groups_gemv"], "tc_allrows": st["n_groups_tc_allrows"],
+                               "tc_gather": st["n_groups_tc_gather"]},
+                })
     summary = {}
     for score in SWEEP_POINTS:
         for T in (1, 16):
