@@ -67,6 +67,18 @@ constexpr int kGemvTokens = 8;      // tokens per GEMV pass (the row-stream mma'
 // launch, CUDA-event timed).
 constexpr int kGemvCandMax = 8;
 constexpr int kCandNum = 4, kCandDen = 5;
+// AUTO and DENSE: when at least kTcJoinNum / kTcJoinDen of a batch's groups
+// take the tensor-core path by their size alone (more than gemv_cand
+// tokens) and all of the batch's groups fit the tensor-core grid in one wave,
+// the batch's smaller groups join them there (all rows) instead of starting
+// the row-stream kernel for a few groups. Measured on the Mixtral-shaped
+// layer at T = 32 (groups of 4, 5, 8, 8, 9, 9, 10, 11 tokens): 466 us per
+// layer with all eight on the tensor cores against 485 us with the two
+// smallest on the row stream (the row-stream launch and its start-up cost
+// more than the extra rows, which take otherwise idle CTAs). With more
+// groups than the grid holds (128 small experts, T = 256) the joiners' rows
+// cost their full time: 272 vs 268 us, so that case keeps the row stream.
+constexpr int kTcJoinNum = 1, kTcJoinDen = 2;
 
 // A candidate group (kPathCand) takes the row stream when its passes over
 // the union rows cost less than all F_e rows on the tensor cores; both down

@@ -209,6 +209,22 @@ struct EntryCut {
   int me, ng, gsz, m_last, F_e, path_full, path_last;
 };
 
+// Whether a batch with n_groups groups, n_tc of them on the all-rows
+// tensor-core path by their size alone, sends its row-stream groups there too:
+// at least kTcJoinNum / kTcJoinDen of the groups are there already, and all
+// groups' units (group x 128 output columns) fit the tensor-core launch's grid
+// at once, so the joining groups take CTAs that would otherwise idle.
+__device__ __forceinline__ bool tc_join(const Dims& dm, int n_tc, int n_groups) {
+  return (dm.mode == kModeAuto || dm.mode == kModeDense) && !dm.no_tc && n_tc > 0 &&
+         static_cast<long long>(n_tc) * kTcJoinDen >=
+             static_cast<long long>(n_groups) * kTcJoinNum &&
+         static_cast<long long>(n_groups) * (dm.d / kDownSlice) <= dm.tc_grid;
+}
+__device__ __forceinline__ int joined_path(int path, bool join) {
+  return join && (path == kPathGemv || path == kPathCand || path == kPathFused) ? kPathTcAll
+                                                                                : path;
+}
+
 __device__ __forceinline__ EntryCut entry_cut(const Dims& dm, const int* cnt, int q) {
   EntryCut c;
   c.me = q < dm.E ? cnt[q] : dm.T;
@@ -253,12 +269,27 @@ __device__ void build_layout(const Dims& dm, const Workspace& ws, const int* cnt
   enum { kSlots, kGroups, kGemv, kTc, kCand, kRoutedGroups, kTcSharedDef, kTouched, kFused, kN };
   int v[kN] = {}, tot[kN];
   EntryCut cut[kPer];
+  // ---- pass 0: groups, and those on the all-rows tensor-core path by size
+  int g2[2] = {0, 0}, gt[2];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int q = q0 + i;
     if (q >= q1) continue;
-    const EntryCut c = entry_cut(dm, cnt, q);
-    cut[i] = c;
+    cut[i] = entry_cut(dm, cnt, q);
+    const EntryCut& c = cut[i];
+    if (c.ng == 0) continue;
+    g2[0] += c.ng;
+    g2[1] += (c.ng - 1) * (c.path_full == kPathTcAll) + (c.path_last == kPathTcAll);
+  }
+  block_exclusive_scan<2>(g2, gt, scan_sm);
+  const bool join = tc_join(dm, gt[1], gt[0]);
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int q = q0 + i;
+    if (q >= q1) continue;
+    cut[i].path_full = joined_path(cut[i].path_full, join);
+    cut[i].path_last = joined_path(cut[i].path_last, join);
+    const EntryCut c = cut[i];
     if (c.ng == 0) continue;
     const int n_gemv = (c.ng - 1) * on_gemv_list(c.path_full) + on_gemv_list(c.path_last);
     const int n_tc = (c.ng - 1) * on_tc_list(c.path_full) + on_tc_list(c.path_last);
@@ -659,6 +690,17 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
   const unsigned lt = (1u << lane) - 1u;
   for (int p = lane; p < P; p += 32) atomicAdd(&L.cnt[sel[p]], 1);
   __syncwarp();
+  // groups on the all-rows tensor-core path by size, for the join rule
+  int n_tc_size = 0, n_grp = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const int c = e < E ? L.cnt[e] : 0;
+    n_grp += __popc(__ballot_sync(0xffffffffu, c > 0));
+    n_tc_size += __popc(__ballot_sync(0xffffffffu, c > 0 && group_path_of(dm, c) == kPathTcAll));
+  }
+  n_grp += S;
+  n_tc_size += group_path_of(dm, T) == kPathTcAll ? S : 0;
+  const bool join = tc_join(dm, n_tc_size, n_grp);
   // touched experts in expert order: group index and path
   int n_touched = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
@@ -667,7 +709,7 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
     const unsigned bal = __ballot_sync(0xffffffffu, c > 0);
     if (c > 0) {
       const int g = n_touched + __popc(bal & lt);
-      const int path = group_path_of(dm, c);
+      const int path = joined_path(group_path_of(dm, c), join);
       L.gidx[e] = g;
       L.gpath[g] = path;
       Group gr;
@@ -682,13 +724,13 @@ __device__ void small_layout(const Dims& dm, const Workspace& ws, const int* sel
       // never used: every kernel masks the columns past a group's count)
       for (int r = c; r < kSlotAlign; ++r) ws.perm[g * kSlotAlign + r] = -1;
     }
-    if (e < E) L.yzero[e] = c > 0 && adds_into_y(group_path_of(dm, c));
+    if (e < E) L.yzero[e] = c > 0 && adds_into_y(joined_path(group_path_of(dm, c), join));
     n_touched += __popc(bal);
   }
   const int n_groups = n_touched + S;
   if (lane < S) {  // shared experts: one group of all T tokens each
     const int g = n_touched + lane;
-    const int path = group_path_of(dm, T);
+    const int path = joined_path(group_path_of(dm, T), join);
     L.gpath[g] = path;
     Group gr;
     gr.expert = E + lane;

@@ -392,6 +392,26 @@ def test_fused_down_matches_row_stream(name, T):
     compare(fused, oracle_forward(dw, x, tau, ts), tau, ts, "bf16", dw=dw)
 
 
+def test_small_groups_join_tensor_cores(mixtral):
+    """When at least half of a batch's groups hold more than 8 tokens (all
+    rows on the tensor cores by size), the batch's smaller groups join them
+    on the tensor cores: Mixtral-shaped decode batch T = 32 has groups of
+    4, 5, 8, 8, 9, 9, 10 and 11 tokens, so all eight read all d_ff rows there
+    and the row-stream kernel gets none; the output matches the oracle."""
+    wl, dw = mixtral
+    tau, _ = tau_of("mixtral_decode", 0.7)
+    x = workload_tokens(wl, 32)
+    gpu, _, _ = _check(make_layer(wl.shape, 64), dw, x, tau, 0.0, "bf16")
+    idx = gpu["topk_idx"].ravel()
+    sizes = np.bincount(idx, minlength=wl.shape.n_experts)
+    sizes = sizes[sizes > 0]
+    assert 2 * int((sizes > 8).sum()) >= len(sizes) and (sizes <= 8).any()
+    st = gpu["stats"]
+    assert st["n_groups_tc_allrows"] == len(sizes) and st["n_groups_gemv"] == 0
+    assert st["down_rows_read"] == len(sizes) * wl.shape.d_ff
+    assert st["down_rows_gemv"] == 0 and st["down_rows_fused"] == 0
+
+
 def test_candidate_groups_choose_by_union(sweep):
     """Groups of 5..8 tokens pick the row stream or all rows on the tensor
     cores after gate/up from their union size: both choices occur (high
