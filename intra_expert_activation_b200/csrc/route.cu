@@ -455,7 +455,7 @@ __device__ __forceinline__ void staged_logits(const Dims& dm, const TX* xs, cons
     for (int t = 0; t < TPC; ++t)
 #pragma unroll
       for (int j = 0; j < EPW; ++j) acc[t][j] = 0.f;
-#pragma unroll(TPC <= 4 ? 2 : 1)
+#pragma unroll(TPC <= 2 ? 4 : TPC <= 4 ? 2 : 1)
     for (int c = c0 + lane * VEC; c < c1; c += 32 * VEC) {
       float w[EPW][VEC];
 #pragma unroll
