@@ -98,9 +98,15 @@ typedef enum {
 } moe_score;
 
 typedef enum {
-  MOE_PATH_AUTO = 0,          /* threshold on; per group: GEMV, gathered TC or all-rows TC */
-  MOE_PATH_DENSE = 1,         /* no threshold: every neuron active (the dense baseline) */
-  MOE_PATH_SPARSE_GEMV = 2,   /* threshold on; every group on the CUDA-core row stream */
+  MOE_PATH_AUTO = 0,          /* threshold on; per group: row stream (GEMV; inside the gate/up
+                                 kernel when every gate/up tile of the batch has its own CTA),
+                                 gathered TC or all-rows TC; small groups join the all-rows TC
+                                 groups when those are at least half of the batch and all
+                                 groups fit one tensor-core wave */
+  MOE_PATH_DENSE = 1,         /* no threshold: every neuron active (the dense baseline; same
+                                 kernels and per-group rules as AUTO) */
+  MOE_PATH_SPARSE_GEMV = 2,   /* threshold on; every group on the CUDA-core row-stream kernel
+                                 (never fused into the gate/up kernel) */
   MOE_PATH_SPARSE_TC = 3,     /* threshold on; gathered-row tensor-core path (groups <= 64 tokens) */
   MOE_PATH_SPARSE_TC_ALLROWS = 4 /* threshold on; tensor cores over all rows with masked h */
 } moe_path;
