@@ -5,17 +5,19 @@
 // densely in shared memory and multiplies densely [gist.science EN
 // "Uncovering Intra-expert Activation Sparsity for Efficient Mixture-of-Expert
 // Model Execution", Technical Summary > Methodology > System Implementation in
-// vLLM > "Fused Up-Down Projection"]. Here the packing is done by TMA: each
-// active row is one 1-row box (128-byte swizzled) placed at its packed
-// position, so the tensor core sees a dense K-block of union rows.
+// vLLM > "Fused Up-Down Projection"]. Here the packing is done by TMA: four
+// active rows per copy (tile::gather4 over a tensor map whose box is one row,
+// 128-byte swizzled) land at their packed positions, so the tensor core sees
+// a dense K-block of union rows.
 //
 // Work unit: (group, 128-column slice of d_model); K = the group's union rows.
 //   D[128 columns][N tokens] = W_down[e][U, slice]^T . H^T[U, group slots]
 // Both operands are MN-major in shared memory: a W_down row is 128
 // contiguous output columns (M), an H^T row is 64 contiguous slots (N).
-//   gathered mode: K-block = 64 union rows, each fetched as 1-row boxes
-//     (A: 2 boxes of 64 columns, B: 1 box of 64 slots); rows past the union
-//     are fetched out of range, which TMA fills with zeros.
+//   gathered mode: K-block = 64 union rows, four per gather4 copy (A: two
+//     copies of 64 columns, B: one of 64 slots, per four rows); in the last
+//     K-block of a unit the positions past the union repeat the last union
+//     row of W_down and fetch H^T rows out of range one by one (zeros).
 //   all-rows mode: K-block = 64 consecutive rows with 64-row boxes; h of
 //     inactive neurons is an exact zero, so the sum is the same.
 // Warp roles as in the gate/up kernel: warp 0 TMA, warp 1 MMA + TMEM owner,
@@ -212,7 +214,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int* rows = p.ws.union_rows + static_cast<size_t>(du.g) * p.dm.F_max;
       const CUtensorMap* wrow = du.shared ? &p.tm_wds_row : &p.tm_wd_row;
       const CUtensorMap* wblk = du.shared ? &p.tm_wds_blk : &p.tm_wd_blk;
-      const int w_oob = du.shared ? p.dm.S * p.dm.Fs : p.dm.E * p.dm.F;
       for (int kc = du.k0; kc < du.k0 + du.nk; ++kc, ++it) {
         const uint32_t s = it % stages;
         const uint32_t ph = (it / stages) & 1u;
@@ -220,19 +221,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sa = smem + s * stage_bytes;
         uint8_t* sb = sa + kABytes;
         if (du.gather) {
+          // four union rows per copy (tile::gather4, boxes one row high): lane
+          // l < 16 fetches packed positions 4 l .. 4 l + 3 of the K-block. Past
+          // the union the W_down rows repeat the last union row (inside the
+          // tensor) and the H^T rows are fetched out of range one by one, which
+          // fills zeros, so those positions add nothing
           if (lane == 0) mbar_arrive_expect_tx(full + s, kABytes + 64 * 128);
           __syncwarp();
+          const int base = kc * kKBlock;
+          const bool whole_blk = base + kKBlock <= du.cnt;
+          if (lane < 16) {
+            int jr[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int r = lane + 32 * h;
-            const int pos = kc * kKBlock + r;
-            const bool valid = pos < du.cnt;
-            const int j = valid ? __ldcg(rows + pos) : 0;
-            const int wy = valid ? du.row_base + j : w_oob;
-            const int hy = valid ? j : ht_oob;
-            tma_load_2d(sa + r * 128, wrow, full + s, x0, wy);
-            tma_load_2d(sa + kAAtom + r * 128, wrow, full + s, x0 + 64, wy);
-            tma_load_2d(sb + r * 128, &p.tm_ht_row, full + s, du.gr.slot0, hy);
+            for (int q = 0; q < 4; ++q)
+              jr[q] = __ldcg(rows + min(base + 4 * lane + q, du.cnt - 1));
+            tma_gather4_2d(sa + lane * 512, wrow, full + s, x0, du.row_base + jr[0],
+                           du.row_base + jr[1], du.row_base + jr[2], du.row_base + jr[3]);
+            tma_gather4_2d(sa + kAAtom + lane * 512, wrow, full + s, x0 + 64, du.row_base + jr[0],
+                           du.row_base + jr[1], du.row_base + jr[2], du.row_base + jr[3]);
+            if (whole_blk)
+              tma_gather4_2d(sb + lane * 512, &p.tm_ht_row, full + s, du.gr.slot0, jr[0], jr[1],
+                             jr[2], jr[3]);
+          }
+          if (!whole_blk) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int r = lane + 32 * h;
+              const int pos = base + r;
+              const int hy = pos < du.cnt ? __ldcg(rows + pos) : ht_oob;
+              tma_load_2d(sb + r * 128, &p.tm_ht_row, full + s, du.gr.slot0, hy);
+            }
           }
         } else {
           const int nb = (N + 63) / 64;
