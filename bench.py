@@ -539,10 +539,12 @@ def run_ours(args, world, rank, local):
                 g_bytes += sh.n_shared * 2 * sh.d_ff_shared * sh.d_model * esize
         rb = sh.d_model * esize
         # W_down rows the gate/up kernel read itself (fused down projection of
-        # the groups of <= 4 tokens) belong to that kernel's bytes
+        # the groups of <= 4 tokens; with the gate score also the W_up rows of
+        # its fused up + down) belong to that kernel's bytes
         fused_rows = st["down_rows_fused"]
-        g_bytes += fused_rows * rb
-        u_bytes = st["up_rows_read"] * rb
+        fused_up = st["up_rows_fused"]
+        g_bytes += (fused_rows + fused_up) * rb
+        u_bytes = (st["up_rows_read"] - fused_up) * rb
         u_ms = avg_stage(per_fwd, i, "updown_gemv")  # gate score: fused sparse up + down
         up_bytes_tot += u_bytes * args.steps
         up_ms_tot += u_ms * args.steps
@@ -588,6 +590,7 @@ def run_ours(args, world, rank, local):
             round(lat_dense[i]["median"] / lat_sparse[i]["median"], 3),
             "down_rows_gemv": gemv_rows,
             "down_rows_fused": fused_rows,
+            "up_rows_fused": fused_up,
             "down_rows_read": st["down_rows_read"],
             "down_rows_dense": touched * sh.d_ff,
             "up_rows_read": st["up_rows_read"],

@@ -154,6 +154,8 @@ typedef struct {
   int64_t down_rows_fused;    /* of down_rows_read, the rows read by the gate/up kernel's fused
                                  down projection (row-stream groups of <= 4 tokens, bf16):
                                  per 128-neuron tile, the tile's active rows */
+  int64_t up_rows_fused;      /* of up_rows_read, the rows read by the gate/up kernel's fused
+                                 up + down projection (gate score, one-token groups) */
 } moe_stats;
 
 typedef struct moe_sparse_ctx moe_sparse_ctx;

@@ -62,7 +62,7 @@ class moe_stats(ctypes.Structure):
         "n_routed_h", "n_routed_active", "n_shared_h", "n_shared_active", "down_rows_read",
         "n_groups", "n_groups_gemv", "n_groups_tc_gather", "n_groups_tc_allrows",
         "n_experts_touched", "up_rows_read", "gate_up_rows_read", "down_rows_gemv",
-        "down_rows_fused")]
+        "down_rows_fused", "up_rows_fused")]
 
 
 _vp = ctypes.c_void_p

@@ -95,7 +95,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, 
   }
   ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
   const int path = __ldcg(p.ws.group_path + g);
-  ui.gate_only = p.dm.sparse_up && path == kPathGemv;
+  ui.gate_only = p.dm.sparse_up && (path == kPathGemv || path == kPathFused);
   ui.fused = path == kPathFused;
   ui.F_e = ui.shared ? p.dm.Fs : p.dm.F;
   const int e_local = ui.shared ? ui.gr.expert - p.dm.E : ui.gr.expert;
@@ -242,11 +242,14 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 // Shared-memory scratch of one unit's fused down projection: the tile's
 // active rows in neuron order with their h values (bf16-rounded, zero for
 // the tokens where the row is inactive).
+constexpr int kFuseHalfMax = 32;  // rows per half of the ring in the bulk path
+
 struct FuseScratch {
   uint64_t bar[2];            // bulk-copy halves of the ring (last unit of a CTA)
   float h[kNeuronTile][kFuseTokens];
   uint8_t rows[kNeuronTile];  // neuron index within the tile
   int cnt[4];                 // active rows of each epilogue warp's 32 neurons
+  float red[4][kFuseHalfMax]; // gate score: the four warps' partial up dots of a batch
 };
 constexpr int kFuseCols = 8;      // bf16 columns per thread and load (16 bytes)
 constexpr int kFuseInFlight = 16;  // row loads in flight per thread
@@ -368,27 +371,30 @@ __device__ void fuse_cols(const GateUpTcParams& p, const UnitInfo& ui, const Fus
   }
 }
 
-constexpr int kFuseHalfMax = 32;  // rows per half of the ring in the bulk path
-
 // The CTA's last unit (its weight ring is idle: every copy landed and every
-// MMA that read the ring has completed): the unit's R active rows, whole
-// (d = 1024 KC, rows of 2 KB KC), come into the ring by bulk copies, H rows
-// per half, the two halves alternating, so that up to 2 H rows are in flight
-// while the 128 threads multiply the landed half from shared memory (thread
-// tid reads 16 bytes at 2 KB k + 16 tid of a row: conflict-free). Thread tid
-// owns the same columns as in fuse_cols; MT <= 2 keeps the accumulators at
-// <= 64 registers.
-template <int MT, int KC>
-__device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, FuseScratch& fs,
-                               int R, int tid, uint8_t* ring, uint32_t ring_bytes,
-                               volatile int* abort_flag) {
-  const int d = p.dm.d, m = ui.gr.m;
+// MMA that read the ring has completed): the unit's R compacted rows of a
+// matrix W (W_down, or with the gate score first W_up), whole (d = 1024 KC,
+// rows of 2 KB KC), come into the ring by bulk copies, H rows per half, the
+// two halves alternating, so that up to 2 H rows are in flight while the 128
+// threads use the landed half from shared memory (thread tid reads 16 bytes
+// at 2 KB k + 16 tid of a row: conflict-free). row(r, i, src) is called by
+// every thread for landed row r (i-th of its batch, src: the thread's first
+// 16 bytes of it), batch(r0, n) by every thread after each batch (it may use
+// epi_sync), then the half is freed. fz_it counts the batches on the two
+// half barriers, whose phases run on from one call to the next. Returns
+// false once a wait has failed (the copies in flight have landed then).
+template <class RowFn, class BatchFn>
+__device__ bool bulk_rows(const GateUpTcParams& p, FuseScratch& fs, const __nv_bfloat16* W,
+                          int R, int tid, uint8_t* ring, uint32_t ring_bytes, uint32_t& fz_it,
+                          volatile int* abort_flag, RowFn row, BatchFn batch) {
+  const int d = p.dm.d;
   const uint32_t row_bytes = static_cast<uint32_t>(d) * 2;
   const int H = min(static_cast<int>(ring_bytes / row_bytes) / 2, kFuseHalfMax);
   const int nb = (R + H - 1) / H;
-  const __nv_bfloat16* W = (ui.shared ? p.wds : p.wd) + static_cast<size_t>(ui.wrow) * d;
-  auto issue = [&](int b) {  // thread 0: batch b into half b & 1
-    const int h = b & 1, r0 = b * H, n = min(H, R - r0);
+  const uint32_t g0 = fz_it;  // barrier index of this call's batch 0
+  fz_it += static_cast<uint32_t>(nb);
+  auto issue = [&](int b) {  // thread 0: batch b into half (g0 + b) & 1
+    const int h = (g0 + b) & 1, r0 = b * H, n = min(H, R - r0);
     mbar_arrive_expect_tx(&fs.bar[h], static_cast<uint32_t>(n) * row_bytes);
     for (int i = 0; i < n; ++i)
       bulk_load(smem_u32(ring + static_cast<size_t>(h * H + i) * row_bytes),
@@ -403,29 +409,19 @@ __device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, Fuse
       issued = 2;
     }
   }
-  float acc[MT][KC * kFuseCols];
-#pragma unroll
-  for (int t = 0; t < MT; ++t)
-#pragma unroll
-    for (int i = 0; i < KC * kFuseCols; ++i) acc[t][i] = 0.f;
   bool ok = true;
   for (int b = 0; b < nb; ++b) {
-    // every epilogue warp runs every batch (named barrier), skipping the
+    // every epilogue warp runs every batch (named barriers), skipping the
     // work once a wait has failed
-    const int h = b & 1;
-    if (ok && !warp_wait(&fs.bar[h], (b >> 1) & 1, abort_flag, p.ws.status)) ok = false;
+    const uint32_t g = g0 + b;
+    const int h = g & 1;
+    if (ok && !warp_wait(&fs.bar[h], (g >> 1) & 1, abort_flag, p.ws.status)) ok = false;
+    const int r0 = b * H, n = min(H, R - r0);
     if (ok) {
-      const int r0 = b * H, n = min(H, R - r0);
       const uint8_t* base = ring + static_cast<size_t>(h * H) * row_bytes + tid * 16;
-      for (int i = 0; i < n; ++i) {
-        const float* hr = fs.h[r0 + i];
-#pragma unroll
-        for (int k = 0; k < KC; ++k) {
-          const uint4 v = *reinterpret_cast<const uint4*>(base + i * row_bytes + k * 2048);
-          fuse_fma<MT, KC>(acc, k, v, hr);
-        }
-      }
+      for (int i = 0; i < n; ++i) row(r0 + i, i, base + static_cast<size_t>(i) * row_bytes);
     }
+    batch(r0, n);
     epi_sync();  // the half is read: it may be refilled
     if (tid == 0 && b + 2 < nb && !*abort_flag) {
       issue(b + 2);
@@ -437,11 +433,22 @@ __device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, Fuse
     // the last batch issued on each half
     volatile int never = 0;
     for (int hh = 0; hh < 2; ++hh) {
-      const int lb = issued - 1 - ((issued - 1 - hh) & 1);
-      if (lb >= 0) mbar_wait(&fs.bar[hh], (lb >> 1) & 1, &never, p.ws.status);
+      int lb = issued - 1;  // this call's last batch on half hh
+      if (lb >= 0 && static_cast<int>((g0 + lb) & 1) != hh) --lb;
+      if (lb >= 0) mbar_wait(&fs.bar[hh], ((g0 + lb) >> 1) & 1, &never, p.ws.status);
     }
   }
-  if (!ok) return;
+  return ok && !*abort_flag;
+}
+
+// Adds w x the sums of this thread's columns (tokens t < m of the group,
+// acc[t][8 k + i] at column 8 tid + 1024 k + i) into Y or, under direct
+// combine, into the tokens' output accumulator rows.
+template <int MT, int KC>
+__device__ __forceinline__ void fuse_flush(const GateUpTcParams& p, const UnitInfo& ui,
+                                           const float (&acc)[MT][KC * kFuseCols], int m,
+                                           int tid) {
+  const int d = p.dm.d;
   const int c0 = tid * kFuseCols;
 #pragma unroll
   for (int t = 0; t < MT; ++t)
@@ -460,11 +467,96 @@ __device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, Fuse
     }
 }
 
+// The last unit's down projection through the ring: y += h_r W_down[r] over
+// its R rows, tokens t < m <= MT (MT <= 2 keeps the accumulators at <= 64
+// registers).
+template <int MT, int KC>
+__device__ void fuse_rows_bulk(const GateUpTcParams& p, const UnitInfo& ui, FuseScratch& fs,
+                               int R, int tid, uint8_t* ring, uint32_t ring_bytes,
+                               uint32_t& fz_it, volatile int* abort_flag) {
+  float acc[MT][KC * kFuseCols];
+#pragma unroll
+  for (int t = 0; t < MT; ++t)
+#pragma unroll
+    for (int i = 0; i < KC * kFuseCols; ++i) acc[t][i] = 0.f;
+  const __nv_bfloat16* W = (ui.shared ? p.wds : p.wd) + static_cast<size_t>(ui.wrow) * p.dm.d;
+  const bool ok = bulk_rows(
+      p, fs, W, R, tid, ring, ring_bytes, fz_it, abort_flag,
+      [&](int r, int, const uint8_t* src) {
+#pragma unroll
+        for (int k = 0; k < KC; ++k)
+          fuse_fma<MT, KC>(acc, k, *reinterpret_cast<const uint4*>(src + k * 2048), fs.h[r]);
+      },
+      [&](int, int) {});
+  if (ok) fuse_flush<MT, KC>(p, ui, acc, ui.gr.m, tid);
+}
+
+// Gate score, a one-token group (the last unit of its CTA): the unit's rows
+// are the neurons with |SiLU(g)| > tau, and fs.h holds their SiLU(g) rounded
+// to bf16. First the rows of W_up come through the ring: each thread dots
+// its columns of a row with the token's x (kept in registers), the four
+// warps' partials of a batch meet in shared memory and are added in warp
+// order, and h = bf16(SiLU(g) u) replaces SiLU(g) in fs.h (as the separate
+// fused kernel rounds it); then the same rows of W_down, as fuse_rows_bulk
+// [same list, "Fused Up-Down Projection": only the active neurons' up and
+// down weights are fetched].
+template <int KC>
+__device__ void fuse_updown_bulk(const GateUpTcParams& p, const UnitInfo& ui, FuseScratch& fs,
+                                 int R, int tid, uint8_t* ring, uint32_t ring_bytes,
+                                 uint32_t& fz_it, volatile int* abort_flag) {
+  const int d = p.dm.d;
+  const int q = tid >> 5, lane = tid & 31;
+  // the token's x: routed groups from X_perm, shared experts' from x
+  const __nv_bfloat16* xr =
+      (ui.shared ? p.x : static_cast<const __nv_bfloat16*>(p.ws.xperm)) +
+      static_cast<size_t>(ui.gr.xrow0) * d;
+  float xv[KC * kFuseCols];
+#pragma unroll
+  for (int k = 0; k < KC; ++k) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + tid * kFuseCols + k * 1024));
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xv[k * kFuseCols + 2 * i] = __uint_as_float(u[i] << 16);
+      xv[k * kFuseCols + 2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+  }
+  const __nv_bfloat16* Wu = (ui.shared ? p.wus : p.wu) + static_cast<size_t>(ui.wrow) * d;
+  const bool ok = bulk_rows(
+      p, fs, Wu, R, tid, ring, ring_bytes, fz_it, abort_flag,
+      [&](int, int i, const uint8_t* src) {
+        float a = 0.f;
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + k * 2048);
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            a = fmaf(xv[k * kFuseCols + 2 * j], __uint_as_float(u[j] << 16), a);
+            a = fmaf(xv[k * kFuseCols + 2 * j + 1], __uint_as_float(u[j] & 0xffff0000u), a);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) fs.red[q][i] = a;
+      },
+      [&](int r0, int n) {
+        epi_sync();  // the batch's partial dots are in
+        if (tid < n) {
+          const float u = ((fs.red[0][tid] + fs.red[1][tid]) + fs.red[2][tid]) + fs.red[3][tid];
+          fs.h[r0 + tid][0] = __bfloat162float(__float2bfloat16_rn(fs.h[r0 + tid][0] * u));
+        }
+      });
+  if (!ok) return;
+  fuse_rows_bulk<1, KC>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+}
+
 // A kPathFused unit after its epilogue, every epilogue warp: compaction, the
-// down projection of the active rows, and a barrier that frees the scratch.
-// uni / hv: this warp's union word and its lane's h values (token t in
-// hv[t]); a warp whose wait failed passes uni = 0. last: the CTA has no
-// further unit (the ring may be used for bulk copies of the rows).
+// down projection of the active rows (with the gate score also their up
+// projection), and a barrier that frees the scratch. uni / hv: this warp's
+// union word and its lane's h values (token t in hv[t]; SiLU(g) for a
+// gate-only unit); a warp whose wait failed passes uni = 0. last: the CTA
+// has no further unit (the ring may be used for bulk copies of the rows).
 __device__ __forceinline__ void fuse_unit(const GateUpTcParams& p, const UnitInfo& ui,
                                           FuseScratch& fs, uint32_t uni,
                                           const float (&hv)[kFuseTokens], int q, int lane,
@@ -473,16 +565,32 @@ __device__ __forceinline__ void fuse_unit(const GateUpTcParams& p, const UnitInf
   const int m = ui.gr.m;
   const int R = fuse_compact(fs, uni, hv, m, q, lane);
   const int tid = 32 * q + lane;
-  if (R > 0) {
-    const int d = p.dm.d;
-    const bool bulk = last && m <= 2 && ring_bytes >= 4u * static_cast<uint32_t>(d);
-    if (bulk && d == 4096) {
-      if (m == 1) fuse_rows_bulk<1, 4>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
-      else fuse_rows_bulk<2, 4>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
-    } else if (bulk && d == 2048) {
-      fuse_rows_bulk<2, 2>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
-    } else if (bulk && d == 1024) {
-      fuse_rows_bulk<2, 1>(p, ui, fs, R, tid, ring, ring_bytes, abort_flag);
+  uint32_t fz_it = 0;  // one fused unit per CTA: the half barriers start here
+  const int d = p.dm.d;
+  const bool bulk = last && ring_bytes >= 4u * static_cast<uint32_t>(d) &&
+                    (d == 4096 || d == 2048 || d == 1024);
+  if (ui.gate_only) {
+    // the host fuses gate-score units only as a CTA's last work, for one-token
+    // groups and these widths; anything else is an internal error
+    if (!(bulk && m == 1)) {
+      report_error(p.ws.status, kErrDeviceInvalid);
+    } else if (R > 0) {
+      if (d == 4096) fuse_updown_bulk<4>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+      else if (d == 2048) fuse_updown_bulk<2>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+      else fuse_updown_bulk<1>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+    }
+    if (tid == 0) {  // W_up rows this unit read
+      atomicAdd(p.ws.counters + kCntUpRows, static_cast<unsigned long long>(R));
+      atomicAdd(p.ws.counters + kCntFusedUpRows, static_cast<unsigned long long>(R));
+    }
+  } else if (R > 0) {
+    if (bulk && m <= 2 && d == 4096) {
+      if (m == 1) fuse_rows_bulk<1, 4>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+      else fuse_rows_bulk<2, 4>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+    } else if (bulk && m <= 2 && d == 2048) {
+      fuse_rows_bulk<2, 2>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
+    } else if (bulk && m <= 2 && d == 1024) {
+      fuse_rows_bulk<2, 1>(p, ui, fs, R, tid, ring, ring_bytes, fz_it, abort_flag);
     } else if (m == 1 && d % 4096 == 0) {
       fuse_cols<1, 4>(p, ui, fs, R, tid);
     } else if (m <= 2 && d % 2048 == 0) {

@@ -99,7 +99,7 @@ enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUse
 enum Counter { kCntRoutedActive = 0, kCntSharedActive = 1, kCntDownRows = 2, kCntGemv = 3,
                kCntTcGather = 4, kCntTc = 5, kCntRoutedH = 6, kCntSharedH = 7,
                kCntUpRows = 8, kCntGateUpRows = 9, kCntGemvRows = 10, kCntFusedRows = 11,
-               kCntWords = 12 };
+               kCntFusedUpRows = 12, kCntWords = 13 };
 
 // kPathCand: GEMV or all-rows TC, chosen after gate/up (cand_takes_gemv).
 // kPathFused: a row-stream group whose down projection the gate/up kernel
@@ -149,9 +149,10 @@ struct Dims {
   // rows Y[0..T) (zeroed by the router) and its last CTA writes out; no
   // combine launch
   int direct_combine;
-  // 1: row-stream groups of <= kFuseTokens tokens take kPathFused: the gate/up
-  // kernel multiplies each tile's active W_down rows by its h values and adds
-  // the sums into Y (bf16 layers, |h| score or a dense up projection)
+  // 1: row-stream groups of <= kFuseTokens tokens (one token with the gate
+  // score's sparse up projection) take kPathFused: the gate/up kernel
+  // multiplies each tile's active W_down rows (with the gate score first the
+  // W_up rows) by its h values and adds the sums into Y (bf16 layers)
   int fuse_down;
   // 1 (with direct_combine): no row-stream launch follows the gate/up kernel,
   // so its last CTA (a ticket) writes out from the accumulator rows
@@ -242,6 +243,9 @@ struct GateUpTcParams {
   int b_blocks;                // activation regions per stage: 2 with the gate score, else 1
   const __nv_bfloat16* wd;     // [E*F][d] W_down (fused down projection, kPathFused groups)
   const __nv_bfloat16* wds;    // [S*Fs][d] shared experts' W_down
+  const __nv_bfloat16* wu;     // [E*F][d] W_up (gate score: fused up + down of one-token groups)
+  const __nv_bfloat16* wus;    // [S*Fs][d] shared experts' W_up
+  const __nv_bfloat16* x;      // [T][d] the layer input (shared experts' tokens)
   void* out;                   // [T][d] layer output (dm.fuse_finish)
   int out_bf16;                // out's type: 1 bf16, 0 fp32
 };

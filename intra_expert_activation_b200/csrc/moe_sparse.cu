@@ -574,21 +574,30 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   // T = 8 on the Mixtral-shaped layer: 384 vs 363 us per layer); with one
   // unit per CTA the fusion saves the row-stream launch and its start-up
   // (T = 1: 110 vs 120 us).
-  dm.fuse_down = c->bf16 && !dm.sparse_up && (mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
-                 gu_units_max <= gu_grid && moe::fuse_enabled() ? 1 : 0;
+  // With the gate score (sparse up projection) the gate/up kernel also does
+  // the up projection of the active rows of one-token groups, for rows of
+  // 1, 2 or 4 KB (the layout of its bulk path).
+  dm.fuse_down = c->bf16 && (mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) &&
+                 gu_units_max <= gu_grid &&
+                 (!dm.sparse_up || cap.d == 1024 || cap.d == 2048 || cap.d == 4096) &&
+                 moe::fuse_enabled() ? 1 : 0;
   if (dm.fuse_down) {
     // the row-stream kernel is only needed for groups the fusion leaves:
     // unfused row-stream groups and candidates
-    const bool big_gemv = std::min(tmax, cap.gemv_max) > moe::kFuseTokens;
+    const int fused_max = dm.sparse_up ? 1 : moe::kFuseTokens;
+    const bool big_gemv = std::min(tmax, cap.gemv_max) > fused_max;
     const bool cand = cap.gemv_cand > cap.gemv_max && tmax > cap.gemv_max;
     need_gemv = big_gemv || cand;
   }
-  // every group on the |h|-score row stream (fused or not) and a small
-  // batch: the row stream combines directly into the output (no combine
-  // launch); with no row-stream launch the gate/up kernel writes out
+  // every group on a row stream (fused or not; with the gate score only when
+  // all of them are fused, since its separate kernel has no direct combine)
+  // and a small batch: the row stream combines directly into the output (no
+  // combine launch); with no row-stream launch the gate/up kernel writes out
   const bool out_bf16 = c->bf16 && !c->desc.out_f32;
-  dm.direct_combine =
-      (need_gemv || dm.fuse_down) && !need_tc && !dm.sparse_up && T <= moe::kDirectMax ? 1 : 0;
+  dm.direct_combine = (need_gemv || dm.fuse_down) && !need_tc &&
+                              (!dm.sparse_up || !need_gemv) && T <= moe::kDirectMax
+                          ? 1
+                          : 0;
   dm.fuse_finish = dm.direct_combine && !need_gemv ? 1 : 0;
   // the tensor-core down launch's grid is fixed here: the router's layout
   // and the kernel both derive the units' K parts from it
@@ -665,6 +674,9 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     const size_t smem = moe::gate_up_tc_smem_bytes(n_max, p.stages, p.b_blocks, dm.fuse_down);
     p.wd = static_cast<const __nv_bfloat16*>(W_down);
     p.wds = static_cast<const __nv_bfloat16*>(c->Wds);
+    p.wu = static_cast<const __nv_bfloat16*>(W_up);
+    p.wus = static_cast<const __nv_bfloat16*>(c->Wus);
+    p.x = static_cast<const __nv_bfloat16*>(x);
     p.out = out;
     p.out_bf16 = out_bf16 ? 1 : 0;
     const int grid = gu_grid;
@@ -789,6 +801,7 @@ moe_status moe_sparse_get_stats(moe_sparse_ctx* c, moe_stats* s, void* stream) {
   s->gate_up_rows_read = (int64_t)cnt[moe::kCntGateUpRows];
   s->down_rows_gemv = (int64_t)cnt[moe::kCntGemvRows];
   s->down_rows_fused = (int64_t)cnt[moe::kCntFusedRows];
+  s->up_rows_fused = (int64_t)cnt[moe::kCntFusedUpRows];
   return MOE_OK;
 }
 

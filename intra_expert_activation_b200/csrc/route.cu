@@ -81,7 +81,7 @@ __device__ __forceinline__ int group_path_of(const Dims& dm, int m) {
   if (dm.mode == kModeTc) return kPathTcAll;  // gathered or not: decided by the union scan
   if (dm.mode == kModeTcAll) return kPathTcAll;
   if (m <= dm.gemv_max)  // auto and dense; the smallest groups inside the gate/up kernel
-    return dm.fuse_down && m <= kFuseTokens ? kPathFused : kPathGemv;
+    return dm.fuse_down && m <= (dm.sparse_up ? 1 : kFuseTokens) ? kPathFused : kPathGemv;
   return m <= dm.gemv_cand ? kPathCand : kPathTcAll;
 }
 

@@ -8,7 +8,7 @@
 #include "moe_sparse.h"
 
 _Static_assert(sizeof(moe_sparse_desc) == 16 * 4, "moe_sparse_desc layout");
-_Static_assert(sizeof(moe_stats) == 14 * 8, "moe_stats layout");
+_Static_assert(sizeof(moe_stats) == 15 * 8, "moe_stats layout");
 
 static int fails = 0;
 #define CHECK(c)                                  \

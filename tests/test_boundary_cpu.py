@@ -54,7 +54,7 @@ def test_only_the_abi_is_exported():
 
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(_lib.moe_sparse_desc) == 16 * 4
-    assert ctypes.sizeof(_lib.moe_stats) == 14 * 8
+    assert ctypes.sizeof(_lib.moe_stats) == 15 * 8
 
 
 def test_valid_desc_accepted(lib):

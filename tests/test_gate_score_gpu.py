@@ -4,13 +4,15 @@ up projection reads only the active-row union of W_up, and an active neuron
 contributes its full h = SiLU(g) u. Same criteria as the |h| score, with the
 band taken on |SiLU(g)|."""
 
+import os
+
 import numpy as np
 import pytest
 import torch
 
 from moe_inputs import LayerShape, make_tokens, make_weights
 from oracle import moe_oracle as om
-from _parity import (DeviceWeights, compare, make_layer, oracle_forward, run_gpu, tau_of,
+from _parity import (TAUS, DeviceWeights, compare, make_layer, oracle_forward, run_gpu, tau_of,
                      workload_tokens, workload_weights)
 
 pytestmark = pytest.mark.gpu
@@ -105,3 +107,32 @@ def test_mixtral_decode_gate(mixtral, T):
     if T == 1:  # both groups on the GEMV path: the up and down kernels read the same rows
         assert st["up_rows_read"] == st["down_rows_read"] > 0
         assert st["up_rows_read"] < 2 * wl.shape.d_ff  # only the active-row unions
+
+@pytest.mark.parametrize("name,T", [("mixtral_decode", 1), ("shared_routed_prefill", 1),
+                                    ("many_small_experts", 1)])
+def test_gate_fused_up_down_matches_separate_kernel(name, T):
+    """One-token groups whose gate/up units fit one per CTA: the gate/up
+    kernel does their sparse up and down projection itself (the rows with
+    |SiLU(g)| > tau of W_up, then of W_down). Against the separate fused
+    up + down kernel (path forced to the row stream): the same rows are read,
+    the fp32 outputs agree to the rounding of h to bf16, and both match the
+    oracle (routed and shared experts)."""
+    if os.environ.get("MOE_FUSE_DOWN") == "0":
+        pytest.skip("fused down projection turned off")
+    wl, dw = workload_weights(name)
+    e = TAUS[name]["taus_gate"][f"{wl.sparsities[0]:.2f}"]
+    tau, ts = e["tau"], e.get("tau_shared", 0.0)
+    x = workload_tokens(wl, T)
+    fused = run_gpu(make_layer(wl.shape, 64, score="gate", out_f32=True), dw, x, tau, ts)
+    sep = run_gpu(make_layer(wl.shape, 64, path="sparse_gemv", score="gate", out_f32=True), dw, x,
+                  tau, ts)
+    assert np.array_equal(fused["active_bits"], sep["active_bits"])
+    sf, ss = fused["stats"], sep["stats"]
+    assert sf["up_rows_fused"] == sf["up_rows_read"] == ss["up_rows_read"] > 0
+    assert sf["down_rows_fused"] == sf["down_rows_read"] == ss["down_rows_read"]
+    assert ss["up_rows_fused"] == 0 and ss["down_rows_fused"] == 0
+    a, b = fused["out"], sep["out"]
+    assert np.abs(a - b).max() <= 2e-3 * np.abs(b).max(), (np.abs(a - b).max(), np.abs(b).max())
+    ref = oracle_forward(dw, x, tau, ts, score="gate")
+    compare(fused, ref, tau, ts, "bf16", dw=dw, score="gate")
+    compare(sep, ref, tau, ts, "bf16", dw=dw, score="gate")
