@@ -45,20 +45,23 @@
 // unit rounds keep the CTAs in step along K.)
 //
 // Fused down projection (groups of kPathFused: the smallest row-stream
-// groups, dm.fuse_down). Once a unit's h is known, the tile's active rows
-// are final: neuron j of the tile contributes h_j W_down[e][j,:] to the
-// group's outputs and nothing else does [same list, "Fused Up-Down
-// Projection": only the active neurons' weight rows are fetched]. So right
-// after the unit's epilogue (and after its TMEM buffer is handed back to the
-// MMA warp) the four epilogue warps compact the tile's active rows and their
-// h values into shared memory, stream those rows of W_down with 16-byte
-// loads (each warp instruction reads 512 contiguous bytes of a row, 16 rows
-// in flight per thread), multiply on the CUDA cores in fp32 and add the sums
-// into Y with vector fp32 atomics (or, under direct combine, w x the sums
-// into the token's output accumulator row). The next unit's weight tiles
-// stream meanwhile, so the down rows ride on the same pass over HBM, with
-// no second kernel, no second start-up and no second walk over the union
-// bitmaps. h is rounded to bf16 first, as H^T holds it for the down kernels.
+// groups of batches whose units fit one per CTA, dm.fuse_down). Once a
+// unit's h is known, the tile's active rows are final: neuron j of the tile
+// contributes h_j W_down[e][j,:] to the group's outputs and nothing else does
+// [same list, "Fused Up-Down Projection": only the active neurons' weight
+// rows are fetched]. So after the unit's epilogue (its TMEM buffer handed
+// back to the MMA warp) the four epilogue warps compact the tile's active
+// rows and their h values into shared memory; as the CTA's last work, when
+// its weight ring is idle, they bring those rows of W_down into the ring by
+// bulk copies, multiply on the CUDA cores in fp32 and add the sums into Y
+// with vector fp32 atomics (or, under direct combine, w x the sums into the
+// token's output accumulator row, the last CTA writing out). A unit that is
+// not its CTA's last (not the case the host arranges) reads the rows with
+// 16-byte loads instead. This saves the row-stream kernel's launch, start-up
+// and walk over the union bitmaps. h is rounded to bf16 first, as H^T holds
+// it for the down kernels. With the gate score a one-token group's unit is
+// gate-only: its active rows (|SiLU(g)| > tau) of W_up come through the ring
+// first, dotted with the token's x, and then the same rows of W_down.
 #include "common.cuh"
 
 namespace moe {
