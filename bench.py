@@ -343,13 +343,16 @@ def run_sweep(dev, local, warmup: int, reps: int, w_host=None) -> dict:
         return lat, st
 
     # batch by batch, smallest first (the large batches run the tensor cores
-    # hardest and are measured last), each batch's dense point just before
-    # its sparse points; every point records the SM clock it ran at
+    # hardest and are measured last), each batch's dense point measured just
+    # before and again just after its sparse points (the reference is the
+    # mean of the two medians, so that a drift of the clock over the batch's
+    # points shows in both); every point records the SM clock it ran at
     dense = {}
     points = []
     for T in sorted(xs):
         lat, st = point(T, "dense", "h", 0.0)
         dense[T] = {"us": lat, "rows": st["down_rows_read"]}
+        first = len(points)
         for score, pts in SWEEP_POINTS.items():
             for T2, q in pts:
                 if T2 != T:
@@ -367,6 +370,13 @@ def run_sweep(dev, local, warmup: int, reps: int, w_host=None) -> dict:
                     "groups": {"gemv": st["n_groups_gemv"], "tc_allrows": st["n_groups_tc_allrows"],
                                "tc_gather": st["n_groups_tc_gather"]},
                 })
+        lat2, _ = point(T, "dense", "h", 0.0)
+        ref = 0.5 * (dense[T]["us"]["median"] + lat2["median"])
+        dense[T]["us"] = dict(dense[T]["us"], median=round(ref, 2), before=dense[T]["us"]["median"],
+                              after=lat2["median"])
+        for pnt in points[first:]:
+            pnt["dense_us"] = dense[T]["us"]
+            pnt["speedup"] = round(ref / pnt["us"]["median"], 3)
     summary = {}
     for score in SWEEP_POINTS:
         for T in (1, 16):
