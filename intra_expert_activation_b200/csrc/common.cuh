@@ -342,6 +342,10 @@ static __device__ void direct_finish(const Dims& dm, const Workspace& ws, void* 
   __syncthreads();
   if (!is_last) return;
   __threadfence();
+  if (threadIdx.x == 0) {  // every CTA has its ticket: ready for the next forward
+    ws.meta[kMetaDownDone] = 0;
+    ws.meta[kMetaRoute1] = 0;
+  }
   const int n4 = dm.T * dm.d / 4;
   const float4* y4 = reinterpret_cast<const float4*>(ws.y);
   for (int i = threadIdx.x; i < n4; i += blockDim.x) {

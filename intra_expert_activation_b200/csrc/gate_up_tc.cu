@@ -63,6 +63,7 @@
 // gate-only: its active rows (|SiLU(g)| > tau) of W_up come through the ring
 // first, dotted with the token's x, and then the same rows of W_down.
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -82,8 +83,18 @@ struct UnitInfo {
   int fused;      // kPathFused: this kernel also does the unit's down projection
 };
 
+// One-token routing inside this kernel (dm.route1): the selected experts in
+// expert order (group g = the g-th of them, its slot block g) and their
+// combine weights.
+struct Route1Groups {
+  int k;
+  int exp[16];
+  float w[16];
+};
+
 __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, int n_rg,
-                                                int tiles_r, int tiles_s) {
+                                                int tiles_r, int tiles_s,
+                                                const Route1Groups* r1) {
   UnitInfo ui;
   int g;
   if (u < n_rg * tiles_r) {
@@ -96,8 +107,17 @@ __device__ __forceinline__ UnitInfo decode_unit(const GateUpTcParams& p, int u, 
     ui.nt = v % tiles_s;
     ui.shared = 1;
   }
-  ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
-  const int path = __ldcg(p.ws.group_path + g);
+  int path;
+  if (r1) {  // the token (row 0 of x) alone, in slot block g
+    ui.gr.expert = r1->exp[g];
+    ui.gr.slot0 = g * kSlotAlign;
+    ui.gr.m = 1;
+    ui.gr.xrow0 = 0;
+    path = kPathFused;
+  } else {
+    ui.gr = p.ws.groups[g];  // expert: routed e, or E + s for shared expert s
+    path = __ldcg(p.ws.group_path + g);
+  }
   ui.gate_only = p.dm.sparse_up && (path == kPathGemv || path == kPathFused);
   ui.fused = path == kPathFused;
   ui.F_e = ui.shared ? p.dm.Fs : p.dm.F;
@@ -249,11 +269,13 @@ constexpr int kFuseHalfMax = 32;  // rows per half of the ring in the bulk path
 
 struct FuseScratch {
   uint64_t bar[2];            // bulk-copy halves of the ring (last unit of a CTA)
-  float h[kNeuronTile][kFuseTokens];
+  alignas(16) float h[kNeuronTile][kFuseTokens];  // read as float4 rows
   uint8_t rows[kNeuronTile];  // neuron index within the tile
   int cnt[4];                 // active rows of each epilogue warp's 32 neurons
   float red[4][kFuseHalfMax]; // gate score: the four warps' partial up dots of a batch
+  Route1Groups r1;            // dm.route1: this CTA's routing of the token
 };
+static_assert(offsetof(FuseScratch, h) % 16 == 0, "h rows are read as float4");
 constexpr int kFuseCols = 8;      // bf16 columns per thread and load (16 bytes)
 constexpr int kFuseInFlight = 16;  // row loads in flight per thread
 
@@ -511,7 +533,7 @@ __device__ void fuse_updown_bulk(const GateUpTcParams& p, const UnitInfo& ui, Fu
   const int q = tid >> 5, lane = tid & 31;
   // the token's x: routed groups from X_perm, shared experts' from x
   const __nv_bfloat16* xr =
-      (ui.shared ? p.x : static_cast<const __nv_bfloat16*>(p.ws.xperm)) +
+      (ui.shared || p.dm.route1 ? p.x : static_cast<const __nv_bfloat16*>(p.ws.xperm)) +
       static_cast<size_t>(ui.gr.xrow0) * d;
   float xv[KC * kFuseCols];
 #pragma unroll
@@ -613,6 +635,106 @@ __device__ __forceinline__ void fuse_unit(const GateUpTcParams& p, const UnitInf
   epi_sync();
 }
 
+// One-token routing in every CTA (dm.route1), all threads, before the warp
+// roles start: the token's logits against every router row (a warp per
+// expert, lanes over d, eight 16-byte loads of each in flight; scratch: the
+// first stage of the weight ring, unused until the roles start), its top-k
+// (topk_warp, as the routers pick), and the selected experts in expert order
+// as the groups, one token each. The first CTA also writes what the router
+// would have written for the getters and the combine (top-k ids and weights,
+// slots, groups, paths, counters, meta), zeroes the output accumulator row,
+// and then publishes meta[kMetaRoute1]; the other CTAs wait for it before
+// their first atomic add (their epilogue, many microseconds later).
+__device__ void route1_prologue(const GateUpTcParams& p, float* lg, Route1Groups& r1, int warp,
+                                int lane) {
+  const int E = p.dm.E, d = p.dm.d, k = p.dm.k;
+  for (int e = warp; e < E; e += kThreads / 32) {
+    const __nv_bfloat16* wr = p.wr + static_cast<size_t>(e) * d;
+    float a = 0.f;
+    for (int c0 = lane * 8; c0 < d; c0 += 32 * 8 * 8) {
+      uint4 wv[8], xv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + u * 32 * 8;
+        wv[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(wr + c)) : make_uint4(0u, 0u, 0u, 0u);
+        xv[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(p.x + c)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t wa[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+        const uint32_t xa[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          a = fmaf(__uint_as_float(xa[j] << 16), __uint_as_float(wa[j] << 16), a);
+          a = fmaf(__uint_as_float(xa[j] & 0xffff0000u), __uint_as_float(wa[j] & 0xffff0000u), a);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) lg[e] = a + (p.rbias ? p.rbias[e] : 0.f);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const TopkResult r = topk_warp(lg, E, k, lane);
+    const float w = p.dm.renorm ? r.my_p / r.psum : r.my_p;
+    int rank = 0;  // position of this lane's expert in expert order (ids are distinct)
+    for (int j = 0; j < k; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, r.my_e, j);
+      if (lane < k && ej < r.my_e) ++rank;
+    }
+    if (lane < k) {
+      r1.exp[rank] = r.my_e;
+      r1.w[rank] = w;
+    }
+    if (lane == 0) r1.k = k;
+    if (blockIdx.x == 0 && lane < k) {
+      const int slot = rank * kSlotAlign;
+      p.ws.topk_idx[lane] = r.my_e;
+      p.ws.topk_w[lane] = w;
+      p.ws.slot_of[lane] = slot;
+      p.ws.slot_w[slot] = w;
+      p.ws.perm[slot] = 0;
+      for (int q = 1; q < kSlotAlign; ++q) p.ws.perm[slot + q] = -1;
+      Group gr;
+      gr.expert = r.my_e;
+      gr.slot0 = slot;
+      gr.m = 1;
+      gr.xrow0 = slot;
+      p.ws.groups[rank] = gr;
+      p.ws.group_path[rank] = kPathFused;
+      p.ws.union_cnt[rank] = 0;
+    }
+  }
+  if (blockIdx.x == 0) {
+    const int tid = threadIdx.x;
+    if (tid < kCntWords) {
+      unsigned long long v = 0ull;
+      if (tid == kCntGemv) v = static_cast<unsigned long long>(k);  // fused row-stream groups
+      if (tid == kCntRoutedH) v = static_cast<unsigned long long>(k) * p.dm.F;
+      p.ws.counters[tid] = v;
+    }
+    if (tid == 0) {
+      p.ws.meta[kMetaGroups] = k;
+      p.ws.meta[kMetaRoutedGroups] = k;
+      p.ws.meta[kMetaSlotsUsed] = k * kSlotAlign;
+      p.ws.meta[kMetaExpertsTouched] = k;
+      p.ws.meta[kMetaGemvCount] = 0;
+      p.ws.meta[kMetaTcCount] = 0;
+      p.ws.meta[kMetaDone] = 0;
+      p.ws.meta[kMetaTcQueue] = 0;
+    }
+    float4* y4 = reinterpret_cast<float4*>(p.ws.y);  // the output accumulator row
+    for (int i = tid; i < d / 4; i += kThreads) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+      asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.ws.meta + kMetaRoute1), "r"(1)
+                   : "memory");
+  }
+  __syncthreads();
+}
+
 // Two CTAs per SM for groups of <= 32 tokens: at most 168 registers a thread.
 __global__ void __launch_bounds__(kThreads, 2)
     gate_up_tc_kernel(const __grid_constant__ GateUpTcParams p) {
@@ -666,8 +788,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int n_rg = __ldcg(p.ws.meta + kMetaRoutedGroups);
-  const int n_g = __ldcg(p.ws.meta + kMetaGroups);
+  const Route1Groups* r1 = nullptr;
+  if (p.dm.route1) {
+    route1_prologue(p, reinterpret_cast<float*>(smem), fscr->r1, warp, lane);
+    r1 = &fscr->r1;
+  }
+  const int n_rg = r1 ? r1->k : __ldcg(p.ws.meta + kMetaRoutedGroups);
+  const int n_g = r1 ? r1->k : __ldcg(p.ws.meta + kMetaGroups);
   const int tiles_r = p.dm.F / kNeuronTile;
   const int tiles_s = p.dm.S > 0 ? p.dm.Fs / kNeuronTile : 1;
   const int n_units = n_rg * tiles_r + (n_g - n_rg) * tiles_s;
@@ -684,20 +811,20 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (p.dm.S > 0) {
         tma_prefetch_desc(&p.tm_wgs);
         tma_prefetch_desc(&p.tm_wus);
-        tma_prefetch_desc(&p.tm_x);
       }
+      if (p.dm.S > 0 || r1) tma_prefetch_desc(&p.tm_x);
     }
     uint32_t it = 0;
     bool ok = true;
     Segs sg = segs_begin(n_units, KB, split);
     int u, kb0, kb1;
     while (ok && segs_next(sg, u, kb0, kb1)) {
-      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
+      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s, r1);
       const int N = (ui.gr.m + 15) & ~15;
       const int nb = N / kBRowBox;
       const CUtensorMap* mg = ui.shared ? &p.tm_wgs : &p.tm_wg;
       const CUtensorMap* mu = ui.shared ? &p.tm_wus : &p.tm_wu;
-      const CUtensorMap* mx = ui.shared ? &p.tm_x : &p.tm_xperm;
+      const CUtensorMap* mx = ui.shared || r1 ? &p.tm_x : &p.tm_xperm;
       const int kstep = ui.gate_only && p.b_blocks == 2 ? 2 : 1;  // K-blocks per stage
       for (int kb = kb0; kb < kb1; kb += kstep, ++it) {
         const uint32_t s = it % stages;
@@ -744,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     Segs sg = segs_begin(n_units, KB, split);
     int u, kb0, kb1;
     for (; ok && segs_next(sg, u, kb0, kb1); ++uidx) {
-      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
+      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s, r1);
       const int N = (ui.gr.m + 15) & ~15;
       const uint32_t idesc = idesc_bf16_f32(kNeuronTile, N, 0, 0);
       const uint32_t b = uidx % p.nbuf;
@@ -806,12 +933,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t uidx = 0;
     bool ok = true;
     int park_u = -1;  // split unit whose last K-block is ours: finished at the end
+    // routing in this kernel: the first CTA's records (and zeroed counters)
+    // are in place before this warp's first atomic add
+    if (r1 && blockIdx.x != 0) {
+      if (lane == 0 && !wait_flag(p.ws.meta + kMetaRoute1, abort_flag, p.ws.status)) ok = false;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
     Segs sg = segs_begin(n_units, KB, split);
     int u, kb0, kb1;
     for (; segs_next(sg, u, kb0, kb1); ++uidx) {
       // every epilogue warp walks every segment (named barriers below), doing
       // nothing once a wait has failed
-      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s);
+      const UnitInfo ui = decode_unit(p, u, n_rg, tiles_r, tiles_s, r1);
       const int g = group_of_unit(u, n_rg, tiles_r, tiles_s);
       const int m = ui.gr.m;
       const int N = (m + 15) & ~15;
@@ -908,7 +1041,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       epi_sync();
       if (*fix_ok) {
-        const UnitInfo ui = decode_unit(p, park_u, n_rg, tiles_r, tiles_s);
+        const UnitInfo ui = decode_unit(p, park_u, n_rg, tiles_r, tiles_s, r1);
         const int g = group_of_unit(park_u, n_rg, tiles_r, tiles_s);
         const int m = ui.gr.m;
         const int N = (m + 15) & ~15;

@@ -93,6 +93,7 @@ enum Meta { kMetaGroups = 0, kMetaRoutedGroups = 1, kMetaDone = 2, kMetaSlotsUse
             kMetaExpertsTouched = 4, kMetaGemvCount = 5, kMetaTcCount = 6,
             kMetaDownDone = 7,  // row-stream CTAs finished (direct combine ticket)
             kMetaTcQueue = 8,   // next tensor-core down unit to hand out
+            kMetaRoute1 = 9,    // one-token routing in the gate/up kernel: layout published
             kMetaWords = 16 };
 
 // counters[] (u64), reset by the router's scan every forward
@@ -157,6 +158,11 @@ struct Dims {
   // 1 (with direct_combine): no row-stream launch follows the gate/up kernel,
   // so its last CTA (a ticket) writes out from the accumulator rows
   int fuse_finish;
+  // 1: a one-token batch with no shared experts whose whole layer runs in the
+  // gate/up kernel: every CTA routes the token itself (logits, top-k; the
+  // selected experts in expert order are the groups, one token each), the
+  // first CTA also writes the routing records, and no router launches
+  int route1;
 };
 
 constexpr int kDirectMax = 16;  // tokens up to which the row stream combines directly
@@ -246,6 +252,8 @@ struct GateUpTcParams {
   const __nv_bfloat16* wu;     // [E*F][d] W_up (gate score: fused up + down of one-token groups)
   const __nv_bfloat16* wus;    // [S*Fs][d] shared experts' W_up
   const __nv_bfloat16* x;      // [T][d] the layer input (shared experts' tokens)
+  const __nv_bfloat16* wr;     // [E][d] W_router (dm.route1)
+  const float* rbias;          // [E] router bias or null (dm.route1)
   void* out;                   // [T][d] layer output (dm.fuse_finish)
   int out_bf16;                // out's type: 1 bf16, 0 fp32
 };

@@ -66,6 +66,16 @@ bool split_enabled() {
   return on;
 }
 
+// One-token routing inside the gate/up kernel (MOE_FUSE_ROUTE=0 turns it off
+// and launches the router, for comparisons).
+bool fuse_route_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_FUSE_ROUTE");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 // Down projection of the smallest row-stream groups inside the gate/up kernel
 // (MOE_FUSE_DOWN=0 turns it off and sends them to the row-stream kernel, for
 // comparisons).
@@ -599,6 +609,13 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
                           ? 1
                           : 0;
   dm.fuse_finish = dm.direct_combine && !need_gemv ? 1 : 0;
+  // one token, every group fused and combined directly, no shared experts, a
+  // small router: the gate/up kernel routes the token itself in every CTA
+  // (no router launch)
+  dm.route1 = dm.fuse_finish && T == 1 && cap.S == 0 && top_k <= 16 &&
+                      (size_t)cap.E * cap.d * 2 <= 64 * 1024 && moe::fuse_route_enabled()
+                  ? 1
+                  : 0;
   // the tensor-core down launch's grid is fixed here: the router's layout
   // and the kernel both derive the units' K parts from it
   const int tc_ctas_per_sm = n_max <= 64 ? 2 : 1;
@@ -612,7 +629,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
 
   if (c->bf16) {
     if (!build_weight_maps(c, W_gate, W_up, W_down)) return MOE_ERR_CUDA;
-    if (cap.S > 0 && (c->c_x != x || c->c_xT != T)) {
+    if ((cap.S > 0 || dm.route1) && (c->c_x != x || c->c_xT != T)) {
       if (!encode2d(&c->tm_x, x, cap.d, (uint64_t)T, (uint64_t)cap.d * 2, 64, 16, c->err))
         return MOE_ERR_CUDA;
       c->c_x = x;
@@ -633,9 +650,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   };
   cudaError_t e;
   mark(0);
-  e = moe::launch_route(dm, c->ws, x, W_router, router_bias, c->bf16, st);
-  if (e != cudaSuccess) return cuda_fail(c, e, "route launch");
-  stage_ran[0] = true;
+  if (!dm.route1) {
+    e = moe::launch_route(dm, c->ws, x, W_router, router_bias, c->bf16, st);
+    if (e != cudaSuccess) return cuda_fail(c, e, "route launch");
+    stage_ran[0] = true;
+  }
   mark(1);
   if (!moe::route_is_small(dm)) {
     e = moe::launch_permute(dm, c->ws, x, c->bf16, st);
@@ -677,6 +696,8 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     p.wu = static_cast<const __nv_bfloat16*>(W_up);
     p.wus = static_cast<const __nv_bfloat16*>(c->Wus);
     p.x = static_cast<const __nv_bfloat16*>(x);
+    p.wr = static_cast<const __nv_bfloat16*>(W_router);
+    p.rbias = router_bias;
     p.out = out;
     p.out_bf16 = out_bf16 ? 1 : 0;
     const int grid = gu_grid;
