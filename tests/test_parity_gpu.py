@@ -392,6 +392,31 @@ def test_fused_down_matches_row_stream(name, T):
     compare(fused, oracle_forward(dw, x, tau, ts), tau, ts, "bf16", dw=dw)
 
 
+def test_one_token_layer_is_one_launch(mixtral):
+    """T = 1 on the Mixtral-shaped layer: every CTA of the gate/up kernel
+    routes the token itself, so the whole layer is one kernel launch (the
+    first CTA writes the routing records the getters read); the routing, the
+    active sets, the statistics and the output match the oracle, with the
+    |h| score and with the gate score."""
+    if os.environ.get("MOE_FUSE_DOWN") == "0" or os.environ.get("MOE_FUSE_ROUTE") == "0":
+        pytest.skip("fused paths turned off")
+    wl, dw = mixtral
+    x = workload_tokens(wl, 1)
+    for score in ("h", "gate"):
+        tau, _ = tau_of("mixtral_decode", 0.7, score=score)
+        layer = make_layer(wl.shape, 64, score=score)
+        before = layer.launch_count()
+        gpu = run_gpu(layer, dw, x, tau)
+        assert layer.launch_count() - before == 1
+        compare(gpu, oracle_forward(dw, x, tau, score=score), tau, 0.0, "bf16", dw=dw,
+                score=score)
+        st = gpu["stats"]
+        assert st["n_groups"] == 2 and st["n_experts_touched"] == 2 and st["n_groups_gemv"] == 2
+        assert st["down_rows_fused"] == st["down_rows_read"] > 0
+        assert layer.status() == 0
+        layer.close()
+
+
 def test_small_groups_join_tensor_cores(mixtral):
     """When at least half of a batch's groups hold more than 8 tokens (all
     rows on the tensor cores by size), the batch's smaller groups join them
