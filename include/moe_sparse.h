@@ -129,7 +129,12 @@ typedef struct {
                                  (|h| score, bf16) groups of 5..8 tokens choose after gate/up:
                                  the GEMV path if their active-row union is <= 0.8 x d_ff,
                                  else all rows on the tensor cores */
-  float gather_max_density;   /* AUTO: gathered TC if union <= this fraction of d_ff (0: never) */
+  float gather_max_density;   /* AUTO (bf16): a tensor-core group of <= 64 tokens whose
+                                 active-row union is <= this fraction of d_ff reads only
+                                 the union rows (gathered copies, packed in shared memory)
+                                 instead of all rows; 0: never. The Python binding's
+                                 default is 0.5 (the gathered stream runs at about 2/3 of
+                                 the all-rows stream's bandwidth) */
   int32_t score;              /* moe_score (0: MOE_SCORE_H) */
   int32_t out_f32;            /* 1: out is float32 [T][d_model] for either dtype (the combine's
                                  fp32 sums, not rounded; for partial outputs that are summed

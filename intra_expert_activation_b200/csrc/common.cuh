@@ -164,20 +164,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Four rows of a 2-D tensor whose box is one row high (tile::gather4): rows
-// y0..y3 at inner coordinate x land one after another at dst (4 box rows),
-// completion counted on bar. Callers pass rows inside the tensor.
-__device__ __forceinline__ void tma_gather4_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                               int32_t x, int32_t y0, int32_t y1, int32_t y2,
-                                               int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-      "r"(y3)
-      : "memory");
-}
-
 // Same with an L2 eviction-priority hint (streamed weights: evict first).
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map,
                                                  uint64_t* bar, int32_t x, int32_t y,

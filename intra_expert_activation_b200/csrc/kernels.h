@@ -184,12 +184,14 @@ constexpr int kDirectMax = 16;  // tokens up to which the row stream combines di
 constexpr int kTcMaxParts = 24;
 constexpr int kTcPartTokens = 64;
 __host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
-  if (dm.mode == kModeTc || n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
+  if (n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
   const int tmax = dm.T < kGroupMax ? dm.T : kGroupMax;
   if ((tmax + 15) / 16 * 16 > kTcPartTokens) return 1;
   const long long grid = dm.tc_grid;
   const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);
-  if (4 * base >= 3 * grid) return 1;
+  // forced gathered rows: the units' lengths follow their groups' unions,
+  // so they are always cut (the queue then evens out the CTAs)
+  if (dm.mode != kModeTc && 4 * base >= 3 * grid) return 1;
   const int f_min = dm.S > 0 && dm.Fs < dm.F ? dm.Fs : dm.F;
   long long ks = (2 * grid + base - 1) / base;
   if (ks > kTcMaxParts) ks = kTcMaxParts;
@@ -260,9 +262,12 @@ struct GateUpTcParams {
 
 // ------------------------------------------------------------ down (tcgen05)
 struct DownTcParams {
-  CUtensorMap tm_wd_row, tm_wd_blk;    // [E*F][d]: box {64,1} and {64,64}
-  CUtensorMap tm_wds_row, tm_wds_blk;  // [S*Fs][d]
-  CUtensorMap tm_ht_row, tm_ht_blk;    // [F_max][slots_total]: box {64,1} and {64,64}
+  CUtensorMap tm_wd_blk;   // [E*F][d], box {64,64}
+  CUtensorMap tm_wds_blk;  // [S*Fs][d]
+  CUtensorMap tm_ht_blk;   // [F_max][slots_total], box {64,64}
+  const void* wd;          // the same three arrays for the gathered rows' 16-byte copies
+  const void* wds;
+  const void* ht;
   Dims dm;
   Workspace ws;
   int n_max;        // largest MMA N of this launch
@@ -293,7 +298,7 @@ cudaError_t launch_down_gemv(const Dims& dm, const Workspace& ws, const void* Wd
                              const void* Wds, bool bf16, int n_sms, void* out, bool out_bf16,
                              cudaStream_t st);
 cudaError_t launch_down_tc(const DownTcParams& p, int grid, size_t smem, cudaStream_t st);
-size_t down_tc_smem_bytes(int b_bytes, int stages);
+size_t down_tc_smem_bytes(int b_bytes, int stages, int fw);
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,
                            cudaStream_t st);
 #if defined(MOE_CHECK) && MOE_CHECK

@@ -339,7 +339,7 @@ struct moe_sparse_ctx {
   int c_xT = -1;
   bool maps_shared_ok = false;
   CUtensorMap tm_wg, tm_wu, tm_wgs, tm_wus, tm_xperm, tm_x;
-  CUtensorMap tm_wd_row, tm_wd_blk, tm_wds_row, tm_wds_blk, tm_ht_row, tm_ht_blk;
+  CUtensorMap tm_wd_blk, tm_wds_blk, tm_ht_blk;
   // last forward
   Dims last;
   bool has_last = false;
@@ -378,7 +378,6 @@ bool build_weight_maps(moe_sparse_ctx* c, const void* Wg, const void* Wu, const 
     c->c_wu = Wu;
   }
   if (c->c_wd != Wd) {
-    if (!encode2d(&c->tm_wd_row, Wd, k.d, (uint64_t)k.E * k.F, rb, 64, 1, c->err)) return false;
     if (!encode2d(&c->tm_wd_blk, Wd, k.d, (uint64_t)k.E * k.F, rb, 64, 64, c->err)) return false;
     c->c_wd = Wd;
   }
@@ -480,7 +479,6 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   if (c->bf16) {
     const Dims& k = c->lay.cap;
     bool ok = encode2d(&c->tm_xperm, w.xperm, k.d, k.slots_routed, (uint64_t)k.d * 2, 64, 16, err) &&
-              encode2d(&c->tm_ht_row, w.ht, k.slots_total, k.F_max, (uint64_t)k.slots_total * 2, 64, 1, err) &&
               encode2d(&c->tm_ht_blk, w.ht, k.slots_total, k.F_max, (uint64_t)k.slots_total * 2, 64, 64, err);
     if (!ok) {
       cudaFree(c->mem);
@@ -492,7 +490,6 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
     c->tm_wgs = c->tm_xperm;
     c->tm_wus = c->tm_xperm;
     c->tm_x = c->tm_xperm;
-    c->tm_wds_row = c->tm_ht_row;
     c->tm_wds_blk = c->tm_ht_blk;
   }
   *out = c;
@@ -512,7 +509,6 @@ moe_status moe_sparse_set_shared(moe_sparse_ctx* c, const void* Wg_s, const void
     const uint64_t rb = (uint64_t)k.d * 2, rows = (uint64_t)k.S * k.Fs;
     if (!encode2d(&c->tm_wgs, Wg_s, k.d, rows, rb, 64, 128, c->err) ||
         !encode2d(&c->tm_wus, Wu_s, k.d, rows, rb, 64, 128, c->err) ||
-        !encode2d(&c->tm_wds_row, Wd_s, k.d, rows, rb, 64, 1, c->err) ||
         !encode2d(&c->tm_wds_blk, Wd_s, k.d, rows, rb, 64, 64, c->err))
       return MOE_ERR_CUDA;
   }
@@ -557,6 +553,9 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   const bool dense = c->desc.path == MOE_PATH_DENSE;
   const int mode = c->desc.path;
   const int tmax = std::min(T, moe::kGroupMax);  // no group holds more tokens
+  // AUTO only: tensor-core groups whose union is at most this fraction of
+  // d_ff read only the union rows (the forced paths fix the rows they read)
+  if (mode != MOE_PATH_AUTO) dm.gather_density = 0.f;
   bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) && tmax <= cap.gemv_max);
@@ -740,23 +739,25 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   mark(6);
   if (need_tc) {
     moe::DownTcParams p;
-    p.tm_wd_row = c->tm_wd_row;
     p.tm_wd_blk = c->tm_wd_blk;
-    p.tm_wds_row = c->tm_wds_row;
     p.tm_wds_blk = c->tm_wds_blk;
-    p.tm_ht_row = c->tm_ht_row;
-    p.tm_ht_blk = c->tm_ht_blk;
+    p.wd = W_down;
+    p.wds = c->Wds;
+    p.ht = c->ws.ht;
     p.dm = dm;
     p.ws = c->ws;
     p.n_max = n_max;
+    p.tm_ht_blk = c->tm_ht_blk;
     p.b_bytes = std::max(8192, (n_max + 63) / 64 * 8192);
     p.tmem_cols = pow2_at_least(2u * n_max);
     // small groups (decode): two CTAs per SM so that a unit's epilogue and
     // the next unit's loads overlap across CTAs; large groups: one CTA
-    const size_t budget = tc_ctas_per_sm == 2 ? 113 * 1024 : 225 * 1024;
-    const size_t stage_bytes = 16384 + (size_t)p.b_bytes;
-    p.stages = (int)std::min<size_t>(8, (budget - 2048) / stage_bytes);
-    const size_t smem = moe::down_tc_smem_bytes(p.b_bytes, p.stages);
+    // (per SM 228 KB, of which each CTA's static shared memory and 1 KB the
+    // system reserves)
+    const size_t budget = tc_ctas_per_sm == 2 ? 113 * 1024 - 128 : 225 * 1024;
+    p.stages = 8;
+    while (p.stages > 2 && moe::down_tc_smem_bytes(p.b_bytes, p.stages, dm.fw) > budget) --p.stages;
+    const size_t smem = moe::down_tc_smem_bytes(p.b_bytes, p.stages, dm.fw);
     e = moe::launch_down_tc(p, dm.tc_grid, smem, st);
     if (e != cudaSuccess) return cuda_fail(c, e, "down_tc launch");
     stage_ran[6] = true;

@@ -34,7 +34,7 @@ class MoESparseLayer:
                  max_tokens: int, renormalize: bool = True, n_shared: int = 0,
                  d_ff_shared: int = 0, dtype: str = "bf16", path: str = "auto",
                  debug: bool = False, device: int = 0, gemv_max_tokens: int = 0,
-                 gather_max_density: float = 0.0, score: str = "h", out_f32: bool = False):
+                 gather_max_density: float = 0.5, score: str = "h", out_f32: bool = False):
         self.lib = _lib.load()
         self.torch_dtype, code = _DT[dtype]
         self.dtype = dtype

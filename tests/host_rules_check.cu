@@ -1,7 +1,8 @@
 // Host-side check of the scheduling rules that the router and the kernels
 // share (compiled with nvcc and run on the CPU, no GPU call): the K parts of
 // the tensor-core down units stay inside the workspace's part buffers and
-// tickets and give every part at least one K-block; the candidate-group rule
+// tickets and give every part of an all-rows unit at least one K-block (a
+// part of a gathered unit may have none: it adds zeros); the candidate-group rule
 // is the stated threshold; the row-stream stage geometry fits its budget.
 // Exits non-zero with the first violated case.
 #include <cstdio>
@@ -58,12 +59,15 @@ static void check_ksplit() {
                     const int ks = tc_ksplit(dm, n_tc);
                     const long long base = (long long)n_tc * nslices;
                     CHECK(ks >= 1 && ks <= kTcMaxParts, "ks %d", ks);
-                    if (mode == kModeTc || n_max > kTcPartTokens || cap_units == 0 || grid == 0)
+                    if (n_max > kTcPartTokens || cap_units == 0 || grid == 0)
                       CHECK(ks == 1, "mode %d n_max %d cap %d grid %d ks %d", mode, n_max,
                             cap_units, grid, ks);
                     if (ks > 1) {
                       CHECK(base * ks <= cap_units, "base %lld ks %d cap %d", base, ks, cap_units);
-                      CHECK(4 * base < 3LL * grid, "base %lld grid %d", base, grid);
+                      // units are cut only when they fill under 3/4 of the grid, except
+                      // forced gathered launches (units as long as their unions)
+                      if (mode != kModeTc)
+                        CHECK(4 * base < 3LL * grid, "base %lld grid %d", base, grid);
                       // every part of every expert kind has at least one K-block
                       for (int kind = 0; kind < (S > 0 ? 2 : 1); ++kind) {
                         const int nk = (kind ? dm.Fs : F) / kKBlock;

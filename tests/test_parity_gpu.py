@@ -457,3 +457,58 @@ def test_candidate_groups_choose_by_union(sweep):
         seen_gemv += cand_gemv
         seen_tc += cand_tc
     assert seen_gemv > 0 and seen_tc > 0
+
+
+def _union_rows(gpu, F):
+    """Active-row union size of every routed expert group, from the GPU's own
+    active sets (one group per expert at these batch sizes)."""
+    act = unpack_bits(gpu["active_bits"], F)
+    idx = gpu["topk_idx"].ravel()
+    return {int(e): (int((idx == e).sum()), int(act[idx == e].any(axis=0).sum()))
+            for e in np.unique(idx)}
+
+
+@pytest.mark.parametrize("T,q", [(16, 0.9), (24, 0.7)])
+def test_auto_gathers_tensor_core_unions(sweep, T, q):
+    """AUTO with gather_max_density = 1 and every group of >= 2 tokens on the
+    tensor cores: each such group reads only its union rows, packed by the
+    gather warps, so every group (row stream or tensor cores) reads exactly
+    its union; with the density at 0 the same groups read all rows. Both
+    outputs match the oracle."""
+    wl, dw = sweep
+    F = wl.shape.d_ff
+    tau, _ = tau_of("mixtral_sweep", q)
+    x = workload_tokens(wl, T)
+    g1, _, _ = _check(make_layer(wl.shape, T, gemv_max_tokens=1, gather_max_density=1.0), dw, x,
+                      tau, 0.0, "bf16")
+    g0, _, _ = _check(make_layer(wl.shape, T, gemv_max_tokens=1, gather_max_density=0.0), dw, x,
+                      tau, 0.0, "bf16")
+    groups = _union_rows(g1, F)
+    s1, s0 = g1["stats"], g0["stats"]
+    assert s1["n_groups_tc_gather"] > 0 and s1["n_groups_tc_allrows"] == 0
+    assert s1["down_rows_read"] == sum(u for _, u in groups.values())
+    assert s0["n_groups_tc_gather"] == 0
+    assert s0["n_groups_tc_allrows"] == s1["n_groups_tc_gather"]
+    assert s0["down_rows_read"] == s1["down_rows_gemv"] + s0["n_groups_tc_allrows"] * F
+
+
+@pytest.mark.parametrize("q", [0.998, None])
+def test_gathered_k_parts_with_tiny_unions(sweep, q):
+    """A few gathered tensor-core groups (6 tokens, groups of 2 and 3 tokens
+    on the tensor cores) are cut into K parts to fill the grid; with unions
+    of a few dozen rows (or none, tau = inf) most parts have no K-block and
+    contribute zeros to the ticketed part sums. The output matches the
+    oracle."""
+    wl, dw = sweep
+    x = workload_tokens(wl, 6)
+    tau = _calibrated(dw, x, q)[0] if q is not None else math.inf
+    layer = make_layer(wl.shape, 6, gemv_max_tokens=1, gather_max_density=1.0)
+    gpu, _, _ = _check(layer, dw, x, tau, 0.0, "bf16")
+    st = gpu["stats"]
+    groups = _union_rows(gpu, wl.shape.d_ff)
+    assert st["n_groups_tc_allrows"] == 0
+    assert st["n_groups_tc_gather"] + st["n_groups_gemv"] == len(groups)
+    assert st["n_groups_tc_gather"] >= sum(1 for m, _ in groups.values() if m >= 2) > 0
+    assert st["down_rows_read"] == sum(u for _, u in groups.values())
+    if q is None:
+        assert not np.abs(gpu["out"]).any()
