@@ -76,6 +76,10 @@ def parse():
                     help="h: active iff |SiLU(g) u| > tau; gate: active iff |SiLU(g)| > tau with "
                          "the sparse up projection (the pages' own system)")
     ap.add_argument("--tokens", type=str, default="", help="comma list overriding the batches")
+    ap.add_argument("--path", default="auto",
+                    choices=("auto", "sparse_gemv", "sparse_tc", "sparse_tc_allrows"),
+                    help="down-projection path of the sparse arm (default: the automatic "
+                         "per-group choice; the others force one path, e.g. to profile it)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-path comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-e2e", action="store_true",
@@ -210,13 +214,16 @@ def replica_value(tokens_per_step: int, steps: int, world: int, ms: float) -> fl
 def workload_config(args, wl, tokens, tau, calib_sparsity, world) -> dict:
     """The config block both arms print for a workload."""
     sh = wl.shape
-    return {"workload": args.workload, "score": args.score, "batches": tokens,
-            "tokens_per_step": sum(tokens),
-            "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
-            "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
-            "calibrated_sparsity": round(calib_sparsity, 4),
-            "l2": "no flush: touched expert weights (>= 470 MB per forward) exceed L2",
-            "parallelism": f"replicas x{world}"}
+    cfg = {"workload": args.workload, "score": args.score, "batches": tokens,
+           "tokens_per_step": sum(tokens),
+           "d_model": sh.d_model, "n_experts": sh.n_experts, "top_k": sh.top_k,
+           "d_ff": sh.d_ff, "target_sparsity": args.sparsity, "tau": tau,
+           "calibrated_sparsity": round(calib_sparsity, 4),
+           "l2": "no flush: touched expert weights (>= 470 MB per forward) exceed L2",
+           "parallelism": f"replicas x{world}"}
+    if getattr(args, "path", "auto") != "auto":
+        cfg["path"] = args.path
+    return cfg
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -482,7 +489,7 @@ def run_ours(args, world, rank, local):
     sweep_on = (not args.no_sweep and world == 1 and args.workload == "mixtral_decode"
                 and args.score == "h" and not args.tokens)
 
-    sparse = make("auto")
+    sparse = make(args.path)
     for _ in range(args.warmup):
         step(sparse)
     torch.cuda.synchronize(dev)
