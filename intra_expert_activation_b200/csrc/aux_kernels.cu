@@ -1,8 +1,9 @@
 // Small kernels between the big ones:
-//  union_scan   (gathered tensor-core mode only) per expert token group:
-//               compact the active-row union bitmap into an ordered row list
-//               and mark groups of <= kGatherMaxTokens tokens for the gathered
-//               path [gist.science EN "Uncovering Intra-expert Activation
+//  union_scan   (forced gathered tensor-core mode only) per expert token
+//               group: mark groups of <= kGatherMaxTokens tokens for the
+//               gathered path and count the rows the down projection reads
+//               (the tensor-core kernel walks the union bitmaps itself)
+//               [gist.science EN "Uncovering Intra-expert Activation
 //               Sparsity for Efficient Mixture-of-Expert Model Execution",
 //               Technical Summary > Methodology > System Implementation in
 //               vLLM > "Fused Up-Down Projection"].
@@ -18,56 +19,15 @@ namespace {
 constexpr int kScanThreads = 256;
 __global__ void __launch_bounds__(kScanThreads) union_scan_kernel(Dims dm, Workspace ws) {
   grid_dep_wait();
-  const int g = blockIdx.x;
-  if (g >= __ldcg(ws.meta + kMetaGroups)) return;
-  const Group gr = ws.groups[g];
-  const bool shared = gr.expert >= dm.E;
-  const int F_e = shared ? dm.Fs : dm.F;
-  const int words = F_e / 32;
-  const uint32_t* bits = ws.union_bits + static_cast<size_t>(g) * dm.fw;
-  int* rows = ws.union_rows + static_cast<size_t>(g) * dm.F_max;
-
-  __shared__ int warp_tot[kScanThreads / 32];
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // word-ordered exclusive scan of popcounts, kScanThreads words per round
-  for (int w0 = 0; w0 < words; w0 += kScanThreads) {
-    const int w = w0 + threadIdx.x;
-    const uint32_t b = w < words ? __ldcg(bits + w) : 0u;
-    const int c = __popc(b);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int base = carry;
-    for (int i = 0; i < warp; ++i) base += warp_tot[i];
-    int pos = base + incl - c;
-    uint32_t bb = b;
-    while (bb) {
-      const int bit = __ffs(bb) - 1;
-      rows[pos++] = w * 32 + bit;
-      bb &= bb - 1;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int tot = 0;
-      for (int i = 0; i < kScanThreads / 32; ++i) tot += warp_tot[i];
-      carry += tot;
-    }
-    __syncthreads();
-  }
-
-  if (threadIdx.x == 0) {
-    // gathered rows for groups of <= kGatherMaxTokens tokens, all rows above
-    const int cnt = carry;
+  const int n_groups = __ldcg(ws.meta + kMetaGroups);
+  for (int g = blockIdx.x * kScanThreads + threadIdx.x; g < n_groups;
+       g += gridDim.x * kScanThreads) {
+    // gathered rows for groups of <= kGatherMaxTokens tokens, all rows above;
+    // the union's rows were counted by the gate/up epilogue
+    const Group gr = ws.groups[g];
+    const int F_e = gr.expert >= dm.E ? dm.Fs : dm.F;
+    const int cnt = __ldcg(ws.union_cnt + g);
     const int path = gr.m <= kGatherMaxTokens ? kPathTcGather : kPathTcAll;
-    ws.union_cnt[g] = cnt;
     ws.group_path[g] = path;
     atomicAdd(ws.counters + kCntDownRows,
               static_cast<unsigned long long>(path == kPathTcAll ? F_e : cnt));
@@ -190,7 +150,8 @@ cudaError_t launch_wait_timeout(int* status, uint32_t limit, int which, cudaStre
 #endif
 
 cudaError_t launch_union_scan(const Dims& dm, const Workspace& ws, cudaStream_t st) {
-  return launch_k(union_scan_kernel, dm.groups_max, kScanThreads, 0, st, dm, ws);
+  return launch_k(union_scan_kernel, (dm.groups_max + kScanThreads - 1) / kScanThreads,
+                  kScanThreads, 0, st, dm, ws);
 }
 
 cudaError_t launch_combine(const Dims& dm, const Workspace& ws, void* out, bool bf16,

@@ -215,7 +215,6 @@ struct Workspace {
   Group* groups;                // [groups_max]
   int* group_path;              // [groups_max]
   uint32_t* union_bits;         // [groups_max][fw]
-  int* union_rows;              // [groups_max][F_max]
   int* union_cnt;               // [groups_max] rows in each group's union (cleared by the router,
                                 //   accumulated by the gate/up epilogue)
   int* gemv_list;               // [groups_max] groups on the GEMV path (count in meta)

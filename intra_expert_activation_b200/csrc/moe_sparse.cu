@@ -175,7 +175,7 @@ struct Layout {
 
 enum Buf { bStatus, bMeta, bCounters, bTopkIdx, bTopkW, bSlotOf, bRankCta, bHist, bExpOff,
            bExpCnt, bPerm, bGroups, bGroupPath,
-           bUnionBits, bUnionRows, bUnionCnt, bGemvList, bTcList, bYZero, bSlotW, bSkFlags, bSkPart,
+           bUnionBits, bUnionCnt, bGemvList, bTcList, bYZero, bSlotW, bSkFlags, bSkPart,
            bTcTicket, bTcPart, bActBits, bXperm, bHt, bY, bCount };
 
 moe_status check_desc(const moe_sparse_desc* d, std::string& err) {
@@ -267,7 +267,6 @@ Layout make_layout(const moe_sparse_desc* d) {
   sz[bGroups] = sizeof(moe::Group) * c.groups_max;
   sz[bGroupPath] = sizeof(int) * c.groups_max;
   sz[bUnionBits] = sizeof(uint32_t) * c.groups_max * c.fw;
-  sz[bUnionRows] = sizeof(int) * (size_t)c.groups_max * c.F_max;
   sz[bUnionCnt] = sizeof(int) * c.groups_max;
   sz[bGemvList] = sizeof(int) * c.groups_max;
   sz[bTcList] = sizeof(int) * c.groups_max;
@@ -461,7 +460,6 @@ moe_status moe_sparse_init(const moe_sparse_desc* desc, moe_sparse_ctx** out) {
   w.groups = reinterpret_cast<moe::Group*>(b + o[bGroups]);
   w.group_path = reinterpret_cast<int*>(b + o[bGroupPath]);
   w.union_bits = reinterpret_cast<uint32_t*>(b + o[bUnionBits]);
-  w.union_rows = reinterpret_cast<int*>(b + o[bUnionRows]);
   w.union_cnt = reinterpret_cast<int*>(b + o[bUnionCnt]);
   w.gemv_list = reinterpret_cast<int*>(b + o[bGemvList]);
   w.tc_list = reinterpret_cast<int*>(b + o[bTcList]);
