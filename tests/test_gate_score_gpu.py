@@ -66,7 +66,7 @@ def small():
 
 
 @pytest.mark.parametrize("T", [1, 3, 8, 37, 100])
-@pytest.mark.parametrize("path", ["auto", "dense", "sparse_gemv", "sparse_tc_allrows"])
+@pytest.mark.parametrize("path", ["auto", "dense", "sparse_gemv", "sparse_tc", "sparse_tc_allrows"])
 def test_small_bf16_gate_paths(small, T, path):
     x = make_tokens(SMALL.d_model, T, 21, "bf16")
     tau, _ = _gate_taus(small, x, 0.7)
