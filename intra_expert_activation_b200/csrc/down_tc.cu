@@ -19,10 +19,12 @@
 //   gathered mode (groups of <= 64 tokens: forced, or in AUTO when the union
 //     is at most gather_density x d_ff): K-block = the next 64 union rows.
 //     Warp 0 walks the group's union bitmap (copied to shared memory once per
-//     unit) and writes the K-block's row numbers into the stage's index slot;
-//     warps 6-9 copy 16 rows each (A: 16 x 256 B, B: 16 x N slots x 2 B) and
-//     the copies complete on the stage's gather barrier. Positions past the
-//     union are zero-filled (src-size 0) in both operands.
+//     unit) and writes each K-block's row numbers into the next of kIxSlots
+//     row slots (a ring that runs ahead of the copies); warps 6-9 copy 16
+//     rows each (A: 16 x 256 B, B: 16 x N slots x 2 B) into the ring stage,
+//     every lane arriving on the stage's gather barrier when its copies land,
+//     and the MMA thread fences the async proxy before reading. Positions
+//     past the union are zero-filled (src-size 0) in both operands.
 //     (TMA tile::gather4 with one-row boxes, tried first, streamed at about a
 //     third of HBM bandwidth: a CTA's gather copies went out one after the
 //     other; sixteen-byte copies from four warps per CTA, two CTAs per SM,
