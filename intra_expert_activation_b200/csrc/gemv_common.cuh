@@ -67,17 +67,18 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 }
 
 // Stage geometry for a row of row_bytes: the column block (<= block_max),
-// the stage size (kBatch rows at the padded stride, then `extra` bytes of
-// per-stage data) and the number of stages that fit the budget.
+// the stage size (`rows` rows, kBatch by default, at the padded stride, then
+// `extra` bytes of per-stage data) and the number of stages that fit the
+// budget.
 struct Geometry {
   int block, stride, stage, n_stages;
 };
 __host__ __device__ inline Geometry geometry(int row_bytes, int extra,
-                                             int block_max = kBlockBytes) {
+                                             int block_max = kBlockBytes, int rows = kBatch) {
   Geometry g;
   g.block = row_bytes < block_max ? row_bytes : block_max;
   g.stride = g.block + kRowPad;
-  g.stage = kBatch * g.stride + extra;
+  g.stage = rows * g.stride + extra;
   g.n_stages = kSmemBudget / g.stage;
   if (g.n_stages > kMaxStages) g.n_stages = kMaxStages;
   return g;

@@ -167,30 +167,34 @@ struct Rows<float, TILES> {
   }
 };
 
-// d += A (16 x 16, bf16) * B (16 x 8, bf16), fp32 accumulation; rows 8..15
-// of A are zero here.
-__device__ __forceinline__ void mma_16x8x16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
-                                            uint32_t b1) {
+// d += A (16 x 16, bf16) * B (16 x 8, bf16), fp32 accumulation, all 16 rows.
+__device__ __forceinline__ void mma_16x8x16_a4(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// Two 8x8 bf16 matrices from shared memory (lanes 0..15 supply the row addresses).
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r0), "=r"(r1)
+// Four 8x8 bf16 matrices from shared memory (every lane supplies a row address).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                       uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
 }
 
 template <typename TW>
 struct UpDots;
 
-// bf16: 16 K-steps of 16 columns over the warp's 256 columns.
+// bf16: 16 K-steps of 16 columns over the warp's 256 columns, 16 rows a
+// stage (the mma's M).
 template <>
 struct UpDots<__nv_bfloat16> {
   static constexpr int MT = kGemvTokens;
+  static constexpr int kRows = 16;   // rows per stage
+  static constexpr int kParts = 4;   // partial dots per lane and stage
   uint32_t xb[16][2];  // B fragments: x[token g][columns of K-step ks]
 
   // x values of the pass's tokens for this warp's columns [col0, col0 + 256)
@@ -203,31 +207,36 @@ struct UpDots<__nv_bfloat16> {
       xb[ks][1] = g < mt ? __ldcg(reinterpret_cast<const unsigned int*>(xr + 16 * ks + 8)) : 0u;
     }
   }
-  // partial dots of the stage's 8 rows over this warp's slice: p[0..1] =
-  // (row g, tokens c2, c2 + 1)
-  __device__ void dots(uint32_t rows_s, const uint8_t*, int stride, float (&p)[2], int lane) {
+  // partial dots of the stage's 16 rows over this warp's slice: p[0..1] =
+  // (row g, tokens c2, c2 + 1), p[2..3] = (row g + 8, the same tokens)
+  __device__ void dots(uint32_t rows_s, const uint8_t*, int stride, float (&p)[kParts], int lane) {
     float d[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t a_addr = rows_s + (lane & 7) * stride + ((lane >> 3) & 1) * 16;
+    // ldmatrix x4: lanes 0-7 rows 0-7 and lanes 8-15 rows 8-15 at the K-step's
+    // first 8 columns, lanes 16-31 the same rows at its last 8
+    const uint32_t a_addr =
+        rows_s + ((lane & 7) + ((lane >> 3) & 1) * 8) * stride + (lane >> 4) * 16;
 #pragma unroll
     for (int ks = 0; ks < 16; ++ks) {
-      uint32_t a0, a2;
-      ldsm_x2(a_addr + 32 * ks, a0, a2);
-      mma_16x8x16(d, a0, a2, xb[ks][0], xb[ks][1]);
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a_addr + 32 * ks, a0, a1, a2, a3);
+      mma_16x8x16_a4(d, a0, a1, a2, a3, xb[ks][0], xb[ks][1]);
     }
-    p[0] = d[0];
-    p[1] = d[1];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = d[i];
   }
-  // where this lane's two partials go: (row, token) pairs
+  // where this lane's partials go: (row, token) pairs
   __device__ static void owner(int lane, int i, int& row, int& tok) {
-    row = lane >> 2;
-    tok = 2 * (lane & 3) + i;
+    row = (lane >> 2) + 8 * (i >> 1);
+    tok = 2 * (lane & 3) + (i & 1);
   }
 };
 
-// fp32: 4 columns per lane, warp reduction per (row, token).
+// fp32: 4 columns per lane, warp reduction per (row, token), 8 rows a stage.
 template <>
 struct UpDots<float> {
   static constexpr int MT = 8;
+  static constexpr int kRows = 8;
+  static constexpr int kParts = 2;
   float xv[MT][4];
 
   __device__ void load_x(const float* xrows, int d, int mt, int col0, int lane) {
@@ -237,11 +246,11 @@ struct UpDots<float> {
       for (int i = 0; i < 4; ++i)
         xv[t][i] = t < mt ? __ldcg(xrows + (size_t)t * d + col0 + 4 * lane + i) : 0.f;
   }
-  __device__ void dots(uint32_t, const uint8_t* rows, int stride, float (&p)[2], int lane) {
+  __device__ void dots(uint32_t, const uint8_t* rows, int stride, float (&p)[kParts], int lane) {
     // 64 (row, token) sums; lane l ends with those of (row l / 8, tokens ..)
     p[0] = p[1] = 0.f;
 #pragma unroll 1
-    for (int r = 0; r < kBatch; ++r) {
+    for (int r = 0; r < kRows; ++r) {
       const float4 w = *reinterpret_cast<const float4*>(rows + r * stride + lane * 16);
 #pragma unroll
       for (int t = 0; t < MT; ++t) {

@@ -34,7 +34,8 @@ namespace moe {
 
 namespace {
 
-constexpr int kMetaBytes = 48;  // per stage after the rows: 2 x int4 + 8 row indices
+constexpr int kStageRowsMax = 16;  // rows per stage: 16 (bf16), 8 (fp32)
+constexpr int kMetaBytes = 32 + 2 * kStageRowsMax;  // per stage after the rows: 2 x int4 + row indices
 constexpr int kKindDown = 1 << 17;
 
 template <typename TW>
@@ -45,6 +46,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   using U = UpDots<TW>;
   using R = Rows<TW>;
   constexpr int MT = U::MT;
+  // rows per stage: the up dots' mma M (bf16: 16), 8 for fp32; the down
+  // projection takes a stage's rows 8 at a time (its mma's K)
+  constexpr int RB = U::kRows;
+  static_assert(RB % kBatch == 0 && RB <= kStageRowsMax, "stage rows");
   static_assert(R::MT == MT, "tokens per pass");
   constexpr int ES = static_cast<int>(sizeof(TW));
   extern __shared__ __align__(128) uint8_t smem[];
@@ -54,7 +59,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint16_t list[kListRows];
   __shared__ uint16_t rowj[kListRows];              // the current run's neuron indices
   __shared__ float hrun[kListRows][kTokStride];      // the run's dots, then its h values
-  __shared__ float red[2][kConsumers][kBatch][kTok];  // one stage's partial dots per warp
+  __shared__ float red[2][kConsumers][RB][kTok];  // one stage's partial dots per warp
   __shared__ int abort_flag;
 
   grid_dep_wait();
@@ -63,7 +68,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = dm.d;
   const int row_bytes = d * ES;
-  const Geometry geo = geometry(row_bytes, kMetaBytes);
+  const Geometry geo = geometry(row_bytes, kMetaBytes, kBlockBytes, RB);
   const int NS = geo.n_stages;
   const int n_blocks = (row_bytes + kBlockBytes - 1) / kBlockBytes;
   if (threadIdx.x == 0) {
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TW* wexp = (phase ? (shared ? Wds : Wd) : (shared ? Wus : Wu)) + eoff;
         for (int cb = 0; cb < (last_run ? 1 : n_blocks) && ok; ++cb) {
           const int cbytes = min(kBlockBytes, row_bytes - cb * kBlockBytes);
-          for (int pos = 0; pos < n_list || (last_run && pos == 0); pos += kBatch) {
+          for (int pos = 0; pos < n_list || (last_run && pos == 0); pos += RB) {
             const int b = s % NS;
             if (s >= NS &&
                 !warp_wait(empty + b, ((s / NS) + 1) & 1, &abort_flag, ws.status, kTight)) {
@@ -107,23 +112,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint8_t* stg = smem + b * geo.stage;
             const uint32_t stg_s = smem_s + b * geo.stage;
-            const int cnt = last_run ? 0 : min(kBatch, n_list - pos);  // 0: the end marker
+            const int cnt = last_run ? 0 : min(RB, n_list - pos);  // 0: the end marker
             const int last_up = phase == 0 && cb == n_blocks - 1 && pos + cnt >= n_list;
-            if (phase == 1 && cnt < kBatch) {
+            if (phase == 1 && cnt < RB) {
               // W_down rows past the run are the mma's K with zero h: give them
               // finite values (never-written shared memory may hold any bits)
-              for (int r = cnt; r < kBatch; ++r)
+              for (int r = cnt; r < RB; ++r)
                 for (int o = lane * 16; o < geo.block; o += 32 * 16)
                   *reinterpret_cast<uint4*>(stg + r * geo.stride + o) = make_uint4(0u, 0u, 0u, 0u);
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             if (lane == 0) {
-              int4* meta = reinterpret_cast<int4*>(stg + kBatch * geo.stride);
+              int4* meta = reinterpret_cast<int4*>(stg + RB * geo.stride);
               meta[0] = make_int4(last_run ? -1 : k.serial * n_blocks + cb, cnt, slot,
                                   mt | (cb << 8) | (last_up << 16) | (phase ? kKindDown : 0));
               meta[1] = make_int4(pos, k.xrow0 + k.p * MT, shared, n_list);
               uint16_t* rj = reinterpret_cast<uint16_t*>(meta + 2);
-              for (int r = 0; r < kBatch; ++r) {
+              for (int r = 0; r < RB; ++r) {
                 const int j = r < cnt ? list[pos + r] : 0;
                 rj[r] = moe_in_bounds(ws.status, j < 32 * k.words) ? j : 0;  // checked build: clamp
               }
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int4 m0 = make_int4(-1, 0, 0, 0), m1 = make_int4(0, 0, 0, 0);
       const uint8_t* stg = smem + b * geo.stage;
       if (ok) {
-        const int4* meta = reinterpret_cast<const int4*>(stg + kBatch * geo.stride);
+        const int4* meta = reinterpret_cast<const int4*>(stg + RB * geo.stride);
         m0 = meta[0];
         m1 = meta[1];
       }
@@ -173,7 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_slices = cbytes / kSliceBytes;
       const bool active = warp < n_slices;
       const int col0 = (cb * kBlockBytes + warp * kSliceBytes) / ES;
-      float p[2] = {0.f, 0.f};
+      float p[U::kParts];
+#pragma unroll
+      for (int i = 0; i < U::kParts; ++i) p[i] = 0.f;
       if (tag >= 0 && !is_down) {
         if (active) {
           if (tag != up_tag) {
@@ -185,9 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   geo.stride, p, lane);
         }
         if (cb == 0 && warp == 0 && lane < cnt)
-          rowj[pos + lane] = reinterpret_cast<const uint16_t*>(stg + kBatch * geo.stride + 32)[lane];
+          rowj[pos + lane] = reinterpret_cast<const uint16_t*>(stg + RB * geo.stride + 32)[lane];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < U::kParts; ++i) {
           int r, t;
           U::owner(lane, i, r, t);
           red[s & 1][warp][r][t] = p[i];
@@ -205,8 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           dn_mt = mt;
           dn_col0 = col0;
         }
-        down.consume_hf(smem_s + b * geo.stage + warp * kSliceBytes, stg + warp * kSliceBytes,
-                        geo.stride, &hrun[pos][0], cnt, mt, lane);
+#pragma unroll
+        for (int h = 0; h < RB / kBatch; ++h)  // the mma's K is 8 rows
+          if (cnt > h * kBatch)
+            down.consume_hf(smem_s + b * geo.stage + h * kBatch * geo.stride + warp * kSliceBytes,
+                            stg + h * kBatch * geo.stride + warp * kSliceBytes, geo.stride,
+                            &hrun[pos + h * kBatch][0], cnt - h * kBatch, mt, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + b);
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (consumers_any(tag < 0 || !ok)) break;
       if (!is_down) {
         // the stage's dots, summed over the warps in warp order
-        if (threadIdx.x < kBatch * kTok) {
+        if (threadIdx.x < RB * kTok) {
           const int r = threadIdx.x / kTok, t = threadIdx.x % kTok;
           if (r < cnt && t < mt) {
             float v = 0.f;
@@ -242,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 size_t updown_gemv_smem_bytes(int d, bool bf16) {
-  const Geometry g = geometry(d * (bf16 ? 2 : 4), kMetaBytes);
+  const Geometry g = geometry(d * (bf16 ? 2 : 4), kMetaBytes, kBlockBytes, bf16 ? 16 : 8);
   return static_cast<size_t>(g.n_stages) * g.stage;
 }
 
