@@ -50,6 +50,11 @@ constexpr int kErrDeviceInvalid = 1;       // == MOE_ERR_INVALID: an internal co
 constexpr int kErrDeviceTimeout = 5;       // == MOE_ERR_DEVICE_TIMEOUT
 
 constexpr int kGroupMax = 128;      // tokens per expert token group (gate/up tile N)
+// Decode batches of 33-64 tokens whose experts average at most 16 tokens
+// (Mixtral-shaped T = 64: 128 pairs over 8 experts) cap their groups at this
+// many tokens, so that gate/up runs 32-column tiles at two CTAs per SM; an
+// expert with more tokens becomes two groups (its weights are read twice).
+constexpr int kGroupMaxDecode = 32;
 constexpr int kGatherMaxTokens = 64;  // groups on the gathered TC path hold <= 64 tokens
 constexpr int kSlotAlign = 8;       // expert slot ranges start at multiples of 8 slots
 constexpr int kNeuronTile = 128;    // gate/up neurons per MMA tile (M)
@@ -163,7 +168,19 @@ struct Dims {
   // selected experts in expert order are the groups, one token each), the
   // first CTA also writes the routing records, and no router launches
   int route1;
+  // tokens per group at most in this forward: kGroupMax, or kGroupMaxDecode
+  // (group_cap); the router's groups and every launch's tile width follow it
+  int gcap;
 };
+
+// The group cap of a forward (Dims::gcap) from the layer's capacity record
+// (E, S, no_tc) and the batch.
+__host__ __device__ inline int group_cap(const Dims& cap, int T, int k) {
+  if (!cap.no_tc && cap.S == 0 && T > kGroupMaxDecode && T <= 2 * kGroupMaxDecode &&
+      2 * T * k <= kGroupMaxDecode * cap.E)
+    return kGroupMaxDecode;
+  return kGroupMax;
+}
 
 constexpr int kDirectMax = 16;  // tokens up to which the row stream combines directly
 
@@ -185,7 +202,7 @@ constexpr int kTcMaxParts = 24;
 constexpr int kTcPartTokens = 64;
 __host__ __device__ inline int tc_ksplit(const Dims& dm, int n_tc) {
   if (n_tc <= 0 || dm.tc_grid <= 0 || dm.tc_part_units <= 0) return 1;
-  const int tmax = dm.T < kGroupMax ? dm.T : kGroupMax;
+  const int tmax = dm.T < dm.gcap ? dm.T : dm.gcap;
   if ((tmax + 15) / 16 * 16 > kTcPartTokens) return 1;
   const long long grid = dm.tc_grid;
   const long long base = static_cast<long long>(n_tc) * (dm.d / kDownSlice);

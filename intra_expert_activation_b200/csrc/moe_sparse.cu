@@ -238,8 +238,17 @@ Layout make_layout(const moe_sparse_desc* d) {
   c.slots_routed = roundup(P + (moe::kSlotAlign - 1) * std::min(c.E, P), moe::kSlotAlign);
   c.T_pad = roundup(c.T, moe::kSlotAlign);
   c.slots_total = c.slots_routed + c.S * c.T_pad;
-  c.groups_max = P / moe::kGroupMax + std::min(c.E, P) +
-                 c.S * ((c.T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
+  // groups at most: whole groups of the forward's cap plus one partial group
+  // per touched expert (the cap is kGroupMaxDecode only for T <= 64)
+  {
+    auto bound = [&](int T_, int cap_) {
+      const int P_ = T_ * c.k;
+      return P_ / cap_ + std::min(c.E, P_) + c.S * ((T_ + cap_ - 1) / cap_) + 1;
+    };
+    c.groups_max = std::max(bound(c.T, moe::kGroupMax),
+                            bound(std::min(c.T, 2 * moe::kGroupMaxDecode), moe::kGroupMaxDecode));
+  }
+  c.gcap = moe::kGroupMax;
   c.mode = d->path;
   c.gemv_max = d->gemv_max_tokens > 0 ? d->gemv_max_tokens : 4;
   // automatic threshold: groups of 5..kGemvCandMax tokens choose after gate/up
@@ -546,11 +555,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   dm.T = T;
   dm.k = top_k;
   const int P = T * top_k;
-  dm.groups_max = P / moe::kGroupMax + std::min(cap.E, P) +
-                  cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) + 1;
+  dm.gcap = moe::group_cap(cap, T, top_k);
+  dm.groups_max = P / dm.gcap + std::min(cap.E, P) + cap.S * ((T + dm.gcap - 1) / dm.gcap) + 1;
   const bool dense = c->desc.path == MOE_PATH_DENSE;
   const int mode = c->desc.path;
-  const int tmax = std::min(T, moe::kGroupMax);  // no group holds more tokens
+  const int tmax = std::min(T, dm.gcap);  // no group holds more tokens
   // AUTO only: tensor-core groups whose union is at most this fraction of
   // d_ff read only the union rows (the forced paths fix the rows they read)
   if (mode != MOE_PATH_AUTO) dm.gather_density = 0.f;
@@ -565,8 +574,8 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   dm.sparse_up = dm.score_gate && tau > 0.f ? 1 : 0;
   // gate/up units (group x 128-neuron tile) at most, and the launch's CTAs
   const int gu_units_max =
-      (P / moe::kGroupMax + std::min(cap.E, P)) * (cap.F / moe::kNeuronTile) +
-      cap.S * ((T + moe::kGroupMax - 1) / moe::kGroupMax) * (cap.Fs / moe::kNeuronTile);
+      (P / dm.gcap + std::min(cap.E, P)) * (cap.F / moe::kNeuronTile) +
+      cap.S * ((T + dm.gcap - 1) / dm.gcap) * (cap.Fs / moe::kNeuronTile);
   const int gu_ctas_per_sm = n_max <= 32 ? 2 : 1;
   // (with fewer units than CTA slots, one unit per CTA: cutting the units
   // along K over the full grid to even out the SMs measured slower, 120 vs

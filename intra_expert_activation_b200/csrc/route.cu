@@ -204,7 +204,7 @@ __device__ __forceinline__ int adds_into_y(int path) {
 }
 
 // ng groups of gsz tokens (a multiple of kSlotAlign; the last one has
-// m_last), each at most kGroupMax.
+// m_last), each at most dm.gcap (a multiple of kSlotAlign).
 struct EntryCut {
   int me, ng, gsz, m_last, F_e, path_full, path_last;
 };
@@ -234,7 +234,7 @@ __device__ __forceinline__ EntryCut entry_cut(const Dims& dm, const int* cnt, in
     c.path_full = c.path_last = kPathGemv;
     return c;
   }
-  const int n_g = (c.me + kGroupMax - 1) / kGroupMax;
+  const int n_g = (c.me + dm.gcap - 1) / dm.gcap;
   c.gsz = ((c.me + n_g - 1) / n_g + kSlotAlign - 1) / kSlotAlign * kSlotAlign;
   c.ng = (c.me + c.gsz - 1) / c.gsz;
   c.m_last = c.me - (c.ng - 1) * c.gsz;

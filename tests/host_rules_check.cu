@@ -42,8 +42,10 @@ static void check_ksplit() {
           for (int Fsh : {128, 1408})
             for (int T : Ts)
               for (int grid : grids)
-                for (int cap_units : units_caps) {
+                for (int cap_units : units_caps)
+                  for (int gcap : {kGroupMax, kGroupMaxDecode}) {
                   Dims dm = {};
+                  dm.gcap = gcap;
                   dm.mode = mode;
                   dm.d = d;
                   dm.F = F;
@@ -53,7 +55,7 @@ static void check_ksplit() {
                   dm.tc_grid = grid;
                   dm.tc_part_units = cap_units;
                   const int nslices = d / kDownSlice;
-                  const int tmax = T < kGroupMax ? T : kGroupMax;
+                  const int tmax = T < gcap ? T : gcap;
                   const int n_max = (tmax + 15) / 16 * 16;
                   for (int n_tc = 0; n_tc <= 700; n_tc += (n_tc < 40 ? 1 : 37)) {
                     const int ks = tc_ksplit(dm, n_tc);
@@ -130,6 +132,23 @@ static void check_geometry() {
 }
 
 int main() {
+  // group cap: a multiple of the slot block (groups stay inside their
+  // expert's slot range), and below kGroupMax only for 33-64 token batches
+  // of routed-only tensor-core layers
+  static_assert(kGroupMaxDecode % kSlotAlign == 0 && kGroupMax % kSlotAlign == 0, "caps");
+  for (int T = 1; T <= 300; ++T)
+    for (int E = 1; E <= 256; E *= 2)
+      for (int S = 0; S <= 1; ++S)
+        for (int no_tc = 0; no_tc <= 1; ++no_tc) {
+          Dims cap = {};
+          cap.E = E;
+          cap.S = S;
+          cap.no_tc = no_tc;
+          const int g = group_cap(cap, T, 2);
+          const bool small = !no_tc && !S && T > 32 && T <= 64 && 4 * T <= 32 * E;
+          CHECK(g == (small ? kGroupMaxDecode : kGroupMax), "T %d E %d S %d cap %d", T, E, S, g);
+        }
+
   check_ksplit();
   check_candidates();
   check_geometry();

@@ -292,6 +292,27 @@ def test_mixtral_decode_paths(mixtral, path):
     _check(layer, dw, workload_tokens(wl, 32), tau, 0.0, "bf16", dense=(path == "dense"))
 
 
+# routed-only layer whose experts average <= 16 tokens at T <= 64, with a
+# router bias that sends most tokens to one or two experts
+SKEWED = LayerShape(d_model=512, n_experts=16, top_k=2, d_ff=384, renormalize=True,
+                    dtype="bf16", router_bias_var=9.0)
+
+
+@pytest.mark.parametrize("T", [40, 48, 64])
+@pytest.mark.parametrize("path", PATHS)
+def test_capped_groups_split_hot_experts(T, path):
+    """Batches of 33-64 tokens whose experts average at most 16 tokens cap
+    their groups at 32 tokens (32-column gate/up tiles); an expert holding
+    more tokens is split into two groups, each read and summed on its own."""
+    dw = DeviceWeights(make_weights(SKEWED, 31))
+    x = make_tokens(SKEWED.d_model, T, 31, "bf16")
+    tau, _ = _calibrated(dw, x, 0.7)
+    layer = make_layer(SKEWED, 64, path=path)
+    gpu, ref, info = _check(layer, dw, x, tau, 0.0, "bf16", dense=(path == "dense"))
+    counts = np.bincount(ref.router.topk_idx.ravel(), minlength=SKEWED.n_experts)
+    assert counts.max() > 32  # at least one expert is split
+
+
 def test_many_small_experts():
     wl, dw = workload_weights("many_small_experts")
     tau, _ = tau_of("many_small_experts", 0.8)
