@@ -563,9 +563,23 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   // AUTO only: tensor-core groups whose union is at most this fraction of
   // d_ff read only the union rows (the forced paths fix the rows they read)
   if (mode != MOE_PATH_AUTO) dm.gather_density = 0.f;
+  // AUTO (|h| score) batches whose groups all fit one row-stream pass: every
+  // group streams its union rows, the 5-8-token candidates included. The
+  // candidate rule prices the tensor cores at their many-group rate; a batch
+  // this small has at most T x k / 5 such groups, and a tensor-core launch
+  // with one to three groups streams at 0.55-0.69 of HBM, below the row
+  // stream's ~0.77. No tensor-core launch then. The combine stays a kernel
+  // of its own for these batches: the row stream's direct combine (adds into
+  // the token rows, the last CTA writing out) measured no faster with groups
+  // of 5-8 tokens (T = 8 on the Mixtral-shaped layer: 95.0 us for the row
+  // stream and the output, against 86.4 + 7.4 us for the row stream and the
+  // combine launch).
+  const bool rs_only = mode == MOE_PATH_AUTO && c->bf16 && cap.gemv_cand > cap.gemv_max &&
+                       tmax > cap.gemv_max && tmax <= cap.gemv_cand;
+  if (rs_only) dm.gemv_max = cap.gemv_cand;
   bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
-                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) && tmax <= cap.gemv_max);
+                       !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) && tmax <= dm.gemv_max);
   const int n_max = roundup(tmax, 16);
   // gate score: the GEMV groups' up projection is sparse (only the active
   // rows) when the threshold can leave rows out; at tau <= 0 every neuron
@@ -601,8 +615,8 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
     // the row-stream kernel is only needed for groups the fusion leaves:
     // unfused row-stream groups and candidates
     const int fused_max = dm.sparse_up ? 1 : moe::kFuseTokens;
-    const bool big_gemv = std::min(tmax, cap.gemv_max) > fused_max;
-    const bool cand = cap.gemv_cand > cap.gemv_max && tmax > cap.gemv_max;
+    const bool big_gemv = std::min(tmax, dm.gemv_max) > fused_max;
+    const bool cand = dm.gemv_cand > dm.gemv_max && tmax > dm.gemv_max;
     need_gemv = big_gemv || cand;
   }
   // every group on a row stream (fused or not; with the gate score only when
@@ -610,7 +624,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   // and a small batch: the row stream combines directly into the output (no
   // combine launch); with no row-stream launch the gate/up kernel writes out
   const bool out_bf16 = c->bf16 && !c->desc.out_f32;
-  dm.direct_combine = (need_gemv || dm.fuse_down) && !need_tc &&
+  dm.direct_combine = (need_gemv || dm.fuse_down) && !need_tc && !rs_only &&
                               (!dm.sparse_up || !need_gemv) && T <= moe::kDirectMax
                           ? 1
                           : 0;
