@@ -128,7 +128,9 @@ typedef struct {
                                  0: automatic -- groups of <= 4 tokens on the GEMV path, and
                                  (|h| score, bf16) groups of 5..8 tokens choose after gate/up:
                                  the GEMV path if their active-row union is <= 0.8 x d_ff,
-                                 else all rows on the tensor cores */
+                                 else all rows on the tensor cores; in batches whose groups
+                                 all hold <= 8 tokens (T <= 8), every group uses the GEMV
+                                 path (either score) */
   float gather_max_density;   /* AUTO (bf16): a tensor-core group of <= 64 tokens whose
                                  active-row union is <= this fraction of d_ff reads only
                                  the union rows (gathered copies, packed in shared memory)

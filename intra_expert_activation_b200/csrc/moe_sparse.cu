@@ -563,7 +563,7 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   // AUTO only: tensor-core groups whose union is at most this fraction of
   // d_ff read only the union rows (the forced paths fix the rows they read)
   if (mode != MOE_PATH_AUTO) dm.gather_density = 0.f;
-  // AUTO (|h| score) batches whose groups all fit one row-stream pass: every
+  // AUTO batches whose groups all fit one row-stream pass: every
   // group streams its union rows, the 5-8-token candidates included. The
   // candidate rule prices the tensor cores at their many-group rate; a batch
   // this small has at most T x k / 5 such groups, and a tensor-core launch
@@ -574,9 +574,11 @@ moe_status moe_sparse_forward(moe_sparse_ctx* c, const void* x, int32_t T, const
   // of 5-8 tokens (T = 8 on the Mixtral-shaped layer: 95.0 us for the row
   // stream and the output, against 86.4 + 7.4 us for the row stream and the
   // combine launch).
-  const bool rs_only = mode == MOE_PATH_AUTO && c->bf16 && cap.gemv_cand > cap.gemv_max &&
-                       tmax > cap.gemv_max && tmax <= cap.gemv_cand;
-  if (rs_only) dm.gemv_max = cap.gemv_cand;
+  // The gate score, whose groups of more than 4 tokens otherwise take the
+  // tensor cores by size, follows the same rule.
+  const bool rs_only = mode == MOE_PATH_AUTO && c->bf16 && c->desc.gemv_max_tokens == 0 &&
+                       tmax > cap.gemv_max && tmax <= moe::kGemvCandMax;
+  if (rs_only) dm.gemv_max = moe::kGemvCandMax;
   bool need_gemv = !(mode == MOE_PATH_SPARSE_TC || mode == MOE_PATH_SPARSE_TC_ALLROWS) || !c->bf16;
   const bool need_tc = c->bf16 && mode != MOE_PATH_SPARSE_GEMV &&
                        !((mode == MOE_PATH_AUTO || mode == MOE_PATH_DENSE) && tmax <= dm.gemv_max);
